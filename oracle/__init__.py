@@ -1,0 +1,167 @@
+"""CPU oracle for the TriAttention prune step -- TEST INFRASTRUCTURE ONLY.
+
+Thin ctypes marshalling around ``oracle.c`` (plain float64 C, term by term).
+Only the tests, the smoke check and the benchmark's CPU-baseline leg may
+import this package; the product path never does.
+
+All arrays are numpy, host memory.  Keys and values are bf16 bit patterns
+(``uint16``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+NO_TRIG = 1
+NO_CONC_WEIGHT = 2
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        _lib = ctypes.CDLL(path)
+        P = ctypes.POINTER
+        _lib.orc_calibrate.argtypes = [P(ctypes.c_double), ctypes.c_int64, ctypes.c_int64,
+                                       ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+                                       P(ctypes.c_double), P(ctypes.c_double), P(ctypes.c_double)]
+        _lib.orc_key_score.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.c_int32, ctypes.c_int64]
+        _lib.orc_key_score.restype = ctypes.c_double
+        _lib.orc_raw_scores.argtypes = [ctypes.c_void_p, P(ctypes.c_double)]
+        _lib.orc_zmax.argtypes = [ctypes.c_void_p, P(ctypes.c_double), P(ctypes.c_double),
+                                  P(ctypes.c_double)]
+        _lib.orc_select.argtypes = [ctypes.c_void_p, P(ctypes.c_double), P(ctypes.c_int32)]
+        _lib.orc_compact.argtypes = [ctypes.c_void_p, P(ctypes.c_int32), P(ctypes.c_uint16),
+                                     P(ctypes.c_uint16), P(ctypes.c_int32), P(ctypes.c_int32)]
+        _lib.orc_num_threads.restype = ctypes.c_int32
+    return _lib
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [
+        ("L", ctypes.c_int32), ("B", ctypes.c_int32), ("Hq", ctypes.c_int32),
+        ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32), ("layout", ctypes.c_int32),
+        ("theta", ctypes.c_double), ("budget", ctypes.c_int32), ("n_offsets", ctypes.c_int32),
+        ("offsets", ctypes.c_void_p), ("flags", ctypes.c_uint32), ("cap", ctypes.c_int64),
+        ("seq_start", ctypes.c_void_p), ("seq_len", ctypes.c_void_p),
+        ("cur_pos", ctypes.c_void_p), ("k", ctypes.c_void_p), ("pos", ctypes.c_void_p),
+        ("centre", ctypes.c_void_p), ("mean_norm", ctypes.c_void_p), ("mrl", ctypes.c_void_p),
+    ]
+
+
+def _ptr(a: np.ndarray, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+class Problem:
+    """One prune problem: cache (post-RoPE bf16 keys as uint16, positions,
+    segments), calibration statistics and hyper-parameters."""
+
+    def __init__(self, *, k: np.ndarray, pos: np.ndarray, seq_start: Sequence[int],
+                 seq_len: Sequence[int], cur_pos: Sequence[int], centre: np.ndarray,
+                 mean_norm: np.ndarray, mrl: np.ndarray, theta: float, budget: int,
+                 offsets: Sequence[int], n_q_heads: int, layout: int = 0, flags: int = 0):
+        L, Hkv, cap, D = k.shape
+        self.k = np.ascontiguousarray(k, dtype=np.uint16)
+        self.pos = np.ascontiguousarray(pos, dtype=np.int32)
+        self.seq_start = np.ascontiguousarray(seq_start, dtype=np.int64)
+        self.seq_len = np.ascontiguousarray(seq_len, dtype=np.int32)
+        self.cur_pos = np.ascontiguousarray(cur_pos, dtype=np.int32)
+        self.centre = np.ascontiguousarray(centre, dtype=np.float64)
+        self.mean_norm = np.ascontiguousarray(mean_norm, dtype=np.float64)
+        self.mrl = np.ascontiguousarray(mrl, dtype=np.float64)
+        self.offsets = np.ascontiguousarray(offsets, dtype=np.int32)
+        self.L, self.Hkv, self.cap, self.D = L, Hkv, cap, D
+        self.Hq, self.B, self.budget = n_q_heads, len(self.seq_len), budget
+        F = D // 2
+        assert self.centre.shape == (L, n_q_heads, F, 2)
+        assert self.mean_norm.shape == (L, n_q_heads, F) and self.mrl.shape == (L, n_q_heads, F)
+        assert self.pos.shape == (L, Hkv, cap) and len(self.seq_start) == self.B + 1
+        self._s = _Problem(L, self.B, n_q_heads, Hkv, D, layout, float(theta), budget,
+                           len(self.offsets), self.offsets.ctypes.data, flags, cap,
+                           self.seq_start.ctypes.data, self.seq_len.ctypes.data,
+                           self.cur_pos.ctypes.data, self.k.ctypes.data, self.pos.ctypes.data,
+                           self.centre.ctypes.data, self.mean_norm.ctypes.data,
+                           self.mrl.ctypes.data)
+
+    @property
+    def ref(self):
+        return ctypes.byref(self._s)
+
+
+def calibrate(q: np.ndarray, layout: int = 0):
+    """q: [L][N][Hq][D] pre-RoPE queries -> (centre [L,Hq,F,2], mean_norm, mrl [L,Hq,F])."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    L, N, Hq, D = q.shape
+    F = D // 2
+    centre = np.zeros((L, Hq, F, 2))
+    mean_norm = np.zeros((L, Hq, F))
+    mrl = np.zeros((L, Hq, F))
+    lib().orc_calibrate(_ptr(q, ctypes.c_double), L, N, Hq, D, layout,
+                        _ptr(centre, ctypes.c_double), _ptr(mean_norm, ctypes.c_double),
+                        _ptr(mrl, ctypes.c_double))
+    return centre, mean_norm, mrl
+
+
+def key_score(p: Problem, l: int, h: int, b: int, t: int) -> float:
+    """Raw score of slot t of sequence b for query head h of layer l."""
+    return lib().orc_key_score(p.ref, l, h, b, t)
+
+
+def raw_scores(p: Problem) -> np.ndarray:
+    """[L][Hq][cap] raw scores; NaN outside the live part of each segment."""
+    raw = np.full((p.L, p.Hq, p.cap), np.nan)
+    lib().orc_raw_scores(p.ref, _ptr(raw, ctypes.c_double))
+    return raw
+
+
+def zmax(p: Problem, raw: np.ndarray):
+    """-> (z [L][Hq][cap], score [L][Hkv][cap]); NaN outside live slots."""
+    raw = np.ascontiguousarray(raw, dtype=np.float64)
+    z = np.full((p.L, p.Hq, p.cap), np.nan)
+    score = np.full((p.L, p.Hkv, p.cap), np.nan)
+    lib().orc_zmax(p.ref, _ptr(raw, ctypes.c_double), _ptr(z, ctypes.c_double),
+                   _ptr(score, ctypes.c_double))
+    return z, score
+
+
+def select(p: Problem, score: np.ndarray) -> np.ndarray:
+    """-> sel [L][Hkv][B][budget] ascending slots within each segment, -1 padded."""
+    score = np.ascontiguousarray(score, dtype=np.float64)
+    sel = np.empty((p.L, p.Hkv, p.B, p.budget), dtype=np.int32)
+    lib().orc_select(p.ref, _ptr(score, ctypes.c_double), _ptr(sel, ctypes.c_int32))
+    return sel
+
+
+def compact(p: Problem, sel: np.ndarray, v: np.ndarray):
+    """Compacted copies -> (k, v, pos, seq_len); the problem's arrays are not modified."""
+    sel = np.ascontiguousarray(sel, dtype=np.int32)
+    k2 = p.k.copy()
+    v2 = np.ascontiguousarray(v, dtype=np.uint16).copy()
+    pos2 = p.pos.copy()
+    sl = np.empty(p.B, dtype=np.int32)
+    lib().orc_compact(p.ref, _ptr(sel, ctypes.c_int32), _ptr(k2, ctypes.c_uint16),
+                      _ptr(v2, ctypes.c_uint16), _ptr(pos2, ctypes.c_int32), _ptr(sl, ctypes.c_int32))
+    return k2, v2, pos2, sl
+
+
+def prune(p: Problem, v: np.ndarray):
+    """Whole prune step -> dict with raw, z, score, sel and the compacted cache."""
+    raw = raw_scores(p)
+    z, score = zmax(p, raw)
+    sel = select(p, score)
+    k2, v2, pos2, sl = compact(p, sel, v)
+    return {"raw": raw, "z": z, "score": score, "sel": sel, "k": k2, "v": v2, "pos": pos2,
+            "seq_len": sl}
+
+
+def num_threads() -> int:
+    return int(lib().orc_num_threads())

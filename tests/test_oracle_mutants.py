@@ -1,0 +1,77 @@
+"""The pins have teeth: plant plausible mistakes in copies of the oracle source
+(compiled on the CPU into a temporary library) and check that each one makes
+at least one pin fail.  The real oracle is untouched."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+MUTANTS = {
+    "rotate forward instead of back": ("const double kx = xt * ca + yt * sa;\n    const double ky = -xt * sa + yt * ca;",
+                                       "const double kx = xt * ca - yt * sa;\n    const double ky = xt * sa + yt * ca;"),
+    "distance sign": ("cur + (double)p->offsets[j] - kpos", "kpos - cur - (double)p->offsets[j]"),
+    "sum instead of mean over offsets": ("s_trig += acc / (double)p->n_offsets;", "s_trig += acc;"),
+    "phase difference sign": ("cos(w * dist + c_arg - k_arg)", "cos(w * dist - c_arg + k_arg)"),
+    "norm weight R instead of 1-R": ("(1.0 - p->mrl[o])", "(p->mrl[o])"),
+    "frequency exponent": ("pow(theta, -2.0 * (double)f / (double)D)", "pow(theta, -(double)f / (double)D)"),
+    "half-split pairing": ("*yi = f + D / 2;", "*yi = f + 1;"),
+    "sample std": ("var /= (double)(T > 0 ? T : 1);", "var /= (double)(T > 1 ? T - 1 : 1);"),
+    "group sum instead of max": ("if (zt > sc[t]) sc[t] = zt;", "sc[t] = (j == 0 ? 0.0 : sc[t]) + zt;"),
+    "ties to the higher slot": ("return (x->slot > y->slot) - (x->slot < y->slot);",
+                                "return (x->slot < y->slot) - (x->slot > y->slot);"),
+    "keep the lowest scores": ("if (x->score > y->score) return -1;\n  if (x->score < y->score) return 1;",
+                               "if (x->score < y->score) return -1;\n  if (x->score > y->score) return 1;"),
+    "gather off by one": ("const int64_t src = base + s[j];", "const int64_t src = base + s[j] + (j > 0);"),
+    "MRL from the sum of norms": ("hypot(centre[2 * o], centre[2 * o + 1]) / mean_norm[o]",
+                                  "hypot(centre[2 * o], centre[2 * o + 1]) / (mean_norm[o] * (double)N)"),
+    "conjugated centre": ("const double cx = p->centre[2 * o], cy = p->centre[2 * o + 1];",
+                          "const double cx = p->centre[2 * o], cy = -p->centre[2 * o + 1];"),
+}
+
+PIN_TESTS = [
+    (pins.test_worked_example_closed_form, {}),
+    (pins.test_calibration_identical_queries_concentrate_fully, {}),
+    (pins.test_calibration_antipodal_and_two_directions, {}),
+    (pins.test_offset_mean_matches_dirichlet_closed_form, {"layout": 0}),
+    (pins.test_zero_spread_equals_mean_post_rope_logit, {"layout": 0}),
+    (pins.test_diffuse_queries_reduce_to_weighted_key_norm, {}),
+    (pins.test_key_position_cancels, {}),
+    (pins.test_zscore_invariants_and_max, {}),
+    (pins.test_select_equals_brute_force_with_ties, {"T": 64, "budget": 7}),
+    (pins.test_compaction_moves_selected_rows_in_order, {}),
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name!r} not found exactly once"
+    path = tmp_path / "mutant.c"
+    path.write_text(src.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-fopenmp", str(path), "-o",
+                    str(lib), "-lm"], check=True)
+    real = oracle.lib()
+    mutant = ctypes.CDLL(str(lib))
+    for fn in ("orc_calibrate", "orc_key_score", "orc_raw_scores", "orc_zmax", "orc_select",
+               "orc_compact"):
+        getattr(mutant, fn).argtypes = getattr(real, fn).argtypes
+        getattr(mutant, fn).restype = getattr(real, fn).restype
+    caught = []
+    oracle._lib = mutant
+    try:
+        for test, kw in PIN_TESTS:
+            try:
+                test(**kw)
+            except AssertionError:
+                caught.append(test.__name__)
+    finally:
+        oracle._lib = real
+    assert caught, f"no pin caught the planted mistake {name!r}"

@@ -1,0 +1,196 @@
+/*
+ * tria.h -- C ABI of the B200 (sm_100a) TriAttention KV-cache prune step.
+ *
+ * What the library computes (TriAttention, arXiv 2604.04921, as described by
+ * the romaanj.github.io review, section "Method", and the dimensionstp.github.io
+ * review, sections 2-2 and 3-2):
+ *
+ *   calibration   per (layer, query head, RoPE pair f): centre E[q_f] (complex),
+ *                 mean norm E|q_f| and concentration R_f = |E[q_f]| / E|q_f|
+ *                 over sample pre-RoPE queries;
+ *   key score     s_h(t) = mean_{delta in offsets} sum_f |E[q_f]| |k_f|
+ *                            cos(w_f (cur + delta - pos_t) + arg E[q_f] - arg k_f)
+ *                        + sum_f (1 - R_f) E|q_f| |k_f|
+ *                 with k_f the pre-RoPE pair of the cached key, w_f = theta^(-2f/D);
+ *   aggregation   z-score of s_h over the sequence's keys (population sigma,
+ *                 z = 0 if sigma = 0), then the max over the query heads h that
+ *                 share the key's KV head (h / G == kv head);
+ *   selection     top-`budget` keys per (layer, KV head, sequence) by
+ *                 (score desc, slot asc);
+ *   compaction    survivors move in place to slots [0, kept) in ascending slot
+ *                 order; seq_len becomes kept.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Pointers marked DEVICE must point to memory of the current CUDA device;
+ *   HOST pointers are read during the call only.  The caller owns every
+ *   buffer, the workspace included; the library allocates nothing and keeps
+ *   no global mutable state.
+ * - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *   stream.  Every call is asynchronous on it: argument errors are returned
+ *   synchronously before anything is launched; launch failures return
+ *   TRIA_ERR_CUDA.  Inconsistencies only the device can see (a sequence
+ *   length beyond its segment, a malformed selection list, a wait that ran
+ *   out) set bits in the workspace's device error word, readable with
+ *   tria_get_device_error() after the stream has been synchronised.
+ *   Nothing traps.
+ * - Cache layout: K and V are bf16 [L][Hkv][cap_total][D] (post-RoPE keys),
+ *   pos is int32 [L][Hkv][cap_total].  Sequence b owns slots
+ *   [seq_start[b], seq_start[b+1]) of every (layer, KV head) row; its live
+ *   keys are the first seq_len[b] of them, with ascending positions.
+ * - Slot indices in selection lists are relative to the segment start.
+ * - Query head h uses KV head h / G, G = n_q_heads / n_kv_heads.
+ * - Supported shapes: head_dim in {64, 128, 256}; G in {1, 2, 4, 8, 16};
+ *   batch <= TRIA_MAX_BATCH; 1 <= n_offsets <= TRIA_MAX_OFFSETS; every
+ *   segment capacity <= TRIA_MAX_SEGMENT; 1 <= budget <= TRIA_MAX_SEGMENT.
+ */
+#ifndef TRIA_H
+#define TRIA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TRIA_OK = 0,
+  TRIA_ERR_INVALID_ARG = 1,   /* a null, negative, inconsistent or misaligned argument */
+  TRIA_ERR_UNSUPPORTED = 2,   /* a valid shape this build has no kernel for */
+  TRIA_ERR_WORKSPACE = 3,     /* workspace null, misaligned or smaller than tria_workspace_size */
+  TRIA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  TRIA_ERR_DEVICE_FLAG = 5    /* returned by tria_get_device_error when a device bit is set */
+} tria_status;
+
+#define TRIA_ROPE_HALF_SPLIT 0   /* pair f = (v[f], v[f + D/2]) */
+#define TRIA_ROPE_INTERLEAVED 1  /* pair f = (v[2f], v[2f + 1]) */
+
+#define TRIA_NO_TRIG 1u          /* ablation: score without the trigonometric term */
+#define TRIA_NO_CONC_WEIGHT 2u   /* ablation: norm term weighted by E|q_f| instead of (1-R_f)E|q_f| */
+
+#define TRIA_DTYPE_F32 0
+#define TRIA_DTYPE_BF16 1
+
+#define TRIA_MAX_BATCH 256
+#define TRIA_MAX_OFFSETS 4096
+#define TRIA_MAX_SEGMENT (1 << 18)
+
+/* device error word bits */
+#define TRIA_DEVERR_SEQ_LEN 1      /* seq_len[b] < 0 or > segment capacity: that sequence skipped */
+#define TRIA_DEVERR_SELECTION 2    /* tria_compact: selection not ascending / out of range: unit skipped */
+#define TRIA_DEVERR_TIMEOUT 4      /* a bounded wait on an mbarrier ran out: results invalid */
+#define TRIA_DEVERR_SEGMENT_BIG 8  /* a live sequence exceeded the kernel's per-unit capacity */
+
+/* Host-side description of the prune problem, copied by value. */
+typedef struct {
+  int32_t num_layers;   /* L >= 1 */
+  int32_t batch;        /* B, 1..TRIA_MAX_BATCH */
+  int32_t n_q_heads;    /* Hq, a multiple of n_kv_heads */
+  int32_t n_kv_heads;   /* Hkv >= 1 */
+  int32_t head_dim;     /* D */
+  double rope_theta;    /* RoPE base, > 1 */
+  int32_t rope_layout;  /* TRIA_ROPE_HALF_SPLIT or TRIA_ROPE_INTERLEAVED */
+  int32_t budget;       /* keys kept per (layer, KV head, sequence) */
+  const int32_t *offsets; /* HOST [n_offsets] future query offsets, each >= 1 */
+  int32_t n_offsets;
+  uint32_t flags;       /* 0, or TRIA_NO_TRIG / TRIA_NO_CONC_WEIGHT */
+} tria_config;
+
+/* The cache.  Device pointers except seq_start. */
+typedef struct {
+  void *k;                 /* DEVICE bf16 [L][Hkv][cap_total][D], 16-byte aligned */
+  void *v;                 /* DEVICE bf16 [L][Hkv][cap_total][D], 16-byte aligned */
+  int32_t *pos;            /* DEVICE int32 [L][Hkv][cap_total], 16-byte aligned */
+  int32_t *seq_len;        /* DEVICE int32 [B], live keys per sequence (in/out) */
+  const int32_t *cur_pos;  /* DEVICE int32 [B], position of each sequence's newest token */
+  const int64_t *seq_start;/* HOST int64 [B+1], nondecreasing, seq_start[B] <= cap_total */
+  int64_t cap_total;       /* slots per (layer, KV head) row */
+} tria_cache;
+
+/* Calibration statistics, DEVICE float32, 16-byte aligned. */
+typedef struct {
+  const float *centre;     /* [L][Hq][D/2][2]  E[q_f] as (re, im) */
+  const float *mean_norm;  /* [L][Hq][D/2]     E|q_f| */
+  const float *mrl;        /* [L][Hq][D/2]     R_f */
+} tria_stats;
+
+/* Bytes of workspace the calls below need for this problem (the largest over
+ * all calls).  Only the shapes and cache->seq_start/cap_total are read. */
+tria_status tria_workspace_size(const tria_config *cfg, const tria_cache *cache, size_t *bytes);
+
+/* Clears the workspace's device error word (async on stream).  Call once after
+ * allocating a workspace; the word is otherwise sticky across calls. */
+tria_status tria_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/* Offline calibration (romaanj.github.io review, "Method"; dimensionstp.github.io
+ * review, section 3-1): q_pre is DEVICE [L][n_samples][Hq][D] pre-RoPE queries,
+ * float32 (q_dtype = TRIA_DTYPE_F32) or bf16 (TRIA_DTYPE_BF16).  Writes the
+ * three DEVICE float32 outputs laid out as in tria_stats.  Accumulates in
+ * float64.  Only L, Hq, head_dim and rope_layout of cfg are read. */
+tria_status tria_calibrate(const tria_config *cfg, const void *q_pre, int32_t q_dtype,
+                           int64_t n_samples, float *centre, float *mean_norm, float *mrl,
+                           void *stream);
+
+/* Key scores (romaanj.github.io review, "Method"; dimensionstp.github.io review,
+ * sections 2-2 and 3-2 (2)-(4), (6)).  Writes DEVICE float32 score
+ * [L][Hkv][cap_total], the group max of the z-scores, for every live slot of
+ * every sequence; if raw is not NULL, also DEVICE float32 raw
+ * [L][Hq][cap_total], the per-query-head score s_h.  Other slots are not
+ * written.  Sequences of any length are scored. */
+tria_status tria_score(const tria_config *cfg, const tria_stats *stats, const tria_cache *cache,
+                       float *score, float *raw, void *ws, size_t ws_bytes, void *stream);
+
+/* Top-budget selection (romaanj.github.io review, "Method"; dimensionstp.github.io
+ * review, section 3-2 (5)).  score is DEVICE float32 [L][Hkv][cap_total] (as
+ * written by tria_score).  Writes DEVICE int32 sel [L][Hkv][B][budget]: the kept
+ * slots in ascending order, -1 after the last one.  A sequence with
+ * seq_len <= budget keeps all its slots.  Ties go to the lower slot. */
+tria_status tria_select(const tria_config *cfg, const tria_cache *cache, const float *score,
+                        int32_t *sel, void *ws, size_t ws_bytes, void *stream);
+
+/* In-place compaction (eviction).  sel is DEVICE int32 [L][Hkv][B][budget] as
+ * written by tria_select: strictly ascending slots then -1.  Moves K, V and pos
+ * rows sel[j] -> j of each segment and sets seq_len[b] to the number of kept
+ * slots (every (layer, KV head) list of a sequence must keep the same count).
+ * A list that is not strictly ascending or leaves the segment sets
+ * TRIA_DEVERR_SELECTION and that unit is left untouched. */
+tria_status tria_compact(const tria_config *cfg, const tria_cache *cache, const int32_t *sel,
+                         void *ws, size_t ws_bytes, void *stream);
+
+/* The whole prune step in one call: score, z-score + group max, select and
+ * compact every (layer, KV head, sequence) with seq_len > budget; shorter
+ * sequences are left untouched.  seq_len is read once at the start and
+ * rewritten at the end.  If sel_out is not NULL it receives the selection
+ * as tria_select would write it (for units that were pruned). */
+tria_status tria_prune(const tria_config *cfg, const tria_stats *stats, const tria_cache *cache,
+                       int32_t *sel_out, void *ws, size_t ws_bytes, void *stream);
+
+/* tria_prune with a cudaEvent_t (as void*) recorded on `stream` before each
+ * of its kernels and after the last: events[0..n_stages].  Returns the number
+ * of stages in *n_stages (events must hold TRIA_PRUNE_MAX_STAGES + 1).  For
+ * per-kernel timing only. */
+#define TRIA_PRUNE_MAX_STAGES 8
+tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
+                                const tria_cache *cache, int32_t *sel_out, void *ws,
+                                size_t ws_bytes, void *stream, void *const *events,
+                                int32_t *n_stages);
+
+/* Names of the kernels tria_prune launches, in order, for stage i. */
+const char *tria_prune_stage_name(int32_t i);
+
+/* Reads the workspace's device error word into *code (synchronous: waits for
+ * `stream`).  Returns TRIA_ERR_DEVICE_FLAG if any bit is set, TRIA_OK otherwise. */
+tria_status tria_get_device_error(const void *ws, int32_t *code, void *stream);
+
+/* Human-readable name of a status. */
+const char *tria_status_string(tria_status s);
+
+/* Library version string. */
+const char *tria_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRIA_H */

@@ -1,0 +1,377 @@
+// Host side of the C ABI declared in include/tria.h: argument validation,
+// workspace layout and kernel launches.  No allocation, no host
+// synchronisation (except tria_get_device_error), no global mutable state
+// beyond per-device launch-configuration caches.
+#include <cmath>
+#include <cstring>
+
+#include "tria_internal.cuh"
+
+namespace tria {
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+WsLayout ws_layout(const tria_config &cfg, int64_t cap) {
+  WsLayout w{};
+  const size_t F = (size_t)cfg.head_dim / 2;
+  size_t o = 0;
+  w.err = o;      o += 256;
+  w.seqlen = o;   o = align_up(o + 4ull * cfg.batch, 256);
+  w.ea = o;       o = align_up(o + 16ull * cfg.batch * F, 256);
+  w.raw = o;      o = align_up(o + 4ull * cfg.num_layers * cfg.n_q_heads * (size_t)cap, 256);
+  w.score = o;
+  w.sel = o;      o = align_up(o + 4ull * cfg.num_layers * cfg.n_kv_heads * cfg.batch * cfg.budget, 256);
+  w.total = o;
+  return w;
+}
+
+int device_sm_count() {
+  static int cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+}  // namespace tria
+
+using namespace tria;
+
+namespace {
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+tria_status check_config(const tria_config *cfg, bool scoring) {
+  if (!cfg) return TRIA_ERR_INVALID_ARG;
+  if (cfg->num_layers < 1 || cfg->batch < 1 || cfg->n_kv_heads < 1 || cfg->n_q_heads < 1)
+    return TRIA_ERR_INVALID_ARG;
+  if (cfg->batch > TRIA_MAX_BATCH) return TRIA_ERR_UNSUPPORTED;
+  if (cfg->n_q_heads % cfg->n_kv_heads != 0) return TRIA_ERR_INVALID_ARG;
+  if (cfg->head_dim < 2 || cfg->head_dim % 2 != 0) return TRIA_ERR_INVALID_ARG;
+  if (cfg->rope_layout != TRIA_ROPE_HALF_SPLIT && cfg->rope_layout != TRIA_ROPE_INTERLEAVED)
+    return TRIA_ERR_INVALID_ARG;
+  if (cfg->budget < 1) return TRIA_ERR_INVALID_ARG;
+  if (cfg->budget > TRIA_MAX_SEGMENT) return TRIA_ERR_UNSUPPORTED;
+  if (cfg->n_q_heads / cfg->n_kv_heads > 16) return TRIA_ERR_UNSUPPORTED;
+  if (scoring) {
+    if (!(cfg->rope_theta > 1.0) || !std::isfinite(cfg->rope_theta)) return TRIA_ERR_INVALID_ARG;
+    if (!cfg->offsets || cfg->n_offsets < 1) return TRIA_ERR_INVALID_ARG;
+    if (cfg->n_offsets > TRIA_MAX_OFFSETS) return TRIA_ERR_UNSUPPORTED;
+    for (int i = 0; i < cfg->n_offsets; ++i)
+      if (cfg->offsets[i] < 1) return TRIA_ERR_INVALID_ARG;
+    if (cfg->flags & ~(TRIA_NO_TRIG | TRIA_NO_CONC_WEIGHT)) return TRIA_ERR_INVALID_ARG;
+    if (!score_supported(cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads, cfg->rope_layout))
+      return TRIA_ERR_UNSUPPORTED;
+  } else {
+    if (cfg->head_dim % 8 != 0) return TRIA_ERR_UNSUPPORTED;
+  }
+  return TRIA_OK;
+}
+
+tria_status check_cache(const tria_config *cfg, const tria_cache *c, bool need_kv) {
+  if (!c) return TRIA_ERR_INVALID_ARG;
+  if (!c->seq_start || !c->seq_len || c->cap_total < 0) return TRIA_ERR_INVALID_ARG;
+  if (need_kv) {
+    if (!c->k || !c->v || !c->pos) return TRIA_ERR_INVALID_ARG;
+    if (!aligned(c->k, 16) || !aligned(c->v, 16) || !aligned(c->pos, 16))
+      return TRIA_ERR_INVALID_ARG;
+  }
+  if (c->seq_start[0] < 0) return TRIA_ERR_INVALID_ARG;
+  for (int b = 0; b < cfg->batch; ++b) {
+    const int64_t a = c->seq_start[b], e = c->seq_start[b + 1];
+    if (e < a) return TRIA_ERR_INVALID_ARG;
+    if (e - a > TRIA_MAX_SEGMENT) return TRIA_ERR_UNSUPPORTED;
+  }
+  if (c->seq_start[cfg->batch] > c->cap_total) return TRIA_ERR_INVALID_ARG;
+  return TRIA_OK;
+}
+
+tria_status check_stats(const tria_stats *s) {
+  if (!s || !s->centre || !s->mean_norm || !s->mrl) return TRIA_ERR_INVALID_ARG;
+  if (!aligned(s->centre, 8) || !aligned(s->mean_norm, 4) || !aligned(s->mrl, 4))
+    return TRIA_ERR_INVALID_ARG;
+  return TRIA_OK;
+}
+
+tria_status check_ws(const tria_config *cfg, const tria_cache *c, void *ws, size_t bytes) {
+  if (!ws || !aligned(ws, 256)) return TRIA_ERR_WORKSPACE;
+  if (bytes < ws_layout(*cfg, c->cap_total).total) return TRIA_ERR_WORKSPACE;
+  return TRIA_OK;
+}
+
+tria_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TRIA_OK : TRIA_ERR_CUDA; }
+
+void fill_fold(FoldParams &fp, const tria_config *cfg, const tria_cache *c, int32_t *seqlen_snap,
+               double2 *ea, int32_t *err) {
+  std::memset(&fp, 0, sizeof fp);
+  fp.cur_pos = c->cur_pos;
+  fp.seq_len = c->seq_len;
+  fp.seqlen_snap = seqlen_snap;
+  fp.ea = ea;
+  fp.err = err;
+  fp.theta = cfg->rope_theta;
+  fp.D = cfg->head_dim;
+  fp.B = cfg->batch;
+  fp.n_offsets = cfg->n_offsets;
+  fp.flags = cfg->flags;
+  for (int b = 0; b < cfg->batch; ++b) fp.seg_cap[b] = c->seq_start[b + 1] - c->seq_start[b];
+  std::memcpy(fp.offsets, cfg->offsets, sizeof(int32_t) * cfg->n_offsets);
+}
+
+// Builds the score kernel parameters; returns the grid size (0: nothing to launch).
+int fill_score(ScoreParams &sp, const tria_config *cfg, const tria_stats *st, const tria_cache *c,
+               const double2 *ea, const int32_t *seqlen, float *raw, int32_t *err, int skip_short) {
+  std::memset(&sp, 0, sizeof sp);
+  const int tile = score_tile_keys(cfg->head_dim);
+  sp.k = static_cast<const uint8_t *>(c->k);
+  sp.centre = reinterpret_cast<const float2 *>(st->centre);
+  sp.mean_norm = st->mean_norm;
+  sp.mrl = st->mrl;
+  sp.ea = ea;
+  sp.seqlen = seqlen;
+  sp.raw = raw;
+  sp.err = err;
+  sp.cap = c->cap_total;
+  sp.L = cfg->num_layers;
+  sp.Hkv = cfg->n_kv_heads;
+  sp.Hq = cfg->n_q_heads;
+  sp.B = cfg->batch;
+  sp.budget = cfg->budget;
+  sp.skip_short = skip_short;
+  sp.no_conc_weight = (cfg->flags & TRIA_NO_CONC_WEIGHT) ? 1 : 0;
+  int32_t acc = 0;
+  for (int b = 0; b <= cfg->batch; ++b) {
+    sp.seg_start[b] = c->seq_start[b];
+    sp.tile_prefix[b] = acc;
+    if (b < cfg->batch) acc += (int32_t)((c->seq_start[b + 1] - c->seq_start[b] + tile - 1) / tile);
+  }
+  sp.tiles_per_row = acc;
+  sp.total_tiles = (int64_t)cfg->num_layers * cfg->n_kv_heads * acc;
+  if (sp.total_tiles == 0) return 0;
+  int64_t grid = device_sm_count();
+  if (grid > sp.total_tiles) grid = sp.total_tiles;
+  sp.tiles_per_cta = (int32_t)((sp.total_tiles + grid - 1) / grid);
+  grid = (sp.total_tiles + sp.tiles_per_cta - 1) / sp.tiles_per_cta;
+  return (int)grid;
+}
+
+void fill_unit(UnitParams &up, const tria_config *cfg, const tria_cache *c, int mode) {
+  std::memset(&up, 0, sizeof up);
+  up.k = static_cast<uint8_t *>(c->k);
+  up.v = static_cast<uint8_t *>(c->v);
+  up.pos = c->pos;
+  up.cap = c->cap_total;
+  up.L = cfg->num_layers;
+  up.Hkv = cfg->n_kv_heads;
+  up.Hq = cfg->n_q_heads;
+  up.B = cfg->batch;
+  up.G = cfg->n_q_heads / cfg->n_kv_heads;
+  up.D = cfg->head_dim;
+  up.budget = cfg->budget;
+  up.mode = mode;
+  for (int b = 0; b <= cfg->batch; ++b) up.seg_start[b] = c->seq_start[b];
+}
+
+struct Ws {
+  WsLayout lay;
+  uint8_t *base;
+  int32_t *err() const { return reinterpret_cast<int32_t *>(base + lay.err); }
+  int32_t *seqlen() const { return reinterpret_cast<int32_t *>(base + lay.seqlen); }
+  double2 *ea() const { return reinterpret_cast<double2 *>(base + lay.ea); }
+  float *raw() const { return reinterpret_cast<float *>(base + lay.raw); }
+  int32_t *sel() const { return reinterpret_cast<int32_t *>(base + lay.sel); }
+};
+
+const char *kStageNames[] = {"fold_kernel", "score_kernel", "unit_kernel"};
+
+}  // namespace
+
+extern "C" {
+
+tria_status tria_workspace_size(const tria_config *cfg, const tria_cache *cache, size_t *bytes) {
+  if (!bytes) return TRIA_ERR_INVALID_ARG;
+  tria_status s = check_config(cfg, false);
+  if (s != TRIA_OK) return s;
+  if (!cache || cache->cap_total < 0) return TRIA_ERR_INVALID_ARG;
+  *bytes = ws_layout(*cfg, cache->cap_total).total;
+  return TRIA_OK;
+}
+
+tria_status tria_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+  if (!ws || ws_bytes < 256 || !aligned(ws, 256)) return TRIA_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)));
+}
+
+tria_status tria_calibrate(const tria_config *cfg, const void *q_pre, int32_t q_dtype,
+                           int64_t n_samples, float *centre, float *mean_norm, float *mrl,
+                           void *stream) {
+  if (!cfg || !q_pre || !centre || !mean_norm || !mrl || n_samples < 1)
+    return TRIA_ERR_INVALID_ARG;
+  if (cfg->num_layers < 1 || cfg->n_q_heads < 1 || cfg->head_dim < 2 || cfg->head_dim % 2)
+    return TRIA_ERR_INVALID_ARG;
+  if (cfg->rope_layout != TRIA_ROPE_HALF_SPLIT && cfg->rope_layout != TRIA_ROPE_INTERLEAVED)
+    return TRIA_ERR_INVALID_ARG;
+  if (q_dtype != TRIA_DTYPE_F32 && q_dtype != TRIA_DTYPE_BF16) return TRIA_ERR_INVALID_ARG;
+  if (cfg->head_dim / 2 > 256) return TRIA_ERR_UNSUPPORTED;
+  if (!aligned(centre, 8) || !aligned(mean_norm, 4) || !aligned(mrl, 4) ||
+      !aligned(q_pre, q_dtype == TRIA_DTYPE_F32 ? 4 : 2))
+    return TRIA_ERR_INVALID_ARG;
+  return cuda_status(launch_calibrate(q_pre, q_dtype, cfg->num_layers, n_samples, cfg->n_q_heads,
+                                      cfg->head_dim, cfg->rope_layout, centre, mean_norm, mrl,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+tria_status tria_score(const tria_config *cfg, const tria_stats *stats, const tria_cache *cache,
+                       float *score, float *raw, void *ws, size_t ws_bytes, void *stream) {
+  tria_status s;
+  if ((s = check_config(cfg, true)) != TRIA_OK) return s;
+  if ((s = check_cache(cfg, cache, false)) != TRIA_OK) return s;
+  if (!cache->k || !aligned(cache->k, 16) || !cache->cur_pos) return TRIA_ERR_INVALID_ARG;
+  if ((s = check_stats(stats)) != TRIA_OK) return s;
+  if (!score || (raw && !aligned(raw, 4))) return TRIA_ERR_INVALID_ARG;
+  if ((s = check_ws(cfg, cache, ws, ws_bytes)) != TRIA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws w{ws_layout(*cfg, cache->cap_total), static_cast<uint8_t *>(ws)};
+  float *rawp = raw ? raw : w.raw();
+
+  static thread_local FoldParams fp;
+  fill_fold(fp, cfg, cache, w.seqlen(), w.ea(), w.err());
+  cudaError_t e = launch_fold(fp, cfg->head_dim / 2, st);
+  if (e != cudaSuccess) return TRIA_ERR_CUDA;
+  ScoreParams sp;
+  const int grid = fill_score(sp, cfg, stats, cache, w.ea(), w.seqlen(), rawp, w.err(), 0);
+  if (grid > 0) {
+    e = launch_score(sp, cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads, cfg->rope_layout, grid, st);
+    if (e != cudaSuccess) return TRIA_ERR_CUDA;
+  }
+  UnitParams up;
+  fill_unit(up, cfg, cache, kModeZmax);
+  up.raw = rawp;
+  up.score = score;
+  up.seqlen = w.seqlen();
+  up.err = w.err();
+  return cuda_status(launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch, st));
+}
+
+tria_status tria_select(const tria_config *cfg, const tria_cache *cache, const float *score,
+                        int32_t *sel, void *ws, size_t ws_bytes, void *stream) {
+  tria_status s;
+  if ((s = check_config(cfg, false)) != TRIA_OK) return s;
+  if ((s = check_cache(cfg, cache, false)) != TRIA_OK) return s;
+  if (!score || !sel || !aligned(score, 4) || !aligned(sel, 4)) return TRIA_ERR_INVALID_ARG;
+  if ((s = check_ws(cfg, cache, ws, ws_bytes)) != TRIA_OK) return s;
+  const Ws w{ws_layout(*cfg, cache->cap_total), static_cast<uint8_t *>(ws)};
+  UnitParams up;
+  fill_unit(up, cfg, cache, kModeSelect);
+  up.score = const_cast<float *>(score);
+  up.sel = sel;
+  up.seqlen = cache->seq_len;
+  up.err = w.err();
+  return cuda_status(launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+tria_status tria_compact(const tria_config *cfg, const tria_cache *cache, const int32_t *sel,
+                         void *ws, size_t ws_bytes, void *stream) {
+  tria_status s;
+  if ((s = check_config(cfg, false)) != TRIA_OK) return s;
+  if ((s = check_cache(cfg, cache, true)) != TRIA_OK) return s;
+  if (!sel || !aligned(sel, 4)) return TRIA_ERR_INVALID_ARG;
+  if ((s = check_ws(cfg, cache, ws, ws_bytes)) != TRIA_OK) return s;
+  const Ws w{ws_layout(*cfg, cache->cap_total), static_cast<uint8_t *>(ws)};
+  UnitParams up;
+  fill_unit(up, cfg, cache, kModeCompact);
+  up.sel = const_cast<int32_t *>(sel);
+  up.seq_len_out = cache->seq_len;
+  up.err = w.err();
+  return cuda_status(launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
+                                const tria_cache *cache, int32_t *sel_out, void *ws,
+                                size_t ws_bytes, void *stream, void *const *events,
+                                int32_t *n_stages) {
+  tria_status s;
+  if ((s = check_config(cfg, true)) != TRIA_OK) return s;
+  if ((s = check_cache(cfg, cache, true)) != TRIA_OK) return s;
+  if (!cache->cur_pos) return TRIA_ERR_INVALID_ARG;
+  if ((s = check_stats(stats)) != TRIA_OK) return s;
+  if (sel_out && !aligned(sel_out, 4)) return TRIA_ERR_INVALID_ARG;
+  if ((s = check_ws(cfg, cache, ws, ws_bytes)) != TRIA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws w{ws_layout(*cfg, cache->cap_total), static_cast<uint8_t *>(ws)};
+  int stage = 0;
+  auto mark = [&]() -> bool {
+    if (events && cudaEventRecord(static_cast<cudaEvent_t>(events[stage]), st) != cudaSuccess)
+      return false;
+    ++stage;
+    return true;
+  };
+
+  static thread_local FoldParams fp;
+  fill_fold(fp, cfg, cache, w.seqlen(), w.ea(), w.err());
+  if (!mark()) return TRIA_ERR_CUDA;
+  if (launch_fold(fp, cfg->head_dim / 2, st) != cudaSuccess) return TRIA_ERR_CUDA;
+  ScoreParams sp;
+  const int grid = fill_score(sp, cfg, stats, cache, w.ea(), w.seqlen(), w.raw(), w.err(), 1);
+  if (!mark()) return TRIA_ERR_CUDA;
+  if (grid > 0 && launch_score(sp, cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads,
+                               cfg->rope_layout, grid, st) != cudaSuccess)
+    return TRIA_ERR_CUDA;
+  UnitParams up;
+  fill_unit(up, cfg, cache, kModePrune);
+  up.raw = w.raw();
+  up.sel = sel_out ? sel_out : w.sel();
+  up.write_short_sel = sel_out ? 1 : 0;
+  up.seqlen = w.seqlen();
+  up.seq_len_out = cache->seq_len;
+  up.err = w.err();
+  if (!mark()) return TRIA_ERR_CUDA;
+  if (launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch, st) != cudaSuccess)
+    return TRIA_ERR_CUDA;
+  if (!mark()) return TRIA_ERR_CUDA;
+  if (n_stages) *n_stages = stage - 1;
+  return TRIA_OK;
+}
+
+tria_status tria_prune(const tria_config *cfg, const tria_stats *stats, const tria_cache *cache,
+                       int32_t *sel_out, void *ws, size_t ws_bytes, void *stream) {
+  return tria_prune_profiled(cfg, stats, cache, sel_out, ws, ws_bytes, stream, nullptr, nullptr);
+}
+
+const char *tria_prune_stage_name(int32_t i) {
+  if (i < 0 || i >= (int32_t)(sizeof kStageNames / sizeof kStageNames[0])) return "";
+  return kStageNames[i];
+}
+
+tria_status tria_get_device_error(const void *ws, int32_t *code, void *stream) {
+  if (!ws || !code) return TRIA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return TRIA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TRIA_ERR_CUDA;
+  *code = v;
+  return v ? TRIA_ERR_DEVICE_FLAG : TRIA_OK;
+}
+
+const char *tria_status_string(tria_status s) {
+  switch (s) {
+    case TRIA_OK: return "TRIA_OK";
+    case TRIA_ERR_INVALID_ARG: return "TRIA_ERR_INVALID_ARG";
+    case TRIA_ERR_UNSUPPORTED: return "TRIA_ERR_UNSUPPORTED";
+    case TRIA_ERR_WORKSPACE: return "TRIA_ERR_WORKSPACE";
+    case TRIA_ERR_CUDA: return "TRIA_ERR_CUDA";
+    case TRIA_ERR_DEVICE_FLAG: return "TRIA_ERR_DEVICE_FLAG";
+  }
+  return "TRIA_UNKNOWN_STATUS";
+}
+
+const char *tria_version(void) { return "tria 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,336 @@
+// Raw key scores, one streaming pass over the cached keys.
+//
+// For every live key t of every (layer l, KV head g, sequence b) and every
+// query head h of g's group (romaanj.github.io review, "Method";
+// dimensionstp.github.io review, sections 2-2 and 3-2 (2)-(4)):
+//   s_h(t) = sum_f [ Re(conj(ktilde_f) * W_hf) + Nw_hf * |ktilde_f| ]
+//   W_hf   = c_hf * EA_bf          (trig term with offsets and cur folded in, see fold.cu)
+//   Nw_hf  = (1 - R_hf) * E|q_hf|  (norm term; |k_f| = |ktilde_f| since RoPE keeps norms)
+// ktilde is the stored post-RoPE bf16 key widened exactly to float; all sums
+// are float32.
+//
+// Design (sm_100a): a persistent grid, one CTA per SM, each taking a
+// contiguous run of 32 KB key tiles.  One producer warp streams tiles into a
+// 4-stage shared-memory ring with 1-D bulk copies (cp.async.bulk, completion
+// on mbarriers, no multicast); eight consumer warps compute.  A consumer lane
+// owns PPL RoPE pairs of one key, so the G x PPL x 3 weights of its unit live
+// in registers and each key costs one pass over D with 3 FMAs per (pair,
+// head); LPK lanes cooperate on a key and combine by xor shuffles.  Raw
+// scores go through a small shared buffer so the global stores are coalesced.
+#include "tria_internal.cuh"
+
+namespace tria {
+
+template <int D, int G>
+struct ScoreShape {
+  static constexpr int F = D / 2;
+  static constexpr int PPL_A = (32 / G) < 8 ? (32 / G) : 8;
+  static constexpr int PPL = (F / 32) > PPL_A ? (F / 32) : PPL_A;  // pairs per lane
+  static constexpr int LPK = F / PPL;                             // lanes per key
+  static constexpr int KPW = 32 / LPK;                            // keys per warp step
+  static constexpr int ROW = 2 * D;                               // bytes per key row
+  static constexpr int TILE = kScoreTileBytes / ROW;              // keys per tile
+  static constexpr int NW = kScoreConsumerWarps;
+  static constexpr int KEYS_PER_WARP = TILE / NW;
+  static constexpr int STEPS = KEYS_PER_WARP / KPW;
+  static constexpr bool OK = (3 * G * PPL <= 96) && (LPK <= 32) && (LPK >= 1) &&
+                             (STEPS * KPW == KEYS_PER_WARP) && (STEPS >= 1);
+  static constexpr size_t SMEM = (size_t)kScoreStages * TILE * ROW + 2ull * G * TILE * 4 +
+                                 2ull * kScoreStages * 8;
+};
+
+struct TileRef {
+  int32_t row;   // l * Hkv + g
+  int32_t b;
+  int64_t key0;  // first key of the tile within the segment
+  int32_t n;     // live keys in the tile (0: nothing to do)
+};
+
+__device__ __forceinline__ TileRef tile_of(const ScoreParams &p, int64_t t, int tile_keys) {
+  TileRef r;
+  r.row = (int32_t)(t / p.tiles_per_row);
+  const int32_t rem = (int32_t)(t - (int64_t)r.row * p.tiles_per_row);
+  int lo = 0, hi = p.B;  // largest b with tile_prefix[b] <= rem
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.tile_prefix[mid] <= rem) lo = mid; else hi = mid;
+  }
+  r.b = lo;
+  r.key0 = (int64_t)(rem - p.tile_prefix[lo]) * tile_keys;
+  const int32_t T = p.seqlen[lo];
+  int64_t n = (int64_t)T - r.key0;
+  n = n < 0 ? 0 : (n > tile_keys ? tile_keys : n);
+  if (p.skip_short && T <= p.budget) n = 0;
+  r.n = (int32_t)n;
+  return r;
+}
+
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float y;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Loads the PPL pairs a lane owns from a key row in shared memory:
+// x[p], y[p] for pairs f0 .. f0+PPL-1.
+template <int D, int PPL, int LAYOUT>
+__device__ __forceinline__ void load_pairs(const uint8_t *rowp, int f0, float (&x)[PPL],
+                                           float (&y)[PPL]) {
+  if constexpr (LAYOUT == TRIA_ROPE_HALF_SPLIT) {
+    uint32_t xw[PPL / 2], yw[PPL / 2];
+    const uint8_t *px = rowp + 2 * f0;
+    const uint8_t *py = rowp + D + 2 * f0;
+    if constexpr (PPL == 8) {
+      const uint4 a = *reinterpret_cast<const uint4 *>(px);
+      const uint4 b = *reinterpret_cast<const uint4 *>(py);
+      xw[0] = a.x; xw[1] = a.y; xw[2] = a.z; xw[3] = a.w;
+      yw[0] = b.x; yw[1] = b.y; yw[2] = b.z; yw[3] = b.w;
+    } else if constexpr (PPL == 4) {
+      const uint2 a = *reinterpret_cast<const uint2 *>(px);
+      const uint2 b = *reinterpret_cast<const uint2 *>(py);
+      xw[0] = a.x; xw[1] = a.y;
+      yw[0] = b.x; yw[1] = b.y;
+    } else {
+      xw[0] = *reinterpret_cast<const uint32_t *>(px);
+      yw[0] = *reinterpret_cast<const uint32_t *>(py);
+    }
+#pragma unroll
+    for (int i = 0; i < PPL / 2; ++i) {
+      x[2 * i] = dev::bf16lo(xw[i]);
+      x[2 * i + 1] = dev::bf16hi(xw[i]);
+      y[2 * i] = dev::bf16lo(yw[i]);
+      y[2 * i + 1] = dev::bf16hi(yw[i]);
+    }
+  } else {
+    uint32_t w[PPL];
+    const uint8_t *pp = rowp + 4 * f0;
+    if constexpr (PPL == 8) {
+      const uint4 a = *reinterpret_cast<const uint4 *>(pp);
+      const uint4 b = *reinterpret_cast<const uint4 *>(pp + 16);
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+      w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    } else if constexpr (PPL == 4) {
+      const uint4 a = *reinterpret_cast<const uint4 *>(pp);
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    } else {
+      const uint2 a = *reinterpret_cast<const uint2 *>(pp);
+      w[0] = a.x; w[1] = a.y;
+    }
+#pragma unroll
+    for (int i = 0; i < PPL; ++i) {
+      x[i] = dev::bf16lo(w[i]);
+      y[i] = dev::bf16hi(w[i]);
+    }
+  }
+}
+
+template <int D, int G, int LAYOUT>
+__global__ void __launch_bounds__(kScoreThreads, 1)
+    score_kernel(const __grid_constant__ ScoreParams p) {
+  using S = ScoreShape<D, G>;
+  constexpr int F = S::F, PPL = S::PPL, LPK = S::LPK, KPW = S::KPW, ROW = S::ROW;
+  constexpr int TILE = S::TILE, NW = S::NW, NST = kScoreStages;
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t *stage = smem;
+  float *rawst = reinterpret_cast<float *>(smem + (size_t)NST * TILE * ROW);  // [2][G][TILE]
+  uint64_t *full = reinterpret_cast<uint64_t *>(rawst + 2 * G * TILE);
+  uint64_t *empty = full + NST;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      dev::mbar_init(&full[s], 1);
+      dev::mbar_init(&empty[s], NW);
+    }
+    dev::fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int64_t t0 = (int64_t)blockIdx.x * p.tiles_per_cta;
+  int64_t t1 = t0 + p.tiles_per_cta;
+  if (t1 > p.total_tiles) t1 = p.total_tiles;
+
+  if (warp == NW) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool failed = false;
+      for (int64_t t = t0; t < t1 && !failed; ++t) {
+        const TileRef tl = tile_of(p, t, TILE);
+        if (tl.n <= 0) continue;
+        const uint32_t s = it % NST, use = it / NST;
+        if (use > 0 && !dev::mbar_wait(&empty[s], (use - 1) & 1)) {
+          dev::set_error(p.err, TRIA_DEVERR_TIMEOUT);
+          failed = true;
+          break;
+        }
+        const uint32_t bytes = (uint32_t)tl.n * ROW;
+        const uint8_t *src =
+            p.k + ((size_t)tl.row * p.cap + p.seg_start[tl.b] + tl.key0) * (size_t)ROW;
+        dev::mbar_arrive_expect_tx(&full[s], bytes);
+        dev::bulk_g2s(stage + (size_t)s * TILE * ROW, src, bytes, &full[s]);
+        ++it;
+      }
+      if (failed) {
+        // let the copies already issued land before the CTA can retire
+        const uint32_t first = it > (uint32_t)NST ? it - NST : 0;
+        for (uint32_t u = first; u < it; ++u) dev::mbar_wait(&full[u % NST], (u / NST) & 1);
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ consumers
+  const int kg = lane / LPK, li = lane % LPK, f0 = li * PPL;
+  float wx[G][PPL], wy[G][PPL], nw[G][PPL];
+  int64_t cached = -1;
+  uint32_t it = 0;
+  bool failed = false;
+  for (int64_t t = t0; t < t1; ++t) {
+    const TileRef tl = tile_of(p, t, TILE);
+    if (tl.n <= 0) continue;
+    const int32_t l = tl.row / p.Hkv, g = tl.row - l * p.Hkv;
+    const int64_t unit = (int64_t)tl.row * p.B + tl.b;
+    if (unit != cached) {
+      cached = unit;
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const size_t base = ((size_t)l * p.Hq + (size_t)g * G + j) * F + f0;
+#pragma unroll
+        for (int q = 0; q < PPL; ++q) {
+          const float2 c = p.centre[base + q];
+          const double2 e = p.ea[(size_t)tl.b * F + f0 + q];
+          wx[j][q] = (float)((double)c.x * e.x - (double)c.y * e.y);
+          wy[j][q] = (float)((double)c.x * e.y + (double)c.y * e.x);
+          const float r = p.no_conc_weight ? 0.0f : p.mrl[base + q];
+          nw[j][q] = (1.0f - r) * p.mean_norm[base + q];
+        }
+      }
+    }
+    const uint32_t s = it % NST, use = it / NST;
+    if (!failed && !dev::mbar_wait(&full[s], use & 1)) {
+      dev::set_error(p.err, TRIA_DEVERR_TIMEOUT);
+      failed = true;
+    }
+    float *rs = rawst + (size_t)(it & 1) * G * TILE;
+    if (!failed) {
+      const uint8_t *sb = stage + (size_t)s * TILE * ROW;
+#pragma unroll 1
+      for (int step = 0; step < S::STEPS; ++step) {
+        const int kk = warp * S::KEYS_PER_WARP + step * KPW + kg;
+        float x[PPL], y[PPL];
+        load_pairs<D, PPL, LAYOUT>(sb + (size_t)kk * ROW, f0, x, y);
+        float acc[G];
+#pragma unroll
+        for (int j = 0; j < G; ++j) acc[j] = 0.0f;
+#pragma unroll
+        for (int q = 0; q < PPL; ++q) {
+          const float nrm = sqrt_approx(fmaf(y[q], y[q], x[q] * x[q]));
+#pragma unroll
+          for (int j = 0; j < G; ++j) {
+            acc[j] = fmaf(wx[j][q], x[q], acc[j]);
+            acc[j] = fmaf(wy[j][q], y[q], acc[j]);
+            acc[j] = fmaf(nw[j][q], nrm, acc[j]);
+          }
+        }
+#pragma unroll
+        for (int o = LPK / 2; o > 0; o >>= 1) {
+#pragma unroll
+          for (int j = 0; j < G; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+        }
+        if (kk < tl.n) {
+#pragma unroll
+          for (int j = 0; j < G; ++j)
+            if (j % LPK == li) rs[j * TILE + kk] = acc[j];
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) dev::mbar_arrive(&empty[s]);
+    dev::named_barrier(1, NW * 32);
+    if (!failed) {
+      const size_t seg = (size_t)p.seg_start[tl.b] + tl.key0;
+      for (int idx = threadIdx.x; idx < G * tl.n; idx += NW * 32) {
+        const int j = idx / tl.n, kk = idx - j * tl.n;
+        p.raw[((size_t)l * p.Hq + (size_t)g * G + j) * p.cap + seg + kk] = rs[j * TILE + kk];
+      }
+    }
+    ++it;
+  }
+}
+
+template <int D, int G, int LAYOUT>
+static cudaError_t launch_one(const ScoreParams &p, int grid, cudaStream_t s) {
+  using S = ScoreShape<D, G>;
+  if constexpr (!S::OK) {
+    return cudaErrorInvalidValue;
+  } else {
+    auto kern = score_kernel<D, G, LAYOUT>;
+    static bool configured = false;  // per instantiation; attribute set once per process
+    if (!configured) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)S::SMEM);
+      if (e != cudaSuccess) return e;
+      configured = true;
+    }
+    kern<<<grid, kScoreThreads, S::SMEM, s>>>(p);
+    return cudaGetLastError();
+  }
+}
+
+template <int D, int LAYOUT>
+static cudaError_t dispatch_g(const ScoreParams &p, int G, int grid, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_one<D, 1, LAYOUT>(p, grid, s);
+    case 2: return launch_one<D, 2, LAYOUT>(p, grid, s);
+    case 4: return launch_one<D, 4, LAYOUT>(p, grid, s);
+    case 8: return launch_one<D, 8, LAYOUT>(p, grid, s);
+    case 16: return launch_one<D, 16, LAYOUT>(p, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int D>
+static bool supported_g(int G) {
+  switch (G) {
+    case 1: return ScoreShape<D, 1>::OK;
+    case 2: return ScoreShape<D, 2>::OK;
+    case 4: return ScoreShape<D, 4>::OK;
+    case 8: return ScoreShape<D, 8>::OK;
+    case 16: return ScoreShape<D, 16>::OK;
+    default: return false;
+  }
+}
+
+bool score_supported(int D, int G, int layout) {
+  if (layout != TRIA_ROPE_HALF_SPLIT && layout != TRIA_ROPE_INTERLEAVED) return false;
+  switch (D) {
+    case 64: return supported_g<64>(G);
+    case 128: return supported_g<128>(G);
+    case 256: return supported_g<256>(G);
+    default: return false;
+  }
+}
+
+int score_tile_keys(int D) { return kScoreTileBytes / (2 * D); }
+
+cudaError_t launch_score(const ScoreParams &p, int D, int G, int layout, int grid,
+                         cudaStream_t s) {
+  if (layout == TRIA_ROPE_HALF_SPLIT) {
+    switch (D) {
+      case 64: return dispatch_g<64, TRIA_ROPE_HALF_SPLIT>(p, G, grid, s);
+      case 128: return dispatch_g<128, TRIA_ROPE_HALF_SPLIT>(p, G, grid, s);
+      case 256: return dispatch_g<256, TRIA_ROPE_HALF_SPLIT>(p, G, grid, s);
+    }
+  } else {
+    switch (D) {
+      case 64: return dispatch_g<64, TRIA_ROPE_INTERLEAVED>(p, G, grid, s);
+      case 128: return dispatch_g<128, TRIA_ROPE_INTERLEAVED>(p, G, grid, s);
+      case 256: return dispatch_g<256, TRIA_ROPE_INTERLEAVED>(p, G, grid, s);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace tria

@@ -124,7 +124,7 @@ void fill_fold(FoldParams &fp, const tria_config *cfg, const tria_cache *c, int3
 
 // Builds the score kernel parameters; returns the grid size (0: nothing to launch).
 int fill_score(ScoreParams &sp, const tria_config *cfg, const tria_stats *st, const tria_cache *c,
-               const double2 *ea, const int32_t *seqlen, float *raw, int32_t *err, int skip_short) {
+               const double2 *ea, float *raw, int32_t *err, int skip_short) {
   std::memset(&sp, 0, sizeof sp);
   const int tile = score_tile_keys(cfg->head_dim);
   sp.k = static_cast<const uint8_t *>(c->k);
@@ -132,7 +132,7 @@ int fill_score(ScoreParams &sp, const tria_config *cfg, const tria_stats *st, co
   sp.mean_norm = st->mean_norm;
   sp.mrl = st->mrl;
   sp.ea = ea;
-  sp.seqlen = seqlen;
+  sp.seq_len = c->seq_len;
   sp.raw = raw;
   sp.err = err;
   sp.cap = c->cap_total;
@@ -173,7 +173,13 @@ void fill_unit(UnitParams &up, const tria_config *cfg, const tria_cache *c, int 
   up.D = cfg->head_dim;
   up.budget = cfg->budget;
   up.mode = mode;
-  for (int b = 0; b <= cfg->batch; ++b) up.seg_start[b] = c->seq_start[b];
+  int64_t max_seg = 0;
+  for (int b = 0; b <= cfg->batch; ++b) {
+    up.seg_start[b] = c->seq_start[b];
+    if (b < cfg->batch && c->seq_start[b + 1] - c->seq_start[b] > max_seg)
+      max_seg = c->seq_start[b + 1] - c->seq_start[b];
+  }
+  up.smem_bytes = unit_smem_bytes(cfg->num_layers * cfg->n_kv_heads * cfg->batch, max_seg);
 }
 
 struct Ws {
@@ -243,9 +249,10 @@ tria_status tria_score(const tria_config *cfg, const tria_stats *stats, const tr
   cudaError_t e = launch_fold(fp, cfg->head_dim / 2, st);
   if (e != cudaSuccess) return TRIA_ERR_CUDA;
   ScoreParams sp;
-  const int grid = fill_score(sp, cfg, stats, cache, w.ea(), w.seqlen(), rawp, w.err(), 0);
+  const int grid = fill_score(sp, cfg, stats, cache, w.ea(), rawp, w.err(), 0);
   if (grid > 0) {
-    e = launch_score(sp, cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads, cfg->rope_layout, grid, st);
+    e = launch_score(sp, cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads, cfg->rope_layout, grid,
+                     st, true);
     if (e != cudaSuccess) return TRIA_ERR_CUDA;
   }
   UnitParams up;
@@ -254,7 +261,7 @@ tria_status tria_score(const tria_config *cfg, const tria_stats *stats, const tr
   up.score = score;
   up.seqlen = w.seqlen();
   up.err = w.err();
-  return cuda_status(launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch, st));
+  return cuda_status(launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch, st, true));
 }
 
 tria_status tria_select(const tria_config *cfg, const tria_cache *cache, const float *score,
@@ -272,7 +279,7 @@ tria_status tria_select(const tria_config *cfg, const tria_cache *cache, const f
   up.seqlen = cache->seq_len;
   up.err = w.err();
   return cuda_status(launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch,
-                                 static_cast<cudaStream_t>(stream)));
+                                 static_cast<cudaStream_t>(stream), false));
 }
 
 tria_status tria_compact(const tria_config *cfg, const tria_cache *cache, const int32_t *sel,
@@ -289,7 +296,7 @@ tria_status tria_compact(const tria_config *cfg, const tria_cache *cache, const 
   up.seq_len_out = cache->seq_len;
   up.err = w.err();
   return cuda_status(launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch,
-                                 static_cast<cudaStream_t>(stream)));
+                                 static_cast<cudaStream_t>(stream), false));
 }
 
 tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
@@ -318,10 +325,11 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
   if (!mark()) return TRIA_ERR_CUDA;
   if (launch_fold(fp, cfg->head_dim / 2, st) != cudaSuccess) return TRIA_ERR_CUDA;
   ScoreParams sp;
-  const int grid = fill_score(sp, cfg, stats, cache, w.ea(), w.seqlen(), w.raw(), w.err(), 1);
+  const int grid = fill_score(sp, cfg, stats, cache, w.ea(), w.raw(), w.err(), 1);
+  const bool pdl = events == nullptr;  // stage events between kernels would defeat the overlap
   if (!mark()) return TRIA_ERR_CUDA;
   if (grid > 0 && launch_score(sp, cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads,
-                               cfg->rope_layout, grid, st) != cudaSuccess)
+                               cfg->rope_layout, grid, st, pdl) != cudaSuccess)
     return TRIA_ERR_CUDA;
   UnitParams up;
   fill_unit(up, cfg, cache, kModePrune);
@@ -332,7 +340,7 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
   up.seq_len_out = cache->seq_len;
   up.err = w.err();
   if (!mark()) return TRIA_ERR_CUDA;
-  if (launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch, st) != cudaSuccess)
+  if (launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch, st, pdl) != cudaSuccess)
     return TRIA_ERR_CUDA;
   if (!mark()) return TRIA_ERR_CUDA;
   if (n_stages) *n_stages = stage - 1;

@@ -16,6 +16,7 @@
 namespace tria {
 
 __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldParams p) {
+  dev::pdl_launch_dependents();  // the score kernel may start streaming keys now
   const int f = blockIdx.x;
   const double w = pow(p.theta, -2.0 * (double)f / (double)p.D);
   double sc = 0.0, ss = 0.0;

@@ -13,10 +13,14 @@
 // contiguous run of 32 KB key tiles.  One producer warp streams tiles into a
 // 4-stage shared-memory ring with 1-D bulk copies (cp.async.bulk, completion
 // on mbarriers, no multicast); eight consumer warps compute.  A consumer lane
-// owns PPL RoPE pairs of one key, so the G x PPL x 3 weights of its unit live
-// in registers and each key costs one pass over D with 3 FMAs per (pair,
-// head); LPK lanes cooperate on a key and combine by xor shuffles.  Raw
-// scores go through a small shared buffer so the global stores are coalesced.
+// owns PPL RoPE pairs of a key, so the G x PPL x 3 weights of its unit live in
+// registers, packed two pairs per 64-bit register for the sm_100 paired FP32
+// FMA (fma.rn.f32x2): one instruction per (two pairs, head, term).  Each lane
+// works on two keys at once for instruction-level parallelism.  The LPK lanes
+// of a key combine their partial sums by a reduce-scatter (each shuffle level
+// halves the values a lane holds); the heads are assigned to register slots in
+// a lane-dependent order at weight-load time so that no selects are needed and
+// each lane ends with one head's total, which it stores.
 #include "tria_internal.cuh"
 
 namespace tria {
@@ -32,11 +36,11 @@ struct ScoreShape {
   static constexpr int TILE = kScoreTileBytes / ROW;              // keys per tile
   static constexpr int NW = kScoreConsumerWarps;
   static constexpr int KEYS_PER_WARP = TILE / NW;
-  static constexpr int STEPS = KEYS_PER_WARP / KPW;
-  static constexpr bool OK = (3 * G * PPL <= 96) && (LPK <= 32) && (LPK >= 1) &&
-                             (STEPS * KPW == KEYS_PER_WARP) && (STEPS >= 1);
-  static constexpr size_t SMEM = (size_t)kScoreStages * TILE * ROW + 2ull * G * TILE * 4 +
-                                 2ull * kScoreStages * 8;
+  static constexpr int STEPS = KEYS_PER_WARP / (2 * KPW);         // two keys per lane per step
+  static constexpr bool OK = (3 * G * PPL <= 96) && (LPK <= 32) && (LPK >= G) &&
+                             (PPL % 2 == 0) && (STEPS * 2 * KPW == KEYS_PER_WARP) &&
+                             (STEPS >= 1);
+  static constexpr size_t SMEM = (size_t)kScoreStages * TILE * ROW + 2ull * kScoreStages * 8;
 };
 
 struct TileRef {
@@ -57,7 +61,8 @@ __device__ __forceinline__ TileRef tile_of(const ScoreParams &p, int64_t t, int 
   }
   r.b = lo;
   r.key0 = (int64_t)(rem - p.tile_prefix[lo]) * tile_keys;
-  const int32_t T = p.seqlen[lo];
+  int32_t T = p.seq_len[lo];
+  if (T < 0 || (int64_t)T > p.seg_start[lo + 1] - p.seg_start[lo]) T = 0;  // flagged by the fold
   int64_t n = (int64_t)T - r.key0;
   n = n < 0 ? 0 : (n > tile_keys ? tile_keys : n);
   if (p.skip_short && T <= p.budget) n = 0;
@@ -69,6 +74,48 @@ __device__ __forceinline__ float sqrt_approx(float x) {
   float y;
   asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Paired float32 arithmetic of sm_100 (two lanes of work per instruction).
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// Reduce-scatter over the lanes of a key: at offset O, a lane holding V values
+// keeps the first V/2 and adds its partner's second half; once one value is
+// left the remaining levels are a plain butterfly sum.
+template <int O, int V, int G>
+__device__ __forceinline__ void reduce_scatter(float (&a)[G], float (&b)[G]) {
+  if constexpr (O >= 1) {
+    if constexpr (V > 1) {
+      constexpr int H = V / 2;
+#pragma unroll
+      for (int k = 0; k < H; ++k) {
+        a[k] += __shfl_xor_sync(0xffffffffu, a[k + H], O);
+        b[k] += __shfl_xor_sync(0xffffffffu, b[k + H], O);
+      }
+      reduce_scatter<O / 2, H, G>(a, b);
+    } else {
+      a[0] += __shfl_xor_sync(0xffffffffu, a[0], O);
+      b[0] += __shfl_xor_sync(0xffffffffu, b[0], O);
+      reduce_scatter<O / 2, 1, G>(a, b);
+    }
+  }
 }
 
 // Loads the PPL pairs a lane owns from a key row in shared memory:
@@ -133,8 +180,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t *stage = smem;
-  float *rawst = reinterpret_cast<float *>(smem + (size_t)NST * TILE * ROW);  // [2][G][TILE]
-  uint64_t *full = reinterpret_cast<uint64_t *>(rawst + 2 * G * TILE);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)NST * TILE * ROW);
   uint64_t *empty = full + NST;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -146,6 +192,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     dev::fence_mbar_init();
   }
   __syncthreads();
+  if (threadIdx.x == 0) dev::pdl_launch_dependents();
 
   const int64_t t0 = (int64_t)blockIdx.x * p.tiles_per_cta;
   int64_t t1 = t0 + p.tiles_per_cta;
@@ -178,12 +225,22 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         for (uint32_t u = first; u < it; ++u) dev::mbar_wait(&full[u % NST], (u / NST) & 1);
       }
     }
+    dev::pdl_wait();  // this grid never completes before the fold it depends on
     return;
   }
 
   // ------------------------------------------------------------------ consumers
+  constexpr int P2 = PPL / 2;
   const int kg = lane / LPK, li = lane % LPK, f0 = li * PPL;
-  float wx[G][PPL], wy[G][PPL], nw[G][PPL];
+  // register slot k of this lane holds head (k ^ hmask) of the group, so that the
+  // reduce-scatter leaves head hmask's total in slot 0 (see reduce_scatter)
+  int hmask = 0;
+#pragma unroll
+  for (int lv = 0; (G >> (lv + 1)) > 0; ++lv)
+    if (li & (LPK >> (lv + 1))) hmask |= (G >> (lv + 1));
+  const bool writer = (li & (LPK / G - 1)) == 0;  // lanes holding duplicate totals stay quiet
+  uint64_t wx[G][P2], wy[G][P2], nw[G][P2];
+  dev::pdl_wait();  // the folded offset factors come from the fold kernel
   int64_t cached = -1;
   uint32_t it = 0;
   bool failed = false;
@@ -195,16 +252,24 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     if (unit != cached) {
       cached = unit;
 #pragma unroll
-      for (int j = 0; j < G; ++j) {
-        const size_t base = ((size_t)l * p.Hq + (size_t)g * G + j) * F + f0;
+      for (int k = 0; k < G; ++k) {
+        const size_t base = ((size_t)l * p.Hq + (size_t)g * G + (k ^ hmask)) * F + f0;
 #pragma unroll
-        for (int q = 0; q < PPL; ++q) {
-          const float2 c = p.centre[base + q];
-          const double2 e = p.ea[(size_t)tl.b * F + f0 + q];
-          wx[j][q] = (float)((double)c.x * e.x - (double)c.y * e.y);
-          wy[j][q] = (float)((double)c.x * e.y + (double)c.y * e.x);
-          const float r = p.no_conc_weight ? 0.0f : p.mrl[base + q];
-          nw[j][q] = (1.0f - r) * p.mean_norm[base + q];
+        for (int i = 0; i < P2; ++i) {
+          float ax[2], ay[2], an[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int q = 2 * i + e;
+            const float2 c = p.centre[base + q];
+            const double2 ea = p.ea[(size_t)tl.b * F + f0 + q];
+            ax[e] = (float)((double)c.x * ea.x - (double)c.y * ea.y);
+            ay[e] = (float)((double)c.x * ea.y + (double)c.y * ea.x);
+            const float r = p.no_conc_weight ? 0.0f : p.mrl[base + q];
+            an[e] = (1.0f - r) * p.mean_norm[base + q];
+          }
+          wx[k][i] = f2_pack(ax[0], ax[1]);
+          wy[k][i] = f2_pack(ay[0], ay[1]);
+          nw[k][i] = f2_pack(an[0], an[1]);
         }
       }
     }
@@ -213,80 +278,100 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       dev::set_error(p.err, TRIA_DEVERR_TIMEOUT);
       failed = true;
     }
-    float *rs = rawst + (size_t)(it & 1) * G * TILE;
     if (!failed) {
       const uint8_t *sb = stage + (size_t)s * TILE * ROW;
+      float *rawh = p.raw + ((size_t)l * p.Hq + (size_t)g * G + hmask) * p.cap +
+                    (size_t)p.seg_start[tl.b] + tl.key0;
 #pragma unroll 1
       for (int step = 0; step < S::STEPS; ++step) {
-        const int kk = warp * S::KEYS_PER_WARP + step * KPW + kg;
-        float x[PPL], y[PPL];
-        load_pairs<D, PPL, LAYOUT>(sb + (size_t)kk * ROW, f0, x, y);
-        float acc[G];
+        const int ka = warp * S::KEYS_PER_WARP + step * 2 * KPW + kg, kb = ka + KPW;
+        float xa[PPL], ya[PPL], xb[PPL], yb[PPL];
+        load_pairs<D, PPL, LAYOUT>(sb + (size_t)ka * ROW, f0, xa, ya);
+        load_pairs<D, PPL, LAYOUT>(sb + (size_t)kb * ROW, f0, xb, yb);
+        uint64_t acca[G], accb[G];
 #pragma unroll
-        for (int j = 0; j < G; ++j) acc[j] = 0.0f;
+        for (int k = 0; k < G; ++k) acca[k] = accb[k] = 0ull;
 #pragma unroll
-        for (int q = 0; q < PPL; ++q) {
-          const float nrm = sqrt_approx(fmaf(y[q], y[q], x[q] * x[q]));
+        for (int i = 0; i < P2; ++i) {
+          const uint64_t XA = f2_pack(xa[2 * i], xa[2 * i + 1]);
+          const uint64_t YA = f2_pack(ya[2 * i], ya[2 * i + 1]);
+          const uint64_t XB = f2_pack(xb[2 * i], xb[2 * i + 1]);
+          const uint64_t YB = f2_pack(yb[2 * i], yb[2 * i + 1]);
+          float n0, n1, m0, m1;
+          f2_unpack(f2_fma(YA, YA, f2_mul(XA, XA)), n0, n1);
+          f2_unpack(f2_fma(YB, YB, f2_mul(XB, XB)), m0, m1);
+          const uint64_t NA = f2_pack(sqrt_approx(n0), sqrt_approx(n1));
+          const uint64_t NB = f2_pack(sqrt_approx(m0), sqrt_approx(m1));
 #pragma unroll
-          for (int j = 0; j < G; ++j) {
-            acc[j] = fmaf(wx[j][q], x[q], acc[j]);
-            acc[j] = fmaf(wy[j][q], y[q], acc[j]);
-            acc[j] = fmaf(nw[j][q], nrm, acc[j]);
+          for (int k = 0; k < G; ++k) {
+            acca[k] = f2_fma(wx[k][i], XA, acca[k]);
+            accb[k] = f2_fma(wx[k][i], XB, accb[k]);
+            acca[k] = f2_fma(wy[k][i], YA, acca[k]);
+            accb[k] = f2_fma(wy[k][i], YB, accb[k]);
+            acca[k] = f2_fma(nw[k][i], NA, acca[k]);
+            accb[k] = f2_fma(nw[k][i], NB, accb[k]);
           }
         }
+        float sa[G], sbv[G];
 #pragma unroll
-        for (int o = LPK / 2; o > 0; o >>= 1) {
-#pragma unroll
-          for (int j = 0; j < G; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+        for (int k = 0; k < G; ++k) {
+          float lo, hi;
+          f2_unpack(acca[k], lo, hi);
+          sa[k] = lo + hi;
+          f2_unpack(accb[k], lo, hi);
+          sbv[k] = lo + hi;
         }
-        if (kk < tl.n) {
-#pragma unroll
-          for (int j = 0; j < G; ++j)
-            if (j % LPK == li) rs[j * TILE + kk] = acc[j];
+        reduce_scatter<LPK / 2, G, G>(sa, sbv);
+        if (writer) {
+          if (ka < tl.n) rawh[ka] = sa[0];
+          if (kb < tl.n) rawh[kb] = sbv[0];
         }
       }
     }
     __syncwarp();
     if (lane == 0) dev::mbar_arrive(&empty[s]);
-    dev::named_barrier(1, NW * 32);
-    if (!failed) {
-      const size_t seg = (size_t)p.seg_start[tl.b] + tl.key0;
-      for (int idx = threadIdx.x; idx < G * tl.n; idx += NW * 32) {
-        const int j = idx / tl.n, kk = idx - j * tl.n;
-        p.raw[((size_t)l * p.Hq + (size_t)g * G + j) * p.cap + seg + kk] = rs[j * TILE + kk];
-      }
-    }
     ++it;
   }
 }
 
 template <int D, int G, int LAYOUT>
-static cudaError_t launch_one(const ScoreParams &p, int grid, cudaStream_t s) {
+static cudaError_t launch_one(const ScoreParams &p, int grid, cudaStream_t s, bool pdl) {
   using S = ScoreShape<D, G>;
   if constexpr (!S::OK) {
     return cudaErrorInvalidValue;
   } else {
     auto kern = score_kernel<D, G, LAYOUT>;
-    static bool configured = false;  // per instantiation; attribute set once per process
-    if (!configured) {
+    static bool configured[64] = {};  // per device: the attribute is set once per process
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)S::SMEM);
       if (e != cudaSuccess) return e;
-      configured = true;
+      if (dev >= 0 && dev < 64) configured[dev] = true;
     }
-    kern<<<grid, kScoreThreads, S::SMEM, s>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(kScoreThreads, 1, 1);
+    cfg.dynamicSmemBytes = S::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, p);
   }
 }
 
 template <int D, int LAYOUT>
-static cudaError_t dispatch_g(const ScoreParams &p, int G, int grid, cudaStream_t s) {
+static cudaError_t dispatch_g(const ScoreParams &p, int G, int grid, cudaStream_t s, bool pdl) {
   switch (G) {
-    case 1: return launch_one<D, 1, LAYOUT>(p, grid, s);
-    case 2: return launch_one<D, 2, LAYOUT>(p, grid, s);
-    case 4: return launch_one<D, 4, LAYOUT>(p, grid, s);
-    case 8: return launch_one<D, 8, LAYOUT>(p, grid, s);
-    case 16: return launch_one<D, 16, LAYOUT>(p, grid, s);
+    case 1: return launch_one<D, 1, LAYOUT>(p, grid, s, pdl);
+    case 2: return launch_one<D, 2, LAYOUT>(p, grid, s, pdl);
+    case 4: return launch_one<D, 4, LAYOUT>(p, grid, s, pdl);
+    case 8: return launch_one<D, 8, LAYOUT>(p, grid, s, pdl);
+    case 16: return launch_one<D, 16, LAYOUT>(p, grid, s, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -316,18 +401,18 @@ bool score_supported(int D, int G, int layout) {
 int score_tile_keys(int D) { return kScoreTileBytes / (2 * D); }
 
 cudaError_t launch_score(const ScoreParams &p, int D, int G, int layout, int grid,
-                         cudaStream_t s) {
+                         cudaStream_t s, bool pdl) {
   if (layout == TRIA_ROPE_HALF_SPLIT) {
     switch (D) {
-      case 64: return dispatch_g<64, TRIA_ROPE_HALF_SPLIT>(p, G, grid, s);
-      case 128: return dispatch_g<128, TRIA_ROPE_HALF_SPLIT>(p, G, grid, s);
-      case 256: return dispatch_g<256, TRIA_ROPE_HALF_SPLIT>(p, G, grid, s);
+      case 64: return dispatch_g<64, TRIA_ROPE_HALF_SPLIT>(p, G, grid, s, pdl);
+      case 128: return dispatch_g<128, TRIA_ROPE_HALF_SPLIT>(p, G, grid, s, pdl);
+      case 256: return dispatch_g<256, TRIA_ROPE_HALF_SPLIT>(p, G, grid, s, pdl);
     }
   } else {
     switch (D) {
-      case 64: return dispatch_g<64, TRIA_ROPE_INTERLEAVED>(p, G, grid, s);
-      case 128: return dispatch_g<128, TRIA_ROPE_INTERLEAVED>(p, G, grid, s);
-      case 256: return dispatch_g<256, TRIA_ROPE_INTERLEAVED>(p, G, grid, s);
+      case 64: return dispatch_g<64, TRIA_ROPE_INTERLEAVED>(p, G, grid, s, pdl);
+      case 128: return dispatch_g<128, TRIA_ROPE_INTERLEAVED>(p, G, grid, s, pdl);
+      case 256: return dispatch_g<256, TRIA_ROPE_INTERLEAVED>(p, G, grid, s, pdl);
     }
   }
   return cudaErrorInvalidValue;

@@ -27,8 +27,10 @@ constexpr int kScoreThreads = (kScoreConsumerWarps + 1) * 32;
 constexpr int kScoreStages = 4;
 constexpr int kScoreTileBytes = 32 * 1024;   // bytes of K per pipeline stage
 
-constexpr int kUnitThreads = 512;
-constexpr int kUnitSmemBytes = 200 * 1024;
+constexpr int kUnitThreads = 256;
+constexpr int kUnitCluster = 8;
+constexpr int kUnitSmemSmall = 112 * 1024;  // two CTAs per SM
+constexpr int kUnitSmemLarge = 200 * 1024;  // one CTA per SM
 
 struct FoldParams {
   const int32_t *cur_pos;   // [B]
@@ -48,8 +50,8 @@ struct ScoreParams {
   const float2 *centre;     // [L][Hq][F]
   const float *mean_norm;   // [L][Hq][F]
   const float *mrl;         // [L][Hq][F]
-  const double2 *ea;        // [B][F]
-  const int32_t *seqlen;    // [B] snapshot
+  const double2 *ea;        // [B][F]  (written by the fold kernel)
+  const int32_t *seq_len;   // [B] caller's live lengths (not modified during the call)
   float *raw;               // [L][Hq][cap]
   int32_t *err;
   int64_t cap;
@@ -79,17 +81,19 @@ struct UnitParams {
   int32_t L, Hkv, Hq, B, G, D, budget;
   int32_t mode;
   int32_t write_short_sel;  // prune: also write identity lists for sequences not pruned
+  int32_t smem_bytes;       // dynamic shared memory of the launch
   int64_t seg_start[TRIA_MAX_BATCH + 1];
 };
 
 // ------------------------------------------------------------------ launchers (host)
 cudaError_t launch_fold(const FoldParams &p, int F, cudaStream_t s);
 cudaError_t launch_score(const ScoreParams &p, int D, int G, int layout, int grid,
-                         cudaStream_t s);
+                         cudaStream_t s, bool pdl);
 bool score_supported(int D, int G, int layout);
 int score_tile_keys(int D);
-cudaError_t launch_unit(const UnitParams &p, int units, cudaStream_t s);
+cudaError_t launch_unit(const UnitParams &p, int units, cudaStream_t s, bool pdl);
 int unit_cluster_size();
+int unit_smem_bytes(int units, int64_t max_segment);
 cudaError_t launch_calibrate(const void *q, int q_dtype, int64_t L, int64_t N, int64_t Hq,
                              int64_t D, int layout, float *centre, float *mean_norm, float *mrl,
                              cudaStream_t s);
@@ -166,6 +170,13 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f == 0.0f ? 0.0f : f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+
+// Programmatic dependent launch: let the next kernel of the stream start / wait
+// until the previous kernel of the stream has completed and its writes are visible.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ void set_error(int32_t *err, int32_t bit) {
   atomicOr(reinterpret_cast<int *>(err), bit);

@@ -3,24 +3,30 @@
 //
 //   z-score + group max (romaanj.github.io review, "Method"; dimensionstp.github.io
 //     review, section 3-2 (6)): mu_h and the population sigma_h of the raw
-//     scores over the sequence's T live keys (two passes, float64 sums reduced
-//     across the cluster in rank order, so the result is deterministic);
-//     z_h = (s_h - mu_h) / sigma_h (0 when sigma_h = 0); score = max_h z_h.
+//     scores over the sequence's T live keys; z_h = (s_h - mu_h) / sigma_h
+//     (0 when sigma_h = 0); score = max_h z_h.  The sums are float64, taken
+//     about a pivot (the unit's first raw score) so that a large mean does not
+//     cancel the variance, and reduced across the cluster in rank order, so the
+//     result is deterministic.
 //   selection (same sources, "prune back to budget"; section 3-2 (5)): the
 //     `budget` largest scores, ties to the lower slot, by a 4-pass 8-bit radix
-//     select on order-preserving 32-bit keys.  Each CTA histograms its slice;
-//     every CTA then sums the cluster's histograms through distributed shared
-//     memory, so all agree on the threshold without a global round trip.
-//     The kept slots are emitted in ascending order.
+//     select on order-preserving 32-bit keys.  Each CTA histograms its slice in
+//     shared memory; every CTA then sums the cluster's histograms through
+//     distributed shared memory (all peers read in parallel), so all agree on
+//     the threshold without a global round trip.  Kept slots are emitted in
+//     ascending order.
 //   compaction (eviction): kept rows of K, V and pos move in place to slots
 //     [0, kept).  A kept slot s_j always satisfies s_j >= j, so reading every
 //     source of a batch of destinations before any of them is written (one
 //     cluster barrier per batch) makes the in-place gather race-free: a
 //     destination row j can only be the source of a kept key with index <= j,
-//     which belongs to this batch or an earlier one.
+//     which belongs to this batch or an earlier one.  Rows move through shared
+//     memory with 1-D bulk copies (cp.async.bulk) in both directions.
 //
-// Cluster barriers are hardware barriers (barrier.cluster); there are no
-// spin-waits in this kernel.
+// Cluster barriers are hardware barriers; the only other waits are on this
+// CTA's own bulk copies and are bounded.  The kernel is launched as a
+// programmatic dependent of the score kernel and waits for it
+// (griddepcontrol.wait) before reading anything that kernel or the fold wrote.
 #include <cooperative_groups.h>
 
 #include "tria_internal.cuh"
@@ -31,35 +37,33 @@ namespace tria {
 
 namespace {
 
-constexpr int kCtl = 8 * 1024;  // control region at the start of shared memory
+constexpr int kCtl = 12 * 1024;  // control region at the start of shared memory
 constexpr int kMaxG = 16;
+constexpr int kMaxCluster = 16;
 constexpr int kWarps = kUnitThreads / 32;
 
 struct Ctl {
+  uint64_t cbar;                    // compaction bulk-load barrier
   uint32_t hist[2][256];
   uint32_t tot[256];
-  double part[2][kMaxG];   // this CTA's partial sums (pass 0: s, pass 1: (s - mu)^2)
+  double part[kMaxG][2];            // this CTA's shifted sums: sum(s - p), sum((s - p)^2)
+  double gath[kMaxCluster][kMaxG][2];
+  double wred[kWarps][kMaxG][2];
   double mu[kMaxG];
   double inv_sigma[kMaxG];
-  double wred[kWarps][kMaxG];
-  int32_t cnt[4];          // gt, eq (selection) / first_neg, bad (compaction check)
-  int32_t bc[8];           // broadcast scalars
-  int32_t scan[2][kWarps + 1];
+  float pivot[kMaxG];
+  int32_t cnt[4];                   // gt, eq of this CTA / first_neg, bad (compaction check)
+  int32_t peer_cnt[kMaxCluster][2];
+  int32_t bc[8];                    // broadcast scalars
+  int32_t scan[kWarps + 1];
 };
 static_assert(sizeof(Ctl) <= kCtl, "control region too small");
 
-__device__ __forceinline__ double block_sum_d(double v, double *wred_col, int stride) {
-  // returns the block sum in thread 0 only; wred_col[w * stride]
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) wred_col[warp * stride] = v;
-  return v;
-}
-
-// exclusive block scan of one int per thread; returns the exclusive prefix and the total
+// Exclusive block scan of one int per thread; also returns the block total.
 __device__ __forceinline__ int block_excl_scan(int v, int32_t *wtot, int *total) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int incl = v;
+#pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int t = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += t;
@@ -67,8 +71,9 @@ __device__ __forceinline__ int block_excl_scan(int v, int32_t *wtot, int *total)
   if (lane == 31) wtot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = lane < kWarps ? wtot[lane] : 0;
+    const int w = lane < kWarps ? wtot[lane] : 0;
     int wi = w;
+#pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int t = __shfl_up_sync(0xffffffffu, wi, o);
       if (lane >= o) wi += t;
@@ -79,13 +84,50 @@ __device__ __forceinline__ int block_excl_scan(int v, int32_t *wtot, int *total)
   __syncthreads();
   const int out = wtot[warp] + incl - v;
   *total = wtot[kWarps];
-  __syncthreads();
   return out;
 }
 
+// 4-byte asynchronous global -> shared copies (any 4-byte alignment) ...
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dev::smem_addr(dst)), "l"(src)
+               : "memory");
+}
+// ... and 16-byte ones for 16-byte aligned runs.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dev::smem_addr(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Copies n floats global -> shared with asynchronous copies (waited by the caller).
+__device__ __forceinline__ void stage_floats(float *dst, const float *src, int n) {
+  const bool vec = ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) == 0;
+  if (vec) {
+    const int n4 = n >> 2;
+    for (int i = threadIdx.x; i < n4; i += blockDim.x) cp_async16(dst + 4 * i, src + 4 * i);
+    for (int i = 4 * n4 + threadIdx.x; i < n; i += blockDim.x) cp_async4(dst + i, src + i);
+  } else {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) cp_async4(dst + i, src + i);
+  }
+}
+
+// 1-D bulk copy shared -> global (bulk-group completion).
+__device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(dev::smem_addr(src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 }  // namespace
 
-__global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_constant__ UnitParams p) {
+__global__ void __launch_bounds__(kUnitThreads, 2) unit_kernel(const __grid_constant__ UnitParams p) {
   cg::cluster_group cl = cg::this_cluster();
   const int CL = (int)cl.num_blocks();
   const int r = (int)cl.block_rank();
@@ -98,18 +140,27 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
   const int64_t seg_cap = p.seg_start[b + 1] - seg;
   const int G = p.G;
   const int tid = threadIdx.x, nthr = blockDim.x;
+  const int warp = tid >> 5, lane = tid & 31;
 
   extern __shared__ __align__(128) uint8_t smem[];
   Ctl &c = *reinterpret_cast<Ctl *>(smem);
   uint8_t *data = smem + kCtl;
-  const size_t data_bytes = (size_t)kUnitSmemBytes - kCtl;
+  const size_t data_bytes = (size_t)p.smem_bytes - kCtl;
   int32_t *sel = p.sel + (row * p.B + b) * (int64_t)p.budget;
 
+  if (tid == 0) {
+    dev::mbar_init(&c.cbar, (uint32_t)nthr);
+    dev::fence_mbar_init();
+  }
+  for (int i = tid; i < 256; i += nthr) c.hist[0][i] = 0;
+  __syncthreads();
+  dev::pdl_wait();
+
   int kept = 0;
-  // ------------------------------------------------------------ compaction only
   if (p.mode == kModeCompact) {
+    // ------------------------------------------------------------ check the list
     const int64_t j0 = (int64_t)p.budget * r / CL, j1 = (int64_t)p.budget * (r + 1) / CL;
-    int first_neg = (int)j1, bad = 0;
+    int first_neg = p.budget, bad = 0;  // index of the first -1 (budget if none)
     for (int64_t j = j0 + tid; j < j1; j += nthr) {
       const int32_t s = __ldcg(sel + j);
       const int32_t prev = j > 0 ? __ldcg(sel + j - 1) : -1;
@@ -117,19 +168,23 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       if (s >= 0 && j > 0 && (prev < 0 || s <= prev)) bad = 1;  // ascending, no slot after a -1
       if (s < 0) first_neg = min(first_neg, (int)j);
     }
-    if (tid == 0) { c.cnt[2] = (int)j1; c.cnt[3] = 0; }
+    if (tid == 0) { c.cnt[2] = p.budget; c.cnt[3] = 0; }
     __syncthreads();
     atomicMin(&c.cnt[2], first_neg);
     if (bad) atomicOr(&c.cnt[3], 1);
     cl.sync();
+    if (tid < CL) {
+      const Ctl *peer = cl.map_shared_rank(&c, tid);
+      c.peer_cnt[tid][0] = peer->cnt[2];
+      c.peer_cnt[tid][1] = peer->cnt[3];
+    }
+    cl.sync();  // peers' control regions are not read after this point
     int any_bad = 0;
     kept = p.budget;
     for (int q = 0; q < CL; ++q) {
-      const Ctl *peer = cl.map_shared_rank(&c, q);
-      kept = min(kept, peer->cnt[2]);
-      any_bad |= peer->cnt[3];
+      kept = min(kept, c.peer_cnt[q][0]);
+      any_bad |= c.peer_cnt[q][1];
     }
-    cl.sync();  // peers' control regions are no longer read after this point
     if (any_bad) {
       if (r == 0 && tid == 0) dev::set_error(p.err, TRIA_DEVERR_SELECTION);
       return;
@@ -153,7 +208,8 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     const int64_t lo = (int64_t)T * r / CL, hi = (int64_t)T * (r + 1) / CL;
     const int n = (int)(hi - lo);
     const int nmax = (int)((T + CL - 1) / CL);
-    if ((size_t)nmax * 4 > data_bytes) {
+    const int nmax4 = (nmax + 3) & ~3;
+    if ((size_t)nmax4 * 4 > data_bytes) {
       if (r == 0 && tid == 0) dev::set_error(p.err, TRIA_DEVERR_SEGMENT_BIG);
       return;  // every CTA of the cluster takes this branch (same T)
     }
@@ -161,54 +217,51 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
 
     if (p.mode == kModeZmax || p.mode == kModePrune) {
       // ---------------------------------------------------- z-score statistics
-      const bool cache = (size_t)(G + 1) * nmax * 4 <= data_bytes;
-      float *rawc = reinterpret_cast<float *>(data) + nmax;  // [G][nmax]
+      const bool cache = (size_t)(G + 1) * nmax4 * 4 <= data_bytes;
+      float *rawc = reinterpret_cast<float *>(data) + nmax4;  // [G][nmax4]
       const float *rawu = p.raw + ((int64_t)l * p.Hq + (int64_t)g * G) * p.cap + seg;
-      for (int j = 0; j < G; ++j) {
-        const float *s = rawu + (int64_t)j * p.cap;
-        double acc = 0.0;
-        for (int i = tid; i < n; i += nthr) {
-          const float v = s[lo + i];
-          if (cache) rawc[(size_t)j * nmax + i] = v;
-          acc += (double)v;
-        }
-        block_sum_d(acc, &c.wred[0][j], kMaxG);
+      if (cache) {
+        for (int j = 0; j < G; ++j) stage_floats(rawc + (size_t)j * nmax4, rawu + (int64_t)j * p.cap + lo, n);
+        cp_async_wait_all();
       }
-      __syncthreads();
-      if (tid < G) {
-        double a = 0.0;
-        for (int w = 0; w < kWarps; ++w) a += c.wred[w][tid];
-        c.part[0][tid] = a;
-      }
-      cl.sync();
-      if (tid < G) {
-        double a = 0.0;
-        for (int q = 0; q < CL; ++q) a += cl.map_shared_rank(&c, q)->part[0][tid];
-        c.mu[tid] = a / (double)T;
-      }
+      if (tid < G) c.pivot[tid] = rawu[(int64_t)tid * p.cap];
       __syncthreads();
       for (int j = 0; j < G; ++j) {
-        const float *s = rawu + (int64_t)j * p.cap;
-        const double mu = c.mu[j];
-        double acc = 0.0;
+        const double pv = (double)c.pivot[j];
+        double a1 = 0.0, a2 = 0.0;
         for (int i = tid; i < n; i += nthr) {
-          const double d = (double)(cache ? rawc[(size_t)j * nmax + i] : s[lo + i]) - mu;
-          acc += d * d;
+          const float v = cache ? rawc[(size_t)j * nmax4 + i] : rawu[(int64_t)j * p.cap + lo + i];
+          const double d = (double)v - pv;
+          a1 += d;
+          a2 = fma(d, d, a2);
         }
-        block_sum_d(acc, &c.wred[0][j], kMaxG);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+          a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+        }
+        if (lane == 0) { c.wred[warp][j][0] = a1; c.wred[warp][j][1] = a2; }
+      }
+      __syncthreads();
+      if (tid < 2 * G) {
+        const int j = tid >> 1, k = tid & 1;
+        double a = 0.0;
+        for (int w = 0; w < kWarps; ++w) a += c.wred[w][j][k];
+        c.part[j][k] = a;
+      }
+      cl.sync();
+      for (int t = tid; t < CL * 2 * G; t += nthr) {
+        const int q = t / (2 * G), j = (t >> 1) % G, k = t & 1;
+        c.gath[q][j][k] = cl.map_shared_rank(&c, q)->part[j][k];
       }
       __syncthreads();
       if (tid < G) {
-        double a = 0.0;
-        for (int w = 0; w < kWarps; ++w) a += c.wred[w][tid];
-        c.part[1][tid] = a;
-      }
-      cl.sync();
-      if (tid < G) {
-        double a = 0.0;
-        for (int q = 0; q < CL; ++q) a += cl.map_shared_rank(&c, q)->part[1][tid];
-        const double sigma = sqrt(a / (double)T);
-        c.inv_sigma[tid] = sigma > 0.0 ? 1.0 / sigma : 0.0;
+        double s1 = 0.0, s2 = 0.0;
+        for (int q = 0; q < CL; ++q) { s1 += c.gath[q][tid][0]; s2 += c.gath[q][tid][1]; }
+        const double m1 = s1 / (double)T;
+        const double var = s2 / (double)T - m1 * m1;
+        c.mu[tid] = (double)c.pivot[tid] + m1;
+        c.inv_sigma[tid] = var > 0.0 ? 1.0 / sqrt(var) : 0.0;
       }
       __syncthreads();
       // ---------------------------------------------------- z and group max
@@ -216,7 +269,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       for (int i = tid; i < n; i += nthr) {
         double zmax = -1.0e300;
         for (int j = 0; j < G; ++j) {
-          const float v = cache ? rawc[(size_t)j * nmax + i] : rawu[(int64_t)j * p.cap + lo + i];
+          const float v = cache ? rawc[(size_t)j * nmax4 + i] : rawu[(int64_t)j * p.cap + lo + i];
           const double z = ((double)v - c.mu[j]) * c.inv_sigma[j];
           zmax = z > zmax ? z : zmax;
         }
@@ -232,25 +285,38 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       const float *score = p.score + row * p.cap + seg;
       for (int i = tid; i < n; i += nthr) zkey[i] = dev::order_key(score[lo + i]);
     }
+    for (int i = n + tid; i < nmax4; i += nthr) zkey[i] = 0u;  // padding never matches a prefix
     __syncthreads();
 
     // ------------------------------------------------------------ radix select
+    // hist[0] was zeroed at kernel start; each pass zeroes the other buffer for
+    // the next pass after the cluster barrier (peers finished reading it then).
     uint32_t prefix = 0, mask = 0;
     int krem = p.budget;
+    const uint4 *zkey4 = reinterpret_cast<const uint4 *>(zkey);
+    const int n4 = nmax4 >> 2;
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
       uint32_t *H = c.hist[pass & 1];
-      for (int i = tid; i < 256; i += nthr) H[i] = 0;
-      __syncthreads();
-      for (int i = tid; i < n; i += nthr) {
-        const uint32_t key = zkey[i];
-        if ((key & mask) == prefix) atomicAdd(&H[(key >> shift) & 255u], 1u);
+      for (int i = tid; i < n4; i += nthr) {
+        const uint4 kv = zkey4[i];
+        const uint32_t ks[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          // padding keys are 0: they match only while prefix == 0 and mask == 0
+          if ((ks[e] & mask) == prefix && 4 * i + e < n) atomicAdd(&H[(ks[e] >> shift) & 255u], 1u);
+        }
       }
       cl.sync();
       for (int i = tid; i < 256; i += nthr) {
+        uint32_t v[kMaxCluster];
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) v[q] = q < CL ? cl.map_shared_rank(H, q)[i] : 0u;
         uint32_t a = 0;
-        for (int q = 0; q < CL; ++q) a += cl.map_shared_rank(H, q)[i];
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) a += v[q];
         c.tot[i] = a;
+        c.hist[(pass + 1) & 1][i] = 0;
       }
       __syncthreads();
       if (tid < 32) {
@@ -258,6 +324,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
 #pragma unroll
         for (int i = 0; i < 8; ++i) { cnt8[i] = c.tot[tid * 8 + i]; s += cnt8[i]; }
         uint32_t incl = s;  // inclusive suffix over lanes (this lane and above)
+#pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const uint32_t t = __shfl_down_sync(0xffffffffu, incl, o);
           if (tid + o < 32) incl += t;
@@ -276,11 +343,9 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
         }
       }
       __syncthreads();
-      const uint32_t d = (uint32_t)c.bc[0];
-      krem = c.bc[1];
-      prefix |= d << shift;
+      prefix |= (uint32_t)c.bc[0] << shift;
       mask |= 255u << shift;
-      __syncthreads();
+      krem = c.bc[1];
     }
     const uint32_t thr = prefix;
     const int k_eq = krem;  // keys equal to thr that are kept (the lowest slots)
@@ -294,34 +359,35 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       gt += key > thr;
       eq += key == thr;
     }
-    int tot_gt, tot_eq;
-    const int gt_x = block_excl_scan(gt, c.scan[0], &tot_gt);
-    const int eq_x = block_excl_scan(eq, c.scan[1], &tot_eq);
-    (void)gt_x;
-    if (tid == 0) { c.cnt[0] = tot_gt; c.cnt[1] = tot_eq; }
+    int tot_pk;
+    const int x_pk = block_excl_scan((gt << 16) | eq, c.scan, &tot_pk);  // n < 65536
+    const int gt_x = x_pk >> 16, eq_x = x_pk & 0xffff;
+    if (tid == 0) { c.cnt[0] = tot_pk >> 16; c.cnt[1] = tot_pk & 0xffff; }
     cl.sync();
+    if (tid < CL) {
+      const Ctl *peer = cl.map_shared_rank(&c, tid);
+      c.peer_cnt[tid][0] = peer->cnt[0];
+      c.peer_cnt[tid][1] = peer->cnt[1];
+    }
+    __syncthreads();
     if (tid == 0) {
       int eqb = 0, base = 0;
       for (int q = 0; q < CL; ++q) {
-        const Ctl *peer = cl.map_shared_rank(&c, q);
-        const int qg = peer->cnt[0], qe = peer->cnt[1];
+        const int qg = c.peer_cnt[q][0], qe = c.peer_cnt[q][1];
         const int take = max(0, min(qe, k_eq - eqb));
-        if (q == r) { c.bc[2] = eqb; c.bc[3] = base; }
+        if (q == r) { c.bc[2] = base; c.bc[3] = take; }
         eqb += qe;
         base += qg + take;
       }
     }
     __syncthreads();
-    const int eq_before = c.bc[2] + eq_x;
-    const int take = max(0, min(eq, k_eq - eq_before));
-    int dummy;
-    const int out0 = c.bc[3] + block_excl_scan(gt + take, c.scan[0], &dummy);
     {
-      int o = out0, er = eq_before;
+      const int take_cta = c.bc[3];  // equal keys this CTA keeps: its first take_cta ones
+      int o = c.bc[2] + gt_x + min(eq_x, take_cta), er = eq_x;
       for (int i = a0; i < a1; ++i) {
         const uint32_t key = zkey[i];
         bool keep = key > thr;
-        if (key == thr) { keep = er < k_eq; ++er; }
+        if (key == thr) { keep = er < take_cta; ++er; }
         if (keep) {
           if (o < p.budget) sel[o] = (int32_t)(lo + i);
           ++o;
@@ -335,100 +401,141 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
   }
 
   // -------------------------------------------------------------- in-place compaction
-  const int ROW = 2 * p.D;                 // bytes per K or V row
-  const int VPR = ROW / 16;                // 16-byte vectors per row
-  const int row_bytes = 2 * ROW + 4;       // staged K + V + pos
-  const int cap_rows = (int)(data_bytes / row_bytes);
-  const int64_t j0 = (int64_t)p.budget * r / CL, j1 = (int64_t)p.budget * (r + 1) / CL;
-  const int range_max = (p.budget + CL - 1) / CL;
-  const int batches = (range_max + cap_rows - 1) / cap_rows;
-  uint4 *sk = reinterpret_cast<uint4 *>(data);                    // [cap_rows][VPR]
-  uint4 *sv = sk + (size_t)cap_rows * VPR;                         // [cap_rows][VPR]
-  int32_t *sp = reinterpret_cast<int32_t *>(sv + (size_t)cap_rows * VPR);  // [cap_rows]
+  const int ROW = 2 * p.D;                          // bytes per K or V row
+  constexpr int kPosPerThread = 4;                   // rows a thread handles per batch
+  const int cap_rows = min((int)(data_bytes / (2 * (size_t)ROW)), kPosPerThread * nthr);
+  // Batch bt covers the destinations [bt * CL * cap_rows, (bt + 1) * CL * cap_rows) of the
+  // whole cluster (CTA r takes the r-th chunk), so every destination written in a batch
+  // precedes every destination, and hence every source, of the batches after it.
+  const int64_t per_batch = (int64_t)CL * cap_rows;
+  const int batches = (int)((kept + per_batch - 1) / per_batch);
   const int64_t rbase = row * p.cap + seg;
-  uint4 *kg4 = reinterpret_cast<uint4 *>(p.k + (size_t)rbase * ROW);
-  uint4 *vg4 = reinterpret_cast<uint4 *>(p.v + (size_t)rbase * ROW);
+  uint8_t *kg = p.k + (size_t)rbase * ROW;
+  uint8_t *vg = p.v + (size_t)rbase * ROW;
   int32_t *pg = p.pos + rbase;
+  uint8_t *sk = data;                                // [cap_rows][ROW]
+  uint8_t *sv = data + (size_t)cap_rows * ROW;       // [cap_rows][ROW]
+  bool failed = false;
   for (int bt = 0; bt < batches; ++bt) {
-    const int64_t a = j0 + (int64_t)bt * cap_rows;
+    const int64_t a = (int64_t)bt * per_batch + (int64_t)r * cap_rows;
     int64_t e = a + cap_rows;
-    if (e > j1) e = j1;
     if (e > kept) e = kept;
     const int nb = e > a ? (int)(e - a) : 0;
-    for (int idx = tid; idx < nb * VPR; idx += nthr) {
-      const int jj = idx / VPR, v = idx - jj * VPR;
-      const int32_t s = __ldcg(sel + a + jj);
-      if (s < 0 || s >= seg_cap) {  // cannot happen for a well-formed list; never read outside
-        if (v == 0) dev::set_error(p.err, TRIA_DEVERR_SELECTION);
-        continue;
+    int32_t src[kPosPerThread], rp[kPosPerThread];
+    uint32_t bytes = 0;
+#pragma unroll
+    for (int u = 0; u < kPosPerThread; ++u) {
+      const int jj = tid + u * nthr;
+      src[u] = -1;
+      if (jj < nb) {
+        const int32_t s = __ldcg(sel + a + jj);
+        if (s >= 0 && s < seg_cap) {
+          if (s != a + jj) { src[u] = s; bytes += 2u * ROW; }
+        } else {
+          dev::set_error(p.err, TRIA_DEVERR_SELECTION);
+        }
       }
-      if (s != a + jj) {
-        sk[(size_t)jj * VPR + v] = kg4[(size_t)s * VPR + v];
-        sv[(size_t)jj * VPR + v] = vg4[(size_t)s * VPR + v];
-        if (v == 0) sp[jj] = pg[s];
+    }
+    if (!failed) {
+      dev::mbar_arrive_expect_tx(&c.cbar, bytes);
+#pragma unroll
+      for (int u = 0; u < kPosPerThread; ++u) {
+        if (src[u] >= 0) {
+          const int jj = tid + u * nthr;
+          dev::bulk_g2s(sk + (size_t)jj * ROW, kg + (size_t)src[u] * ROW, ROW, &c.cbar);
+          dev::bulk_g2s(sv + (size_t)jj * ROW, vg + (size_t)src[u] * ROW, ROW, &c.cbar);
+          rp[u] = pg[src[u]];
+        }
+      }
+      if (!dev::mbar_wait(&c.cbar, bt & 1)) {
+        dev::set_error(p.err, TRIA_DEVERR_TIMEOUT);
+        failed = true;
       }
     }
     cl.sync();  // every source row of this batch has been read, cluster-wide
-    for (int idx = tid; idx < nb * VPR; idx += nthr) {
-      const int jj = idx / VPR, v = idx - jj * VPR;
-      const int32_t s = __ldcg(sel + a + jj);
-      if (s >= 0 && s < seg_cap && s != a + jj) {
-        kg4[(size_t)(a + jj) * VPR + v] = sk[(size_t)jj * VPR + v];
-        vg4[(size_t)(a + jj) * VPR + v] = sv[(size_t)jj * VPR + v];
-        if (v == 0) pg[a + jj] = sp[jj];
+    if (!failed) {
+#pragma unroll
+      for (int u = 0; u < kPosPerThread; ++u) {
+        if (src[u] >= 0) {
+          const int jj = tid + u * nthr;
+          bulk_s2g(kg + (size_t)(a + jj) * ROW, sk + (size_t)jj * ROW, ROW);
+          bulk_s2g(vg + (size_t)(a + jj) * ROW, sv + (size_t)jj * ROW, ROW);
+          pg[a + jj] = rp[u];
+        }
       }
+      bulk_commit();
+      bulk_wait_read0();  // this thread's staged rows may be overwritten by the next batch
     }
-    __syncthreads();  // staging buffer reused by the next batch
+    __syncthreads();
   }
+  bulk_wait0();
   if (r == 0 && tid == 0 && l == 0 && g == 0) p.seq_len_out[b] = kept;
 }
 
-static int g_cluster[64];  // per device: chosen cluster size (0 = not yet chosen)
+// Launch configuration: 8-CTA clusters (portable; 15 fit at once with the large
+// shared-memory size, 33 with the small one); the large size is used when one
+// wave holds every unit or a segment needs it.
+namespace {
+struct UnitCfg {
+  int max_small = 0, max_large = 0;
+  bool ready = false;
+};
+UnitCfg g_unit_cfg[64];
 
-int unit_cluster_size() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
-  if (g_cluster[dev]) return g_cluster[dev];
-  cudaFuncSetAttribute(unit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUnitSmemBytes);
-  cudaFuncSetAttribute(unit_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  int chosen = 8;
-  for (int cs : {16, 8}) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cs, 1, 1);
-    cfg.blockDim = dim3(kUnitThreads, 1, 1);
-    cfg.dynamicSmemBytes = kUnitSmemBytes;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = cs;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, unit_kernel, &cfg) == cudaSuccess && n > 0) {
-      chosen = cs;
-      break;
-    }
-    cudaGetLastError();
-  }
-  g_cluster[dev] = chosen;
-  return chosen;
-}
-
-cudaError_t launch_unit(const UnitParams &p, int units, cudaStream_t s) {
-  const int cs = unit_cluster_size();
+int max_clusters(int smem) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)units * cs, 1, 1);
+  cfg.gridDim = dim3(kUnitCluster, 1, 1);
   cfg.blockDim = dim3(kUnitThreads, 1, 1);
-  cfg.dynamicSmemBytes = kUnitSmemBytes;
-  cfg.stream = s;
+  cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = cs;
+  attr.val.clusterDim.x = kUnitCluster;
   attr.val.clusterDim.y = 1;
   attr.val.clusterDim.z = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, unit_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 1;
+  }
+  return n > 0 ? n : 1;
+}
+}  // namespace
+
+int unit_cluster_size() { return kUnitCluster; }
+
+int unit_smem_bytes(int units, int64_t max_segment) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  UnitCfg &uc = g_unit_cfg[dev];
+  if (!uc.ready) {
+    cudaFuncSetAttribute(unit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUnitSmemLarge);
+    uc.max_small = max_clusters(kUnitSmemSmall);
+    uc.max_large = max_clusters(kUnitSmemLarge);
+    uc.ready = true;
+  }
+  const int64_t keys_per_cta = (max_segment + kUnitCluster - 1) / kUnitCluster;
+  const bool need_large = (keys_per_cta + 4) * 4 + 12 * 1024 > kUnitSmemSmall;
+  return (need_large || units <= uc.max_large) ? kUnitSmemLarge : kUnitSmemSmall;
+}
+
+cudaError_t launch_unit(const UnitParams &p, int units, cudaStream_t s, bool pdl) {
+  const int cs = kUnitCluster;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)units * cs, 1, 1);
+  cfg.blockDim = dim3(kUnitThreads, 1, 1);
+  cfg.dynamicSmemBytes = p.smem_bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, unit_kernel, p);
 }
 

@@ -241,6 +241,9 @@ def tria_prune(cfg: Config, stats: Stats, cache: Cache, ws: torch.Tensor,
 def tria_prune_profiled(cfg: Config, stats: Stats, cache: Cache, ws: torch.Tensor, events,
                         sel_out: Optional[torch.Tensor] = None, stream=None) -> int:
     """events: PRUNE_MAX_STAGES + 1 torch.cuda.Event(enable_timing=True); returns n_stages."""
+    for e in events:
+        if not e.cuda_event:  # torch creates the CUDA event on its first record
+            e.record(stream if stream is not None else torch.cuda.current_stream())
     arr = (ctypes.c_void_p * (PRUNE_MAX_STAGES + 1))(
         *[ctypes.c_void_p(e.cuda_event) for e in events])
     n = ctypes.c_int32(0)

@@ -260,6 +260,38 @@ def test_compact_in_place_is_bit_exact(kind):
     np.testing.assert_array_equal(case.dev["pos"].cpu().numpy(), opos)
 
 
+@pytest.mark.parametrize("kind", ["last", "alternating", "random"])
+def test_compact_many_units_multi_batch(kind):
+    """More units than fit in one wave of clusters: the kernel stages fewer rows
+    per batch, so a 2000-row budget needs two cluster-wide batches."""
+    wl = small("compact-multi", L=2, Hq=32, Hkv=8, B=1, seq_lens=[2500], budget=2000)
+    case = Case(wl)
+    rng = np.random.default_rng(11)
+    sel = np.stack([np.stack([np.stack([_adversarial_sel(kind, T, wl.budget, rng)
+                                        for T in case.lens]) for _ in range(wl.n_kv_heads)])
+                    for _ in range(wl.num_layers)])
+    tria.tria_compact(case.cfg, case.cache, torch.from_numpy(sel).cuda(), case.ws)
+    torch.cuda.synchronize()
+    assert tria.tria_get_device_error(case.ws) == 0
+    assert case.dev["seq_len"].cpu().tolist() == [2000]
+    check_compacted(case, sel, [2000])
+
+
+def test_prune_many_units_matches_oracle():
+    case = Case(small("prune-multi", L=2, Hq=32, Hkv=8, B=1, seq_lens=[2500], budget=2000,
+                      offsets=range(1, 17)))
+    wl = case.wl
+    ref = oracle.prune(case.prob, common.bf16_bits(case.host["v"]))
+    sel = torch.empty((wl.num_layers, wl.n_kv_heads, wl.batch, wl.budget), dtype=torch.int32,
+                      device="cuda")
+    tria.tria_prune(case.cfg, case.stats, case.cache, case.ws, sel_out=sel)
+    torch.cuda.synchronize()
+    assert tria.tria_get_device_error(case.ws) == 0
+    gsel = sel.cpu().numpy()
+    check_selection(gsel, ref["sel"], ref["raw"], ref["score"], case)
+    check_compacted(case, gsel, [2000])
+
+
 def test_compact_rejects_malformed_selection():
     wl = small("badsel", B=2, seq_lens=[300, 300], budget=50)
     case = Case(wl)

@@ -11,16 +11,26 @@ namespace tria {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-WsLayout ws_layout(const tria_config &cfg, int64_t cap) {
+WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap) {
   WsLayout w{};
   const size_t F = (size_t)cfg.head_dim / 2;
+  const int64_t tile = score_tile_keys(cfg.head_dim > 0 ? cfg.head_dim : 2);
+  int64_t max_tiles = 0;
+  for (int b = 0; b < cfg.batch; ++b) {
+    const int64_t t = (seq_start[b + 1] - seq_start[b] + tile - 1) / tile;
+    if (t > max_tiles) max_tiles = t;
+  }
+  w.max_slots = (int32_t)(max_tiles + 1);
+  const size_t units = (size_t)cfg.num_layers * cfg.n_kv_heads * cfg.batch;
+  const size_t G = cfg.n_kv_heads > 0 ? (size_t)(cfg.n_q_heads / cfg.n_kv_heads) : 1;
   size_t o = 0;
   w.err = o;      o += 256;
   w.seqlen = o;   o = align_up(o + 4ull * cfg.batch, 256);
   w.ea = o;       o = align_up(o + 16ull * cfg.batch * F, 256);
   w.raw = o;      o = align_up(o + 4ull * cfg.num_layers * cfg.n_q_heads * (size_t)cap, 256);
   w.score = o;
-  w.sel = o;      o = align_up(o + 4ull * cfg.num_layers * cfg.n_kv_heads * cfg.batch * cfg.budget, 256);
+  w.sel = o;      o = align_up(o + 4ull * units * cfg.budget, 256);
+  w.partials = o; o = align_up(o + 16ull * units * w.max_slots * G, 256);
   w.total = o;
   return w;
 }
@@ -99,7 +109,7 @@ tria_status check_stats(const tria_stats *s) {
 
 tria_status check_ws(const tria_config *cfg, const tria_cache *c, void *ws, size_t bytes) {
   if (!ws || !aligned(ws, 256)) return TRIA_ERR_WORKSPACE;
-  if (bytes < ws_layout(*cfg, c->cap_total).total) return TRIA_ERR_WORKSPACE;
+  if (bytes < ws_layout(*cfg, c->seq_start, c->cap_total).total) return TRIA_ERR_WORKSPACE;
   return TRIA_OK;
 }
 
@@ -124,7 +134,8 @@ void fill_fold(FoldParams &fp, const tria_config *cfg, const tria_cache *c, int3
 
 // Builds the score kernel parameters; returns the grid size (0: nothing to launch).
 int fill_score(ScoreParams &sp, const tria_config *cfg, const tria_stats *st, const tria_cache *c,
-               const double2 *ea, float *raw, int32_t *err, int skip_short) {
+               const double2 *ea, float *raw, double *partials, int32_t max_slots, int32_t *err,
+               int skip_short) {
   std::memset(&sp, 0, sizeof sp);
   const int tile = score_tile_keys(cfg->head_dim);
   sp.k = static_cast<const uint8_t *>(c->k);
@@ -134,6 +145,8 @@ int fill_score(ScoreParams &sp, const tria_config *cfg, const tria_stats *st, co
   sp.ea = ea;
   sp.seq_len = c->seq_len;
   sp.raw = raw;
+  sp.partials = partials;
+  sp.max_slots = max_slots;
   sp.err = err;
   sp.cap = c->cap_total;
   sp.L = cfg->num_layers;
@@ -182,6 +195,17 @@ void fill_unit(UnitParams &up, const tria_config *cfg, const tria_cache *c, int 
   up.smem_bytes = unit_smem_bytes(cfg->num_layers * cfg->n_kv_heads * cfg->batch, max_seg);
 }
 
+// The unit kernel finds the score kernel's partial sums through its tile decomposition.
+void link_unit_to_score(UnitParams &up, const ScoreParams &sp, const double *partials,
+                        int tile_keys) {
+  up.partials = partials;
+  up.max_slots = sp.max_slots;
+  up.tiles_per_cta = sp.tiles_per_cta > 0 ? sp.tiles_per_cta : 1;
+  up.tiles_per_row = sp.tiles_per_row;
+  up.tile_keys = tile_keys;
+  for (int b = 0; b <= TRIA_MAX_BATCH; ++b) up.tile_prefix[b] = sp.tile_prefix[b];
+}
+
 struct Ws {
   WsLayout lay;
   uint8_t *base;
@@ -190,6 +214,7 @@ struct Ws {
   double2 *ea() const { return reinterpret_cast<double2 *>(base + lay.ea); }
   float *raw() const { return reinterpret_cast<float *>(base + lay.raw); }
   int32_t *sel() const { return reinterpret_cast<int32_t *>(base + lay.sel); }
+  double *partials() const { return reinterpret_cast<double *>(base + lay.partials); }
 };
 
 const char *kStageNames[] = {"fold_kernel", "score_kernel", "unit_kernel"};
@@ -203,7 +228,8 @@ tria_status tria_workspace_size(const tria_config *cfg, const tria_cache *cache,
   tria_status s = check_config(cfg, false);
   if (s != TRIA_OK) return s;
   if (!cache || cache->cap_total < 0) return TRIA_ERR_INVALID_ARG;
-  *bytes = ws_layout(*cfg, cache->cap_total).total;
+  if (!cache->seq_start) return TRIA_ERR_INVALID_ARG;
+  *bytes = ws_layout(*cfg, cache->seq_start, cache->cap_total).total;
   return TRIA_OK;
 }
 
@@ -241,7 +267,7 @@ tria_status tria_score(const tria_config *cfg, const tria_stats *stats, const tr
   if (!score || (raw && !aligned(raw, 4))) return TRIA_ERR_INVALID_ARG;
   if ((s = check_ws(cfg, cache, ws, ws_bytes)) != TRIA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Ws w{ws_layout(*cfg, cache->cap_total), static_cast<uint8_t *>(ws)};
+  const Ws w{ws_layout(*cfg, cache->seq_start, cache->cap_total), static_cast<uint8_t *>(ws)};
   float *rawp = raw ? raw : w.raw();
 
   static thread_local FoldParams fp;
@@ -249,7 +275,8 @@ tria_status tria_score(const tria_config *cfg, const tria_stats *stats, const tr
   cudaError_t e = launch_fold(fp, cfg->head_dim / 2, st);
   if (e != cudaSuccess) return TRIA_ERR_CUDA;
   ScoreParams sp;
-  const int grid = fill_score(sp, cfg, stats, cache, w.ea(), rawp, w.err(), 0);
+  const int grid = fill_score(sp, cfg, stats, cache, w.ea(), rawp, w.partials(),
+                              w.lay.max_slots, w.err(), 0);
   if (grid > 0) {
     e = launch_score(sp, cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads, cfg->rope_layout, grid,
                      st, true);
@@ -257,6 +284,7 @@ tria_status tria_score(const tria_config *cfg, const tria_stats *stats, const tr
   }
   UnitParams up;
   fill_unit(up, cfg, cache, kModeZmax);
+  link_unit_to_score(up, sp, w.partials(), score_tile_keys(cfg->head_dim));
   up.raw = rawp;
   up.score = score;
   up.seqlen = w.seqlen();
@@ -271,7 +299,7 @@ tria_status tria_select(const tria_config *cfg, const tria_cache *cache, const f
   if ((s = check_cache(cfg, cache, false)) != TRIA_OK) return s;
   if (!score || !sel || !aligned(score, 4) || !aligned(sel, 4)) return TRIA_ERR_INVALID_ARG;
   if ((s = check_ws(cfg, cache, ws, ws_bytes)) != TRIA_OK) return s;
-  const Ws w{ws_layout(*cfg, cache->cap_total), static_cast<uint8_t *>(ws)};
+  const Ws w{ws_layout(*cfg, cache->seq_start, cache->cap_total), static_cast<uint8_t *>(ws)};
   UnitParams up;
   fill_unit(up, cfg, cache, kModeSelect);
   up.score = const_cast<float *>(score);
@@ -289,7 +317,7 @@ tria_status tria_compact(const tria_config *cfg, const tria_cache *cache, const 
   if ((s = check_cache(cfg, cache, true)) != TRIA_OK) return s;
   if (!sel || !aligned(sel, 4)) return TRIA_ERR_INVALID_ARG;
   if ((s = check_ws(cfg, cache, ws, ws_bytes)) != TRIA_OK) return s;
-  const Ws w{ws_layout(*cfg, cache->cap_total), static_cast<uint8_t *>(ws)};
+  const Ws w{ws_layout(*cfg, cache->seq_start, cache->cap_total), static_cast<uint8_t *>(ws)};
   UnitParams up;
   fill_unit(up, cfg, cache, kModeCompact);
   up.sel = const_cast<int32_t *>(sel);
@@ -311,7 +339,7 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
   if (sel_out && !aligned(sel_out, 4)) return TRIA_ERR_INVALID_ARG;
   if ((s = check_ws(cfg, cache, ws, ws_bytes)) != TRIA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Ws w{ws_layout(*cfg, cache->cap_total), static_cast<uint8_t *>(ws)};
+  const Ws w{ws_layout(*cfg, cache->seq_start, cache->cap_total), static_cast<uint8_t *>(ws)};
   int stage = 0;
   auto mark = [&]() -> bool {
     if (events && cudaEventRecord(static_cast<cudaEvent_t>(events[stage]), st) != cudaSuccess)
@@ -325,7 +353,8 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
   if (!mark()) return TRIA_ERR_CUDA;
   if (launch_fold(fp, cfg->head_dim / 2, st) != cudaSuccess) return TRIA_ERR_CUDA;
   ScoreParams sp;
-  const int grid = fill_score(sp, cfg, stats, cache, w.ea(), w.raw(), w.err(), 1);
+  const int grid = fill_score(sp, cfg, stats, cache, w.ea(), w.raw(), w.partials(),
+                              w.lay.max_slots, w.err(), 1);
   const bool pdl = events == nullptr;  // stage events between kernels would defeat the overlap
   if (!mark()) return TRIA_ERR_CUDA;
   if (grid > 0 && launch_score(sp, cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads,
@@ -333,6 +362,7 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
     return TRIA_ERR_CUDA;
   UnitParams up;
   fill_unit(up, cfg, cache, kModePrune);
+  link_unit_to_score(up, sp, w.partials(), score_tile_keys(cfg->head_dim));
   up.raw = w.raw();
   up.sel = sel_out ? sel_out : w.sel();
   up.write_short_sel = sel_out ? 1 : 0;

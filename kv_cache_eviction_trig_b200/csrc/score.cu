@@ -7,20 +7,21 @@
 //   W_hf   = c_hf * EA_bf          (trig term with offsets and cur folded in, see fold.cu)
 //   Nw_hf  = (1 - R_hf) * E|q_hf|  (norm term; |k_f| = |ktilde_f| since RoPE keeps norms)
 // ktilde is the stored post-RoPE bf16 key widened exactly to float; all sums
-// are float32.
+// are float32.  The kernel also leaves, per (unit, CTA, head), the float64
+// sums of s and s^2 over the keys it scored, which the z-score needs.
 //
 // Design (sm_100a): a persistent grid, one CTA per SM, each taking a
-// contiguous run of 32 KB key tiles.  One producer warp streams tiles into a
-// 4-stage shared-memory ring with 1-D bulk copies (cp.async.bulk, completion
-// on mbarriers, no multicast); eight consumer warps compute.  A consumer lane
-// owns PPL RoPE pairs of a key, so the G x PPL x 3 weights of its unit live in
-// registers, packed two pairs per 64-bit register for the sm_100 paired FP32
-// FMA (fma.rn.f32x2): one instruction per (two pairs, head, term).  Each lane
-// works on two keys at once for instruction-level parallelism.  The LPK lanes
-// of a key combine their partial sums by a reduce-scatter (each shuffle level
-// halves the values a lane holds); the heads are assigned to register slots in
-// a lane-dependent order at weight-load time so that no selects are needed and
-// each lane ends with one head's total, which it stores.
+// contiguous run of 64 KB key tiles.  One producer warp streams tiles into a
+// 3-stage shared-memory ring with 1-D bulk copies (cp.async.bulk, completion
+// on mbarriers, no multicast); sixteen consumer warps compute.  A consumer
+// lane owns PPL RoPE pairs of a key and works on two keys at once; the unit's
+// weights sit in shared memory in lane order (one broadcast read serves the
+// lanes of all keys in a warp) and pair up two RoPE pairs per 64-bit register
+// for the sm_100 paired FP32 FMA (fma.rn.f32x2).  The LPK lanes of a key
+// combine their partial sums by a reduce-scatter (each shuffle level halves
+// the values a lane holds); the heads are assigned to register slots in a
+// lane-dependent order when the weights are laid out, so no selects are
+// needed and each lane ends with its heads' totals, which it stores.
 #include "tria_internal.cuh"
 
 namespace tria {
@@ -28,19 +29,23 @@ namespace tria {
 template <int D, int G>
 struct ScoreShape {
   static constexpr int F = D / 2;
-  static constexpr int PPL_A = (32 / G) < 8 ? (32 / G) : 8;
-  static constexpr int PPL = (F / 32) > PPL_A ? (F / 32) : PPL_A;  // pairs per lane
+  static constexpr int PPL = 8;                                   // pairs per lane
+  static constexpr int P2 = PPL / 2;                              // paired registers per lane
   static constexpr int LPK = F / PPL;                             // lanes per key
-  static constexpr int KPW = 32 / LPK;                            // keys per warp step
+  static constexpr int KPW = 32 / LPK;                            // key groups per warp
+  static constexpr int VL = G > LPK ? G / LPK : 1;                // head totals a lane ends with
   static constexpr int ROW = 2 * D;                               // bytes per key row
   static constexpr int TILE = kScoreTileBytes / ROW;              // keys per tile
   static constexpr int NW = kScoreConsumerWarps;
   static constexpr int KEYS_PER_WARP = TILE / NW;
   static constexpr int STEPS = KEYS_PER_WARP / (2 * KPW);         // two keys per lane per step
-  static constexpr bool OK = (3 * G * PPL <= 96) && (LPK <= 32) && (LPK >= G) &&
-                             (PPL % 2 == 0) && (STEPS * 2 * KPW == KEYS_PER_WARP) &&
-                             (STEPS >= 1);
-  static constexpr size_t SMEM = (size_t)kScoreStages * TILE * ROW + 2ull * kScoreStages * 8;
+  static constexpr int WENT = P2 * G * LPK;                       // weight entries per unit
+  static constexpr bool OK = (LPK >= 1) && (LPK <= 32) && (STEPS * 2 * KPW == KEYS_PER_WARP) &&
+                             (STEPS >= 1) && (G <= 16);
+  static constexpr size_t SMEM_STAGES = (size_t)kScoreStages * TILE * ROW;
+  static constexpr size_t SMEM_W = (size_t)WENT * 24;             // float4 (wx, wy) + float2 nw
+  static constexpr size_t SMEM_PART = (size_t)NW * G * 2 * 8;     // per-warp float64 partials
+  static constexpr size_t SMEM = SMEM_STAGES + SMEM_W + SMEM_PART + 2ull * kScoreStages * 8;
 };
 
 struct TileRef {
@@ -95,6 +100,10 @@ __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
 __device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
+// A bf16 pair (one 32-bit word) widened into a float pair in one 64-bit register.
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
+  return f2_pack(dev::bf16lo(w), dev::bf16hi(w));
+}
 
 // Reduce-scatter over the lanes of a key: at offset O, a lane holding V values
 // keeps the first V/2 and adds its partner's second half; once one value is
@@ -118,55 +127,26 @@ __device__ __forceinline__ void reduce_scatter(float (&a)[G], float (&b)[G]) {
   }
 }
 
-// Loads the PPL pairs a lane owns from a key row in shared memory:
-// x[p], y[p] for pairs f0 .. f0+PPL-1.
+// The PPL pairs a lane owns in a key row held in shared memory, as two words
+// of x (and of y) per paired register: x pairs (f0+2i, f0+2i+1) in xw[i].
 template <int D, int PPL, int LAYOUT>
-__device__ __forceinline__ void load_pairs(const uint8_t *rowp, int f0, float (&x)[PPL],
-                                           float (&y)[PPL]) {
+__device__ __forceinline__ void load_row(const uint8_t *rowp, int f0, uint32_t (&xw)[PPL / 2],
+                                         uint32_t (&yw)[PPL / 2]) {
+  static_assert(PPL == 8, "lanes own eight pairs");
   if constexpr (LAYOUT == TRIA_ROPE_HALF_SPLIT) {
-    uint32_t xw[PPL / 2], yw[PPL / 2];
-    const uint8_t *px = rowp + 2 * f0;
-    const uint8_t *py = rowp + D + 2 * f0;
-    if constexpr (PPL == 8) {
-      const uint4 a = *reinterpret_cast<const uint4 *>(px);
-      const uint4 b = *reinterpret_cast<const uint4 *>(py);
-      xw[0] = a.x; xw[1] = a.y; xw[2] = a.z; xw[3] = a.w;
-      yw[0] = b.x; yw[1] = b.y; yw[2] = b.z; yw[3] = b.w;
-    } else if constexpr (PPL == 4) {
-      const uint2 a = *reinterpret_cast<const uint2 *>(px);
-      const uint2 b = *reinterpret_cast<const uint2 *>(py);
-      xw[0] = a.x; xw[1] = a.y;
-      yw[0] = b.x; yw[1] = b.y;
-    } else {
-      xw[0] = *reinterpret_cast<const uint32_t *>(px);
-      yw[0] = *reinterpret_cast<const uint32_t *>(py);
-    }
-#pragma unroll
-    for (int i = 0; i < PPL / 2; ++i) {
-      x[2 * i] = dev::bf16lo(xw[i]);
-      x[2 * i + 1] = dev::bf16hi(xw[i]);
-      y[2 * i] = dev::bf16lo(yw[i]);
-      y[2 * i + 1] = dev::bf16hi(yw[i]);
-    }
+    const uint4 a = *reinterpret_cast<const uint4 *>(rowp + 2 * f0);
+    const uint4 b = *reinterpret_cast<const uint4 *>(rowp + D + 2 * f0);
+    xw[0] = a.x; xw[1] = a.y; xw[2] = a.z; xw[3] = a.w;
+    yw[0] = b.x; yw[1] = b.y; yw[2] = b.z; yw[3] = b.w;
   } else {
-    uint32_t w[PPL];
-    const uint8_t *pp = rowp + 4 * f0;
-    if constexpr (PPL == 8) {
-      const uint4 a = *reinterpret_cast<const uint4 *>(pp);
-      const uint4 b = *reinterpret_cast<const uint4 *>(pp + 16);
-      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-      w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-    } else if constexpr (PPL == 4) {
-      const uint4 a = *reinterpret_cast<const uint4 *>(pp);
-      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-    } else {
-      const uint2 a = *reinterpret_cast<const uint2 *>(pp);
-      w[0] = a.x; w[1] = a.y;
-    }
+    // interleaved: word q holds (x_q, y_q); regroup into x and y pairs
+    const uint4 a = *reinterpret_cast<const uint4 *>(rowp + 4 * f0);
+    const uint4 b = *reinterpret_cast<const uint4 *>(rowp + 4 * f0 + 16);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int i = 0; i < PPL; ++i) {
-      x[i] = dev::bf16lo(w[i]);
-      y[i] = dev::bf16hi(w[i]);
+    for (int i = 0; i < 4; ++i) {
+      xw[i] = __byte_perm(w[2 * i], w[2 * i + 1], 0x5410);  // (x_2i, x_2i+1)
+      yw[i] = __byte_perm(w[2 * i], w[2 * i + 1], 0x7632);  // (y_2i, y_2i+1)
     }
   }
 }
@@ -175,12 +155,15 @@ template <int D, int G, int LAYOUT>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ ScoreParams p) {
   using S = ScoreShape<D, G>;
-  constexpr int F = S::F, PPL = S::PPL, LPK = S::LPK, KPW = S::KPW, ROW = S::ROW;
-  constexpr int TILE = S::TILE, NW = S::NW, NST = kScoreStages;
+  constexpr int F = S::F, PPL = S::PPL, P2 = S::P2, LPK = S::LPK, KPW = S::KPW, VL = S::VL;
+  constexpr int ROW = S::ROW, TILE = S::TILE, NW = S::NW, NST = kScoreStages;
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t *stage = smem;
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)NST * TILE * ROW);
+  float4 *wxy = reinterpret_cast<float4 *>(smem + S::SMEM_STAGES);           // [P2][G][LPK]
+  float2 *wn = reinterpret_cast<float2 *>(wxy + S::WENT);                     // [P2][G][LPK]
+  double *wpart = reinterpret_cast<double *>(wn + S::WENT);                   // [NW][G][2]
+  uint64_t *full = reinterpret_cast<uint64_t *>(wpart + NW * G * 2);
   uint64_t *empty = full + NST;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -230,48 +213,92 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   }
 
   // ------------------------------------------------------------------ consumers
-  constexpr int P2 = PPL / 2;
+  const int ct = threadIdx.x;  // consumer thread index, 0 .. NW*32-1
   const int kg = lane / LPK, li = lane % LPK, f0 = li * PPL;
   // register slot k of this lane holds head (k ^ hmask) of the group, so that the
-  // reduce-scatter leaves head hmask's total in slot 0 (see reduce_scatter)
+  // reduce-scatter leaves heads (v ^ hmask), v < VL, in slots 0 .. VL-1
   int hmask = 0;
 #pragma unroll
-  for (int lv = 0; (G >> (lv + 1)) > 0; ++lv)
+  for (int lv = 0; (G >> (lv + 1)) > 0 && (LPK >> (lv + 1)) > 0; ++lv)
     if (li & (LPK >> (lv + 1))) hmask |= (G >> (lv + 1));
-  const bool writer = (li & (LPK / G - 1)) == 0;  // lanes holding duplicate totals stay quiet
-  uint64_t wx[G][P2], wy[G][P2], nw[G][P2];
+  const bool writer = LPK <= G || (li & (LPK / G - 1)) == 0;  // duplicates stay quiet
   dev::pdl_wait();  // the folded offset factors come from the fold kernel
-  int64_t cached = -1;
+
+  double st1[VL], st2[VL];  // this lane's float64 sums of s and s^2 for its heads
+  int64_t cached = -1, cur_l = 0, cur_g = 0, cur_b = 0;
   uint32_t it = 0;
   bool failed = false;
+
+  // Publishes this CTA's partial sums for a unit: a fixed-order reduction over
+  // the lanes and warps holding each head, then one slot per (unit, CTA).
+  auto flush = [&](int64_t unit) {
+#pragma unroll
+    for (int v = 0; v < VL; ++v) {
+      double a = st1[v], b2 = st2[v];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        bool halving = false;  // lanes across a halving level hold different heads
+#pragma unroll
+        for (int lv = 0; (G >> (lv + 1)) > 0 && (LPK >> (lv + 1)) > 0; ++lv)
+          if (o == (LPK >> (lv + 1))) halving = true;
+        if (!halving) {
+          a += __shfl_xor_sync(0xffffffffu, a, o);
+          b2 += __shfl_xor_sync(0xffffffffu, b2, o);
+        }
+      }
+      if (kg == 0 && writer) {
+        const int h = v ^ hmask;
+        wpart[(warp * G + h) * 2 + 0] = a;
+        wpart[(warp * G + h) * 2 + 1] = b2;
+      }
+    }
+    dev::named_barrier(1, NW * 32);
+    if (ct < 2 * G) {
+      double a = 0.0;
+      for (int w = 0; w < NW; ++w) a += wpart[w * G * 2 + ct];
+      const int64_t first_tile = (unit / p.B) * p.tiles_per_row + p.tile_prefix[unit % p.B];
+      const int64_t slot = blockIdx.x - first_tile / p.tiles_per_cta;
+      p.partials[(unit * p.max_slots + slot) * (2 * G) + ct] = a;
+    }
+    dev::named_barrier(1, NW * 32);
+  };
+
   for (int64_t t = t0; t < t1; ++t) {
     const TileRef tl = tile_of(p, t, TILE);
     if (tl.n <= 0) continue;
-    const int32_t l = tl.row / p.Hkv, g = tl.row - l * p.Hkv;
     const int64_t unit = (int64_t)tl.row * p.B + tl.b;
     if (unit != cached) {
+      if (cached >= 0) flush(cached);
       cached = unit;
+      cur_l = tl.row / p.Hkv;
+      cur_g = tl.row - cur_l * p.Hkv;
+      cur_b = tl.b;
 #pragma unroll
-      for (int k = 0; k < G; ++k) {
-        const size_t base = ((size_t)l * p.Hq + (size_t)g * G + (k ^ hmask)) * F + f0;
+      for (int v = 0; v < VL; ++v) { st1[v] = 0.0; st2[v] = 0.0; }
+      // lay out the unit's weights in lane order (the previous unit's readers are
+      // past the barrier in flush, or this is the first unit)
+      for (int e = ct; e < S::WENT; e += NW * 32) {
+        const int el = e % LPK, ek = (e / LPK) % G, ei = e / (LPK * G);
+        int em = 0;
 #pragma unroll
-        for (int i = 0; i < P2; ++i) {
-          float ax[2], ay[2], an[2];
+        for (int lv = 0; (G >> (lv + 1)) > 0 && (LPK >> (lv + 1)) > 0; ++lv)
+          if (el & (LPK >> (lv + 1))) em |= (G >> (lv + 1));
+        const int h = ek ^ em;
+        const size_t base = ((size_t)cur_l * p.Hq + (size_t)cur_g * G + h) * F + el * PPL + 2 * ei;
+        float wxv[2], wyv[2], nv[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int q = 2 * i + e;
-            const float2 c = p.centre[base + q];
-            const double2 ea = p.ea[(size_t)tl.b * F + f0 + q];
-            ax[e] = (float)((double)c.x * ea.x - (double)c.y * ea.y);
-            ay[e] = (float)((double)c.x * ea.y + (double)c.y * ea.x);
-            const float r = p.no_conc_weight ? 0.0f : p.mrl[base + q];
-            an[e] = (1.0f - r) * p.mean_norm[base + q];
-          }
-          wx[k][i] = f2_pack(ax[0], ax[1]);
-          wy[k][i] = f2_pack(ay[0], ay[1]);
-          nw[k][i] = f2_pack(an[0], an[1]);
+        for (int q = 0; q < 2; ++q) {
+          const float2 c = p.centre[base + q];
+          const double2 ea = p.ea[(size_t)cur_b * F + el * PPL + 2 * ei + q];
+          wxv[q] = (float)((double)c.x * ea.x - (double)c.y * ea.y);
+          wyv[q] = (float)((double)c.x * ea.y + (double)c.y * ea.x);
+          const float r = p.no_conc_weight ? 0.0f : p.mrl[base + q];
+          nv[q] = (1.0f - r) * p.mean_norm[base + q];
         }
+        wxy[e] = make_float4(wxv[0], wxv[1], wyv[0], wyv[1]);
+        wn[e] = make_float2(nv[0], nv[1]);
       }
+      dev::named_barrier(1, NW * 32);
     }
     const uint32_t s = it % NST, use = it / NST;
     if (!failed && !dev::mbar_wait(&full[s], use & 1)) {
@@ -280,23 +307,21 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     }
     if (!failed) {
       const uint8_t *sb = stage + (size_t)s * TILE * ROW;
-      float *rawh = p.raw + ((size_t)l * p.Hq + (size_t)g * G + hmask) * p.cap +
-                    (size_t)p.seg_start[tl.b] + tl.key0;
+      float *rawrow = p.raw + ((size_t)cur_l * p.Hq + (size_t)cur_g * G) * p.cap +
+                      (size_t)p.seg_start[cur_b] + tl.key0;
 #pragma unroll 1
       for (int step = 0; step < S::STEPS; ++step) {
         const int ka = warp * S::KEYS_PER_WARP + step * 2 * KPW + kg, kb = ka + KPW;
-        float xa[PPL], ya[PPL], xb[PPL], yb[PPL];
-        load_pairs<D, PPL, LAYOUT>(sb + (size_t)ka * ROW, f0, xa, ya);
-        load_pairs<D, PPL, LAYOUT>(sb + (size_t)kb * ROW, f0, xb, yb);
+        uint32_t xa[P2], ya[P2], xb[P2], yb[P2];
+        load_row<D, PPL, LAYOUT>(sb + (size_t)ka * ROW, f0, xa, ya);
+        load_row<D, PPL, LAYOUT>(sb + (size_t)kb * ROW, f0, xb, yb);
         uint64_t acca[G], accb[G];
 #pragma unroll
         for (int k = 0; k < G; ++k) acca[k] = accb[k] = 0ull;
 #pragma unroll
         for (int i = 0; i < P2; ++i) {
-          const uint64_t XA = f2_pack(xa[2 * i], xa[2 * i + 1]);
-          const uint64_t YA = f2_pack(ya[2 * i], ya[2 * i + 1]);
-          const uint64_t XB = f2_pack(xb[2 * i], xb[2 * i + 1]);
-          const uint64_t YB = f2_pack(yb[2 * i], yb[2 * i + 1]);
+          const uint64_t XA = bf16x2_to_f2(xa[i]), YA = bf16x2_to_f2(ya[i]);
+          const uint64_t XB = bf16x2_to_f2(xb[i]), YB = bf16x2_to_f2(yb[i]);
           float n0, n1, m0, m1;
           f2_unpack(f2_fma(YA, YA, f2_mul(XA, XA)), n0, n1);
           f2_unpack(f2_fma(YB, YB, f2_mul(XB, XB)), m0, m1);
@@ -304,12 +329,17 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           const uint64_t NB = f2_pack(sqrt_approx(m0), sqrt_approx(m1));
 #pragma unroll
           for (int k = 0; k < G; ++k) {
-            acca[k] = f2_fma(wx[k][i], XA, acca[k]);
-            accb[k] = f2_fma(wx[k][i], XB, accb[k]);
-            acca[k] = f2_fma(wy[k][i], YA, acca[k]);
-            accb[k] = f2_fma(wy[k][i], YB, accb[k]);
-            acca[k] = f2_fma(nw[k][i], NA, acca[k]);
-            accb[k] = f2_fma(nw[k][i], NB, accb[k]);
+            const int e = (i * G + k) * LPK + li;
+            const float4 w4 = wxy[e];
+            const float2 w2 = wn[e];
+            const uint64_t WX = f2_pack(w4.x, w4.y), WY = f2_pack(w4.z, w4.w);
+            const uint64_t WN = f2_pack(w2.x, w2.y);
+            acca[k] = f2_fma(WX, XA, acca[k]);
+            accb[k] = f2_fma(WX, XB, accb[k]);
+            acca[k] = f2_fma(WY, YA, acca[k]);
+            accb[k] = f2_fma(WY, YB, accb[k]);
+            acca[k] = f2_fma(WN, NA, acca[k]);
+            accb[k] = f2_fma(WN, NB, accb[k]);
           }
         }
         float sa[G], sbv[G];
@@ -323,8 +353,20 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
         reduce_scatter<LPK / 2, G, G>(sa, sbv);
         if (writer) {
-          if (ka < tl.n) rawh[ka] = sa[0];
-          if (kb < tl.n) rawh[kb] = sbv[0];
+#pragma unroll
+          for (int v = 0; v < VL; ++v) {
+            float *rh = rawrow + (size_t)(v ^ hmask) * p.cap;
+            if (ka < tl.n) {
+              rh[ka] = sa[v];
+              st1[v] += (double)sa[v];
+              st2[v] = fma((double)sa[v], (double)sa[v], st2[v]);
+            }
+            if (kb < tl.n) {
+              rh[kb] = sbv[v];
+              st1[v] += (double)sbv[v];
+              st2[v] = fma((double)sbv[v], (double)sbv[v], st2[v]);
+            }
+          }
         }
       }
     }
@@ -332,6 +374,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     if (lane == 0) dev::mbar_arrive(&empty[s]);
     ++it;
   }
+  if (cached >= 0) flush(cached);
 }
 
 template <int D, int G, int LAYOUT>

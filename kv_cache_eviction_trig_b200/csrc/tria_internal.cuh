@@ -17,19 +17,21 @@ struct WsLayout {
   size_t raw;       // float [L][Hq][cap]  raw scores when the caller gives none
   size_t score;     // float [L][Hkv][cap] group-max z-scores (tria_prune does not need it)
   size_t sel;       // int32 [L][Hkv][B][budget] selection scratch
+  size_t partials;  // double [L*Hkv*B][max_slots][G][2] per-CTA sums of s and s^2
+  int32_t max_slots;
   size_t total;
 };
-WsLayout ws_layout(const tria_config &cfg, int64_t cap_total);
+WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap_total);
 
 // ------------------------------------------------------------------ kernel parameters
-constexpr int kScoreConsumerWarps = 8;
+constexpr int kScoreConsumerWarps = 16;
 constexpr int kScoreThreads = (kScoreConsumerWarps + 1) * 32;
-constexpr int kScoreStages = 4;
-constexpr int kScoreTileBytes = 32 * 1024;   // bytes of K per pipeline stage
+constexpr int kScoreStages = 3;
+constexpr int kScoreTileBytes = 64 * 1024;   // bytes of K per pipeline stage
 
-constexpr int kUnitThreads = 256;
+constexpr int kUnitThreads = 1024;
 constexpr int kUnitCluster = 8;
-constexpr int kUnitSmemSmall = 112 * 1024;  // two CTAs per SM
+constexpr int kUnitSmemSmall = 112 * 1024;  // smaller footprint (more clusters resident)
 constexpr int kUnitSmemLarge = 200 * 1024;  // one CTA per SM
 
 struct FoldParams {
@@ -53,8 +55,10 @@ struct ScoreParams {
   const double2 *ea;        // [B][F]  (written by the fold kernel)
   const int32_t *seq_len;   // [B] caller's live lengths (not modified during the call)
   float *raw;               // [L][Hq][cap]
+  double *partials;         // [units][max_slots][G][2]
   int32_t *err;
   int64_t cap;
+  int32_t max_slots;
   int32_t L, Hkv, Hq, B, budget;
   int32_t skip_short;       // 1: sequences with seq_len <= budget are not scored
   int32_t no_conc_weight;   // ablation flag
@@ -72,6 +76,9 @@ struct UnitParams {
   uint8_t *v;
   int32_t *pos;
   const float *raw;         // [L][Hq][cap]      (zmax, prune)
+  const double *partials;   // [units][max_slots][G][2] from the score kernel (zmax, prune)
+  int32_t max_slots, tiles_per_cta, tiles_per_row, tile_keys;
+  int32_t tile_prefix[TRIA_MAX_BATCH + 1];
   float *score;             // [L][Hkv][cap]     (zmax writes, select reads)
   int32_t *sel;             // [L][Hkv][B][budget]
   const int32_t *seqlen;    // [B] snapshot (zmax, select, prune)

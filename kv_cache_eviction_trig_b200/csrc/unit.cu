@@ -4,10 +4,9 @@
 //   z-score + group max (romaanj.github.io review, "Method"; dimensionstp.github.io
 //     review, section 3-2 (6)): mu_h and the population sigma_h of the raw
 //     scores over the sequence's T live keys; z_h = (s_h - mu_h) / sigma_h
-//     (0 when sigma_h = 0); score = max_h z_h.  The sums are float64, taken
-//     about a pivot (the unit's first raw score) so that a large mean does not
-//     cancel the variance, and reduced across the cluster in rank order, so the
-//     result is deterministic.
+//     (0 when sigma_h = 0); score = max_h z_h.  mu and sigma come from the
+//     float64 sums of s and s^2 the score kernel leaves per (CTA, head), added
+//     here in a fixed order, so the result is deterministic.
 //   selection (same sources, "prune back to budget"; section 3-2 (5)): the
 //     `budget` largest scores, ties to the lower slot, by a 4-pass 8-bit radix
 //     select on order-preserving 32-bit keys.  Each CTA histograms its slice in
@@ -37,7 +36,7 @@ namespace tria {
 
 namespace {
 
-constexpr int kCtl = 12 * 1024;  // control region at the start of shared memory
+constexpr int kCtl = 20 * 1024;  // control region at the start of shared memory
 constexpr int kMaxG = 16;
 constexpr int kMaxCluster = 16;
 constexpr int kWarps = kUnitThreads / 32;
@@ -46,12 +45,9 @@ struct Ctl {
   uint64_t cbar;                    // compaction bulk-load barrier
   uint32_t hist[2][256];
   uint32_t tot[256];
-  double part[kMaxG][2];            // this CTA's shifted sums: sum(s - p), sum((s - p)^2)
-  double gath[kMaxCluster][kMaxG][2];
-  double wred[kWarps][kMaxG][2];
-  double mu[kMaxG];
-  double inv_sigma[kMaxG];
-  float pivot[kMaxG];
+  double gath[1][kMaxG][2];         // the unit's sums of s and s^2 per head
+  float mu_hi[kMaxG], mu_lo[kMaxG];  // mean split into two floats (hi + lo)
+  float inv_sigma[kMaxG];
   int32_t cnt[4];                   // gt, eq of this CTA / first_neg, bad (compaction check)
   int32_t peer_cnt[kMaxCluster][2];
   int32_t bc[8];                    // broadcast scalars
@@ -87,32 +83,6 @@ __device__ __forceinline__ int block_excl_scan(int v, int32_t *wtot, int *total)
   return out;
 }
 
-// 4-byte asynchronous global -> shared copies (any 4-byte alignment) ...
-__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dev::smem_addr(dst)), "l"(src)
-               : "memory");
-}
-// ... and 16-byte ones for 16-byte aligned runs.
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dev::smem_addr(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
-}
-
-// Copies n floats global -> shared with asynchronous copies (waited by the caller).
-__device__ __forceinline__ void stage_floats(float *dst, const float *src, int n) {
-  const bool vec = ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) == 0;
-  if (vec) {
-    const int n4 = n >> 2;
-    for (int i = threadIdx.x; i < n4; i += blockDim.x) cp_async16(dst + 4 * i, src + 4 * i);
-    for (int i = 4 * n4 + threadIdx.x; i < n; i += blockDim.x) cp_async4(dst + i, src + i);
-  } else {
-    for (int i = threadIdx.x; i < n; i += blockDim.x) cp_async4(dst + i, src + i);
-  }
-}
-
 // 1-D bulk copy shared -> global (bulk-group completion).
 __device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
@@ -127,7 +97,7 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 
 }  // namespace
 
-__global__ void __launch_bounds__(kUnitThreads, 2) unit_kernel(const __grid_constant__ UnitParams p) {
+__global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_constant__ UnitParams p) {
   cg::cluster_group cl = cg::this_cluster();
   const int CL = (int)cl.num_blocks();
   const int r = (int)cl.block_rank();
@@ -140,7 +110,7 @@ __global__ void __launch_bounds__(kUnitThreads, 2) unit_kernel(const __grid_cons
   const int64_t seg_cap = p.seg_start[b + 1] - seg;
   const int G = p.G;
   const int tid = threadIdx.x, nthr = blockDim.x;
-  const int warp = tid >> 5, lane = tid & 31;
+  const int lane = tid & 31;
 
   extern __shared__ __align__(128) uint8_t smem[];
   Ctl &c = *reinterpret_cast<Ctl *>(smem);
@@ -217,70 +187,41 @@ __global__ void __launch_bounds__(kUnitThreads, 2) unit_kernel(const __grid_cons
 
     if (p.mode == kModeZmax || p.mode == kModePrune) {
       // ---------------------------------------------------- z-score statistics
-      const bool cache = (size_t)(G + 1) * nmax4 * 4 <= data_bytes;
-      float *rawc = reinterpret_cast<float *>(data) + nmax4;  // [G][nmax4]
+      // The score kernel left float64 sums of s and s^2 per (CTA, head) for this
+      // unit; the CTAs that scored it are those whose tile runs meet its live tiles.
       const float *rawu = p.raw + ((int64_t)l * p.Hq + (int64_t)g * G) * p.cap + seg;
-      if (cache) {
-        for (int j = 0; j < G; ++j) stage_floats(rawc + (size_t)j * nmax4, rawu + (int64_t)j * p.cap + lo, n);
-        cp_async_wait_all();
-      }
-      if (tid < G) c.pivot[tid] = rawu[(int64_t)tid * p.cap];
-      __syncthreads();
-      for (int j = 0; j < G; ++j) {
-        const double pv = (double)c.pivot[j];
-        double a1 = 0.0, a2 = 0.0;
-        for (int i = tid; i < n; i += nthr) {
-          const float v = cache ? rawc[(size_t)j * nmax4 + i] : rawu[(int64_t)j * p.cap + lo + i];
-          const double d = (double)v - pv;
-          a1 += d;
-          a2 = fma(d, d, a2);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          a1 += __shfl_xor_sync(0xffffffffu, a1, o);
-          a2 += __shfl_xor_sync(0xffffffffu, a2, o);
-        }
-        if (lane == 0) { c.wred[warp][j][0] = a1; c.wred[warp][j][1] = a2; }
-      }
-      __syncthreads();
       if (tid < 2 * G) {
-        const int j = tid >> 1, k = tid & 1;
+        const int64_t first_tile = row * p.tiles_per_row + p.tile_prefix[b];
+        const int64_t live_tiles = ((int64_t)T + p.tile_keys - 1) / p.tile_keys;
+        const int64_t c0 = first_tile / p.tiles_per_cta;
+        const int64_t c1 = (first_tile + live_tiles - 1) / p.tiles_per_cta;
+        const double *pu = p.partials + unit * (int64_t)p.max_slots * (2 * G);
         double a = 0.0;
-        for (int w = 0; w < kWarps; ++w) a += c.wred[w][j][k];
-        c.part[j][k] = a;
-      }
-      cl.sync();
-      for (int t = tid; t < CL * 2 * G; t += nthr) {
-        const int q = t / (2 * G), j = (t >> 1) % G, k = t & 1;
-        c.gath[q][j][k] = cl.map_shared_rank(&c, q)->part[j][k];
+        for (int64_t q = 0; q <= c1 - c0; ++q) a += pu[q * (2 * G) + tid];  // fixed order
+        c.gath[0][tid >> 1][tid & 1] = a;
       }
       __syncthreads();
       if (tid < G) {
-        double s1 = 0.0, s2 = 0.0;
-        for (int q = 0; q < CL; ++q) { s1 += c.gath[q][tid][0]; s2 += c.gath[q][tid][1]; }
-        const double m1 = s1 / (double)T;
-        const double var = s2 / (double)T - m1 * m1;
-        c.mu[tid] = (double)c.pivot[tid] + m1;
-        c.inv_sigma[tid] = var > 0.0 ? 1.0 / sqrt(var) : 0.0;
+        const double m = c.gath[0][tid][0] / (double)T;
+        const double var = c.gath[0][tid][1] / (double)T - m * m;
+        c.mu_hi[tid] = (float)m;
+        c.mu_lo[tid] = (float)(m - (double)c.mu_hi[tid]);
+        c.inv_sigma[tid] = var > 0.0 ? (float)(1.0 / sqrt(var)) : 0.0f;
       }
       __syncthreads();
       // ---------------------------------------------------- z and group max
       float *score = p.score + row * p.cap + seg;
       for (int i = tid; i < n; i += nthr) {
-        double zmax = -1.0e300;
+        float zf = -3.0e38f;
         for (int j = 0; j < G; ++j) {
-          const float v = cache ? rawc[(size_t)j * nmax4 + i] : rawu[(int64_t)j * p.cap + lo + i];
-          const double z = ((double)v - c.mu[j]) * c.inv_sigma[j];
-          zmax = z > zmax ? z : zmax;
+          const float v = rawu[(int64_t)j * p.cap + lo + i];
+          const float z = ((v - c.mu_hi[j]) - c.mu_lo[j]) * c.inv_sigma[j];
+          zf = fmaxf(zf, z);
         }
-        const float zf = (float)zmax;
         if (p.mode == kModeZmax) score[lo + i] = zf == 0.0f ? 0.0f : zf;
         else zkey[i] = dev::order_key(zf);
       }
-      if (p.mode == kModeZmax) {
-        cl.sync();  // peers may still read this CTA's partial sums
-        return;
-      }
+      if (p.mode == kModeZmax) return;
     } else {
       const float *score = p.score + row * p.cap + seg;
       for (int i = tid; i < n; i += nthr) zkey[i] = dev::order_key(score[lo + i]);
@@ -304,7 +245,11 @@ __global__ void __launch_bounds__(kUnitThreads, 2) unit_kernel(const __grid_cons
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           // padding keys are 0: they match only while prefix == 0 and mask == 0
-          if ((ks[e] & mask) == prefix && 4 * i + e < n) atomicAdd(&H[(ks[e] >> shift) & 255u], 1u);
+          if ((ks[e] & mask) == prefix && 4 * i + e < n) {
+            const uint32_t d = (ks[e] >> shift) & 255u;
+            const uint32_t peers = __match_any_sync(__activemask(), d);
+            if ((uint32_t)lane == (uint32_t)(__ffs(peers) - 1)) atomicAdd(&H[d], (uint32_t)__popc(peers));
+          }
         }
       }
       cl.sync();
@@ -402,8 +347,8 @@ __global__ void __launch_bounds__(kUnitThreads, 2) unit_kernel(const __grid_cons
 
   // -------------------------------------------------------------- in-place compaction
   const int ROW = 2 * p.D;                          // bytes per K or V row
-  constexpr int kPosPerThread = 4;                   // rows a thread handles per batch
-  const int cap_rows = min((int)(data_bytes / (2 * (size_t)ROW)), kPosPerThread * nthr);
+  constexpr int kItemsPerThread = 2;                 // row copies a thread issues per batch
+  const int cap_rows = min((int)(data_bytes / (2 * (size_t)ROW)), kItemsPerThread * nthr / 2);
   // Batch bt covers the destinations [bt * CL * cap_rows, (bt + 1) * CL * cap_rows) of the
   // whole cluster (CTA r takes the r-th chunk), so every destination written in a batch
   // precedes every destination, and hence every source, of the batches after it.
@@ -421,17 +366,18 @@ __global__ void __launch_bounds__(kUnitThreads, 2) unit_kernel(const __grid_cons
     int64_t e = a + cap_rows;
     if (e > kept) e = kept;
     const int nb = e > a ? (int)(e - a) : 0;
-    int32_t src[kPosPerThread], rp[kPosPerThread];
+    // item it = 2 * row + {0: K row (and pos), 1: V row}
+    int32_t src[kItemsPerThread], rp[kItemsPerThread];
     uint32_t bytes = 0;
 #pragma unroll
-    for (int u = 0; u < kPosPerThread; ++u) {
-      const int jj = tid + u * nthr;
+    for (int u = 0; u < kItemsPerThread; ++u) {
+      const int item = tid + u * nthr, jj = item >> 1;
       src[u] = -1;
       if (jj < nb) {
         const int32_t s = __ldcg(sel + a + jj);
         if (s >= 0 && s < seg_cap) {
-          if (s != a + jj) { src[u] = s; bytes += 2u * ROW; }
-        } else {
+          if (s != a + jj) { src[u] = s; bytes += (uint32_t)ROW; }
+        } else if ((item & 1) == 0) {
           dev::set_error(p.err, TRIA_DEVERR_SELECTION);
         }
       }
@@ -439,12 +385,15 @@ __global__ void __launch_bounds__(kUnitThreads, 2) unit_kernel(const __grid_cons
     if (!failed) {
       dev::mbar_arrive_expect_tx(&c.cbar, bytes);
 #pragma unroll
-      for (int u = 0; u < kPosPerThread; ++u) {
+      for (int u = 0; u < kItemsPerThread; ++u) {
         if (src[u] >= 0) {
-          const int jj = tid + u * nthr;
-          dev::bulk_g2s(sk + (size_t)jj * ROW, kg + (size_t)src[u] * ROW, ROW, &c.cbar);
-          dev::bulk_g2s(sv + (size_t)jj * ROW, vg + (size_t)src[u] * ROW, ROW, &c.cbar);
-          rp[u] = pg[src[u]];
+          const int item = tid + u * nthr, jj = item >> 1;
+          if ((item & 1) == 0) {
+            dev::bulk_g2s(sk + (size_t)jj * ROW, kg + (size_t)src[u] * ROW, ROW, &c.cbar);
+            rp[u] = pg[src[u]];
+          } else {
+            dev::bulk_g2s(sv + (size_t)jj * ROW, vg + (size_t)src[u] * ROW, ROW, &c.cbar);
+          }
         }
       }
       if (!dev::mbar_wait(&c.cbar, bt & 1)) {
@@ -455,12 +404,15 @@ __global__ void __launch_bounds__(kUnitThreads, 2) unit_kernel(const __grid_cons
     cl.sync();  // every source row of this batch has been read, cluster-wide
     if (!failed) {
 #pragma unroll
-      for (int u = 0; u < kPosPerThread; ++u) {
+      for (int u = 0; u < kItemsPerThread; ++u) {
         if (src[u] >= 0) {
-          const int jj = tid + u * nthr;
-          bulk_s2g(kg + (size_t)(a + jj) * ROW, sk + (size_t)jj * ROW, ROW);
-          bulk_s2g(vg + (size_t)(a + jj) * ROW, sv + (size_t)jj * ROW, ROW);
-          pg[a + jj] = rp[u];
+          const int item = tid + u * nthr, jj = item >> 1;
+          if ((item & 1) == 0) {
+            bulk_s2g(kg + (size_t)(a + jj) * ROW, sk + (size_t)jj * ROW, ROW);
+            pg[a + jj] = rp[u];
+          } else {
+            bulk_s2g(vg + (size_t)(a + jj) * ROW, sv + (size_t)jj * ROW, ROW);
+          }
         }
       }
       bulk_commit();
@@ -472,52 +424,20 @@ __global__ void __launch_bounds__(kUnitThreads, 2) unit_kernel(const __grid_cons
   if (r == 0 && tid == 0 && l == 0 && g == 0) p.seq_len_out[b] = kept;
 }
 
-// Launch configuration: 8-CTA clusters (portable; 15 fit at once with the large
-// shared-memory size, 33 with the small one); the large size is used when one
-// wave holds every unit or a segment needs it.
-namespace {
-struct UnitCfg {
-  int max_small = 0, max_large = 0;
-  bool ready = false;
-};
-UnitCfg g_unit_cfg[64];
-
-int max_clusters(int smem) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kUnitCluster, 1, 1);
-  cfg.blockDim = dim3(kUnitThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = kUnitCluster;
-  attr.val.clusterDim.y = 1;
-  attr.val.clusterDim.z = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, unit_kernel, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    return 1;
-  }
-  return n > 0 ? n : 1;
-}
-}  // namespace
-
+// Launch configuration: 8-CTA clusters of 1024 threads, one CTA per SM
+// (portable cluster size; 15 clusters are resident at once on a B200).
 int unit_cluster_size() { return kUnitCluster; }
 
 int unit_smem_bytes(int units, int64_t max_segment) {
+  (void)units;
+  (void)max_segment;  // the large size holds the keys of a TRIA_MAX_SEGMENT segment per CTA
+  static bool configured[64] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  UnitCfg &uc = g_unit_cfg[dev];
-  if (!uc.ready) {
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && !configured[dev]) {
     cudaFuncSetAttribute(unit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUnitSmemLarge);
-    uc.max_small = max_clusters(kUnitSmemSmall);
-    uc.max_large = max_clusters(kUnitSmemLarge);
-    uc.ready = true;
+    configured[dev] = true;
   }
-  const int64_t keys_per_cta = (max_segment + kUnitCluster - 1) / kUnitCluster;
-  const bool need_large = (keys_per_cta + 4) * 4 + 12 * 1024 > kUnitSmemSmall;
-  return (need_large || units <= uc.max_large) ? kUnitSmemLarge : kUnitSmemSmall;
+  return kUnitSmemLarge;
 }
 
 cudaError_t launch_unit(const UnitParams &p, int units, cudaStream_t s, bool pdl) {

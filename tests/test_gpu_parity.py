@@ -261,10 +261,11 @@ def test_compact_in_place_is_bit_exact(kind):
 
 
 @pytest.mark.parametrize("kind", ["last", "alternating", "random"])
-def test_compact_many_units_multi_batch(kind):
-    """More units than fit in one wave of clusters: the kernel stages fewer rows
-    per batch, so a 2000-row budget needs two cluster-wide batches."""
-    wl = small("compact-multi", L=2, Hq=32, Hkv=8, B=1, seq_lens=[2500], budget=2000)
+@pytest.mark.parametrize("D,budget,T", [(128, 3500, 4000), (256, 2000, 2500)])
+def test_compact_many_units_multi_batch(kind, D, budget, T):
+    """Budgets larger than one cluster can stage at once (about 2900 rows of
+    D=128, 1400 of D=256) are compacted in several cluster-wide batches."""
+    wl = small("compact-multi", L=2, Hq=32, Hkv=8, B=1, D=D, seq_lens=[T], budget=budget)
     case = Case(wl)
     rng = np.random.default_rng(11)
     sel = np.stack([np.stack([np.stack([_adversarial_sel(kind, T, wl.budget, rng)
@@ -273,12 +274,12 @@ def test_compact_many_units_multi_batch(kind):
     tria.tria_compact(case.cfg, case.cache, torch.from_numpy(sel).cuda(), case.ws)
     torch.cuda.synchronize()
     assert tria.tria_get_device_error(case.ws) == 0
-    assert case.dev["seq_len"].cpu().tolist() == [2000]
-    check_compacted(case, sel, [2000])
+    assert case.dev["seq_len"].cpu().tolist() == [budget]
+    check_compacted(case, sel, [budget])
 
 
 def test_prune_many_units_matches_oracle():
-    case = Case(small("prune-multi", L=2, Hq=32, Hkv=8, B=1, seq_lens=[2500], budget=2000,
+    case = Case(small("prune-multi", L=2, Hq=32, Hkv=8, B=1, seq_lens=[4000], budget=3500,
                       offsets=range(1, 17)))
     wl = case.wl
     ref = oracle.prune(case.prob, common.bf16_bits(case.host["v"]))
@@ -289,7 +290,7 @@ def test_prune_many_units_matches_oracle():
     assert tria.tria_get_device_error(case.ws) == 0
     gsel = sel.cpu().numpy()
     check_selection(gsel, ref["sel"], ref["raw"], ref["score"], case)
-    check_compacted(case, gsel, [2000])
+    check_compacted(case, gsel, [3500])
 
 
 def test_compact_rejects_malformed_selection():

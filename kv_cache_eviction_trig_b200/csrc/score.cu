@@ -17,7 +17,7 @@
 // lane owns PPL RoPE pairs of a key and works on two keys at once; the unit's
 // weights sit in shared memory in lane order (one broadcast read serves the
 // lanes of all keys in a warp) and pair up two RoPE pairs per 64-bit register
-// for the sm_100 paired FP32 FMA (fma.rn.f32x2).  The LPK lanes of a key
+// for the sm_100 paired FP32 FMA (__ffma2_rn).  The LPK lanes of a key
 // combine their partial sums by a reduce-scatter (each shuffle level halves
 // the values a lane holds); the heads are assigned to register slots in a
 // lane-dependent order when the weights are laid out, so no selects are
@@ -81,28 +81,9 @@ __device__ __forceinline__ float sqrt_approx(float x) {
   return y;
 }
 
-// Paired float32 arithmetic of sm_100 (two lanes of work per instruction).
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t d;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
-  return d;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-// A bf16 pair (one 32-bit word) widened into a float pair in one 64-bit register.
-__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
-  return f2_pack(dev::bf16lo(w), dev::bf16hi(w));
+// A bf16 pair (one 32-bit word) widened exactly into a float pair.
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
+  return make_float2(dev::bf16lo(w), dev::bf16hi(w));
 }
 
 // Reduce-scatter over the lanes of a key: at offset O, a lane holding V values
@@ -315,41 +296,37 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         uint32_t xa[P2], ya[P2], xb[P2], yb[P2];
         load_row<D, PPL, LAYOUT>(sb + (size_t)ka * ROW, f0, xa, ya);
         load_row<D, PPL, LAYOUT>(sb + (size_t)kb * ROW, f0, xb, yb);
-        uint64_t acca[G], accb[G];
+        // paired float32 arithmetic of sm_100: __ffma2_rn does two FMAs per instruction
+        float2 acca[G], accb[G];
 #pragma unroll
-        for (int k = 0; k < G; ++k) acca[k] = accb[k] = 0ull;
+        for (int k = 0; k < G; ++k) acca[k] = accb[k] = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int i = 0; i < P2; ++i) {
-          const uint64_t XA = bf16x2_to_f2(xa[i]), YA = bf16x2_to_f2(ya[i]);
-          const uint64_t XB = bf16x2_to_f2(xb[i]), YB = bf16x2_to_f2(yb[i]);
-          float n0, n1, m0, m1;
-          f2_unpack(f2_fma(YA, YA, f2_mul(XA, XA)), n0, n1);
-          f2_unpack(f2_fma(YB, YB, f2_mul(XB, XB)), m0, m1);
-          const uint64_t NA = f2_pack(sqrt_approx(n0), sqrt_approx(n1));
-          const uint64_t NB = f2_pack(sqrt_approx(m0), sqrt_approx(m1));
+          const float2 XA = bf16x2_to_f2(xa[i]), YA = bf16x2_to_f2(ya[i]);
+          const float2 XB = bf16x2_to_f2(xb[i]), YB = bf16x2_to_f2(yb[i]);
+          const float2 na2 = __ffma2_rn(YA, YA, __fmul2_rn(XA, XA));
+          const float2 nb2 = __ffma2_rn(YB, YB, __fmul2_rn(XB, XB));
+          const float2 NA = make_float2(sqrt_approx(na2.x), sqrt_approx(na2.y));
+          const float2 NB = make_float2(sqrt_approx(nb2.x), sqrt_approx(nb2.y));
 #pragma unroll
           for (int k = 0; k < G; ++k) {
             const int e = (i * G + k) * LPK + li;
             const float4 w4 = wxy[e];
-            const float2 w2 = wn[e];
-            const uint64_t WX = f2_pack(w4.x, w4.y), WY = f2_pack(w4.z, w4.w);
-            const uint64_t WN = f2_pack(w2.x, w2.y);
-            acca[k] = f2_fma(WX, XA, acca[k]);
-            accb[k] = f2_fma(WX, XB, accb[k]);
-            acca[k] = f2_fma(WY, YA, acca[k]);
-            accb[k] = f2_fma(WY, YB, accb[k]);
-            acca[k] = f2_fma(WN, NA, acca[k]);
-            accb[k] = f2_fma(WN, NB, accb[k]);
+            const float2 WX = make_float2(w4.x, w4.y), WY = make_float2(w4.z, w4.w);
+            const float2 WN = wn[e];
+            acca[k] = __ffma2_rn(WX, XA, acca[k]);
+            accb[k] = __ffma2_rn(WX, XB, accb[k]);
+            acca[k] = __ffma2_rn(WY, YA, acca[k]);
+            accb[k] = __ffma2_rn(WY, YB, accb[k]);
+            acca[k] = __ffma2_rn(WN, NA, acca[k]);
+            accb[k] = __ffma2_rn(WN, NB, accb[k]);
           }
         }
         float sa[G], sbv[G];
 #pragma unroll
         for (int k = 0; k < G; ++k) {
-          float lo, hi;
-          f2_unpack(acca[k], lo, hi);
-          sa[k] = lo + hi;
-          f2_unpack(accb[k], lo, hi);
-          sbv[k] = lo + hi;
+          sa[k] = acca[k].x + acca[k].y;
+          sbv[k] = accb[k].x + accb[k].y;
         }
         reduce_scatter<LPK / 2, G, G>(sa, sbv);
         if (writer) {

@@ -183,6 +183,32 @@ const char *tria_prune_stage_name(int32_t i);
  * `stream`).  Returns TRIA_ERR_DEVICE_FLAG if any bit is set, TRIA_OK otherwise. */
 tria_status tria_get_device_error(const void *ws, int32_t *code, void *stream);
 
+/* tria_prune for callers that cannot allocate device memory.  This entry point
+ * has no counterpart in the paper: it exists for callers such as a serving
+ * engine that reserves all device memory at start-up and forbids allocation in
+ * its decode loop (cudaMalloc may fail once its pool owns the memory, and
+ * cudaFree waits for the whole device).  Same inputs, outputs and results as
+ * tria_prune, but the workspace is a fixed array of TRIA_NOALLOC_SCRATCH_BYTES
+ * inside the library's device image, held by every device that loads the
+ * library until the process exits; the call allocates nothing.
+ *   - Problems whose tria_workspace_size exceeds TRIA_NOALLOC_SCRATCH_BYTES
+ *     return TRIA_ERR_UNSUPPORTED before anything is launched (16 MiB holds,
+ *     for example, one layer of 32 query heads over 32768 cached slots).
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress (with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the array.  Each call clears the array's
+ *     error word, the only part that must start at zero; calls whose kernels
+ *     may overlap on one device (different streams, no ordering) race.
+ *   - device_error, if not NULL, is a DEVICE int32 that receives the call's
+ *     device error word (TRIA_DEVERR_* bits, 0 if none) at the end of the call,
+ *     in stream order; the scratch cannot be passed to tria_get_device_error.
+ */
+#define TRIA_NOALLOC_SCRATCH_BYTES (16 << 20)
+tria_status tria_prune_noalloc(const tria_config *cfg, const tria_stats *stats,
+                               const tria_cache *cache, int32_t *sel_out, int32_t *device_error,
+                               void *stream);
+
 /* Human-readable name of a status. */
 const char *tria_status_string(tria_status s);
 

@@ -32,6 +32,7 @@ MAX_BATCH = 256
 MAX_OFFSETS = 4096
 MAX_SEGMENT = 1 << 18
 PRUNE_MAX_STAGES = 8
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 DEVERR_SEQ_LEN = 1
 DEVERR_SELECTION = 2
@@ -40,7 +41,8 @@ DEVERR_SEGMENT_BIG = 8
 
 EXPORTS = ["tria_workspace_size", "tria_workspace_init", "tria_calibrate", "tria_score",
            "tria_select", "tria_compact", "tria_prune", "tria_prune_profiled",
-           "tria_prune_stage_name", "tria_get_device_error", "tria_status_string", "tria_version"]
+           "tria_prune_stage_name", "tria_get_device_error", "tria_status_string", "tria_version",
+           "tria_prune_noalloc"]
 
 
 class TriaError(RuntimeError):
@@ -94,6 +96,8 @@ def lib():
                                  ctypes.c_size_t, vp]
         L.tria_prune_profiled.argtypes = [P(tria_config), P(tria_stats), P(tria_cache), vp, vp,
                                           ctypes.c_size_t, vp, P(vp), P(ctypes.c_int32)]
+        L.tria_prune_noalloc.argtypes = [P(tria_config), P(tria_stats), P(tria_cache), vp, vp,
+                                         vp]
         L.tria_prune_stage_name.argtypes = [ctypes.c_int32]
         L.tria_prune_stage_name.restype = ctypes.c_char_p
         L.tria_get_device_error.argtypes = [vp, P(ctypes.c_int32), vp]
@@ -252,6 +256,18 @@ def tria_prune_profiled(cfg: Config, stats: Stats, cache: Cache, ws: torch.Tenso
                                      _stream(stream), arr, ctypes.byref(n)),
            "tria_prune_profiled")
     return int(n.value)
+
+
+def tria_prune_noalloc(cfg: Config, stats: Stats, cache: Cache,
+                       sel_out: Optional[torch.Tensor] = None,
+                       device_error: Optional[torch.Tensor] = None, stream=None):
+    """tria_prune without a workspace argument: the library's fixed device
+    scratch array stands in for it (see include/tria.h).  device_error, if
+    given, is an int32 device tensor of one element that receives the call's
+    device error word."""
+    _check(lib().tria_prune_noalloc(ctypes.byref(cfg.c), ctypes.byref(stats.c),
+                                    ctypes.byref(cache.c), _ptr(sel_out), _ptr(device_error),
+                                    _stream(stream)), "tria_prune_noalloc")
 
 
 def tria_prune_stage_name(i: int) -> str:

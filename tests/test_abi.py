@@ -45,6 +45,7 @@ def test_header_constants_match_binding():
     assert int(consts["TRIA_NO_TRIG"]) == tria.NO_TRIG
     assert int(consts["TRIA_NO_CONC_WEIGHT"]) == tria.NO_CONC_WEIGHT
     assert int(consts["TRIA_PRUNE_MAX_STAGES"]) == tria.PRUNE_MAX_STAGES
+    assert eval(consts["TRIA_NOALLOC_SCRATCH_BYTES"]) == tria.NOALLOC_SCRATCH_BYTES
 
 
 def test_status_strings(L):

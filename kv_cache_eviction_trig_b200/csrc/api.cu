@@ -12,25 +12,17 @@ namespace tria {
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap) {
+  (void)seq_start;
   WsLayout w{};
   const size_t F = (size_t)cfg.head_dim / 2;
-  const int64_t tile = score_tile_keys(cfg.head_dim > 0 ? cfg.head_dim : 2);
-  int64_t max_tiles = 0;
-  for (int b = 0; b < cfg.batch; ++b) {
-    const int64_t t = (seq_start[b + 1] - seq_start[b] + tile - 1) / tile;
-    if (t > max_tiles) max_tiles = t;
-  }
-  w.max_slots = (int32_t)(max_tiles + 1);
   const size_t units = (size_t)cfg.num_layers * cfg.n_kv_heads * cfg.batch;
   const size_t G = cfg.n_kv_heads > 0 ? (size_t)(cfg.n_q_heads / cfg.n_kv_heads) : 1;
   size_t o = 0;
   w.err = o;      o += 256;
   w.seqlen = o;   o = align_up(o + 4ull * cfg.batch, 256);
-  w.ea = o;       o = align_up(o + 16ull * cfg.batch * F, 256);
+  w.w = o;        o = align_up(o + 4ull * units * (F / 2) * G * 6, 256);
   w.raw = o;      o = align_up(o + 4ull * cfg.num_layers * cfg.n_q_heads * (size_t)cap, 256);
-  w.score = o;
   w.sel = o;      o = align_up(o + 4ull * units * cfg.budget, 256);
-  w.partials = o; o = align_up(o + 16ull * units * w.max_slots * G, 256);
   w.total = o;
   return w;
 }
@@ -100,6 +92,12 @@ tria_status check_cache(const tria_config *cfg, const tria_cache *c, bool need_k
   return TRIA_OK;
 }
 
+// The score kernel addresses keys by 32-bit tensor coordinates.
+tria_status check_key_rows(const tria_config *cfg, const tria_cache *c) {
+  const int64_t rows = (int64_t)cfg->num_layers * cfg->n_kv_heads * c->cap_total;
+  return rows <= INT32_MAX ? TRIA_OK : TRIA_ERR_UNSUPPORTED;
+}
+
 tria_status check_stats(const tria_stats *s) {
   if (!s || !s->centre || !s->mean_norm || !s->mrl) return TRIA_ERR_INVALID_ARG;
   if (!aligned(s->centre, 8) || !aligned(s->mean_norm, 4) || !aligned(s->mrl, 4))
@@ -115,38 +113,39 @@ tria_status check_ws(const tria_config *cfg, const tria_cache *c, void *ws, size
 
 tria_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TRIA_OK : TRIA_ERR_CUDA; }
 
-void fill_fold(FoldParams &fp, const tria_config *cfg, const tria_cache *c, int32_t *seqlen_snap,
-               double2 *ea, int32_t *err) {
+void fill_fold(FoldParams &fp, const tria_config *cfg, const tria_stats *st,
+               const tria_cache *c, int32_t *seqlen_snap, float *w, int32_t *err) {
   std::memset(&fp, 0, sizeof fp);
   fp.cur_pos = c->cur_pos;
   fp.seq_len = c->seq_len;
   fp.seqlen_snap = seqlen_snap;
-  fp.ea = ea;
   fp.err = err;
+  fp.centre = reinterpret_cast<const float2 *>(st->centre);
+  fp.mean_norm = st->mean_norm;
+  fp.mrl = st->mrl;
+  fp.w = w;
   fp.theta = cfg->rope_theta;
   fp.D = cfg->head_dim;
   fp.B = cfg->batch;
+  fp.L = cfg->num_layers;
+  fp.Hkv = cfg->n_kv_heads;
+  fp.Hq = cfg->n_q_heads;
+  fp.G = cfg->n_q_heads / cfg->n_kv_heads;
   fp.n_offsets = cfg->n_offsets;
   fp.flags = cfg->flags;
   for (int b = 0; b < cfg->batch; ++b) fp.seg_cap[b] = c->seq_start[b + 1] - c->seq_start[b];
   std::memcpy(fp.offsets, cfg->offsets, sizeof(int32_t) * cfg->n_offsets);
 }
 
-// Builds the score kernel parameters; returns the grid size (0: nothing to launch).
-int fill_score(ScoreParams &sp, const tria_config *cfg, const tria_stats *st, const tria_cache *c,
-               const double2 *ea, float *raw, double *partials, int32_t max_slots, int32_t *err,
-               int skip_short) {
+// Builds the score kernel parameters; *grid receives the grid size (0: nothing to launch).
+cudaError_t fill_score(ScoreParams &sp, const tria_config *cfg, const tria_cache *c,
+                       const float *w, float *raw, int32_t *err, int skip_short, int *grid) {
   std::memset(&sp, 0, sizeof sp);
-  const int tile = score_tile_keys(cfg->head_dim);
-  sp.k = static_cast<const uint8_t *>(c->k);
-  sp.centre = reinterpret_cast<const float2 *>(st->centre);
-  sp.mean_norm = st->mean_norm;
-  sp.mrl = st->mrl;
-  sp.ea = ea;
+  const int G = cfg->n_q_heads / cfg->n_kv_heads;
+  const int ch = score_chunk_keys(cfg->head_dim, G);
+  sp.w = w;
   sp.seq_len = c->seq_len;
   sp.raw = raw;
-  sp.partials = partials;
-  sp.max_slots = max_slots;
   sp.err = err;
   sp.cap = c->cap_total;
   sp.L = cfg->num_layers;
@@ -155,21 +154,27 @@ int fill_score(ScoreParams &sp, const tria_config *cfg, const tria_stats *st, co
   sp.B = cfg->batch;
   sp.budget = cfg->budget;
   sp.skip_short = skip_short;
-  sp.no_conc_weight = (cfg->flags & TRIA_NO_CONC_WEIGHT) ? 1 : 0;
   int32_t acc = 0;
   for (int b = 0; b <= cfg->batch; ++b) {
     sp.seg_start[b] = c->seq_start[b];
-    sp.tile_prefix[b] = acc;
-    if (b < cfg->batch) acc += (int32_t)((c->seq_start[b + 1] - c->seq_start[b] + tile - 1) / tile);
+    sp.chunk_prefix[b] = acc;
+    if (b < cfg->batch) acc += (int32_t)((c->seq_start[b + 1] - c->seq_start[b] + ch - 1) / ch);
   }
-  sp.tiles_per_row = acc;
-  sp.total_tiles = (int64_t)cfg->num_layers * cfg->n_kv_heads * acc;
-  if (sp.total_tiles == 0) return 0;
-  int64_t grid = device_sm_count();
-  if (grid > sp.total_tiles) grid = sp.total_tiles;
-  sp.tiles_per_cta = (int32_t)((sp.total_tiles + grid - 1) / grid);
-  grid = (sp.total_tiles + sp.tiles_per_cta - 1) / sp.tiles_per_cta;
-  return (int)grid;
+  sp.chunks_per_row = acc;
+  const int64_t total = (int64_t)cfg->num_layers * cfg->n_kv_heads * acc;
+  *grid = 0;
+  if (total > INT32_MAX - 64) return cudaErrorInvalidValue;  // excluded by check_key_rows
+  sp.total_chunks = (int32_t)total;
+  if (total == 0) return cudaSuccess;
+  int64_t g = device_sm_count();
+  if (g > total) g = total;
+  sp.chunks_per_cta = (int32_t)((total + g - 1) / g);
+  g = (total + sp.chunks_per_cta - 1) / sp.chunks_per_cta;
+  const int64_t rows = (int64_t)cfg->num_layers * cfg->n_kv_heads * c->cap_total;
+  cudaError_t e = make_key_tensor_map(&sp.tmap, c->k, cfg->head_dim, rows, ch);
+  if (e != cudaSuccess) return e;
+  *grid = (int)g;
+  return cudaSuccess;
 }
 
 void fill_unit(UnitParams &up, const tria_config *cfg, const tria_cache *c, int mode) {
@@ -186,24 +191,8 @@ void fill_unit(UnitParams &up, const tria_config *cfg, const tria_cache *c, int 
   up.D = cfg->head_dim;
   up.budget = cfg->budget;
   up.mode = mode;
-  int64_t max_seg = 0;
-  for (int b = 0; b <= cfg->batch; ++b) {
-    up.seg_start[b] = c->seq_start[b];
-    if (b < cfg->batch && c->seq_start[b + 1] - c->seq_start[b] > max_seg)
-      max_seg = c->seq_start[b + 1] - c->seq_start[b];
-  }
-  up.smem_bytes = unit_smem_bytes(cfg->num_layers * cfg->n_kv_heads * cfg->batch, max_seg);
-}
-
-// The unit kernel finds the score kernel's partial sums through its tile decomposition.
-void link_unit_to_score(UnitParams &up, const ScoreParams &sp, const double *partials,
-                        int tile_keys) {
-  up.partials = partials;
-  up.max_slots = sp.max_slots;
-  up.tiles_per_cta = sp.tiles_per_cta > 0 ? sp.tiles_per_cta : 1;
-  up.tiles_per_row = sp.tiles_per_row;
-  up.tile_keys = tile_keys;
-  for (int b = 0; b <= TRIA_MAX_BATCH; ++b) up.tile_prefix[b] = sp.tile_prefix[b];
+  for (int b = 0; b <= cfg->batch; ++b) up.seg_start[b] = c->seq_start[b];
+  up.smem_bytes = unit_smem_bytes();
 }
 
 struct Ws {
@@ -211,10 +200,9 @@ struct Ws {
   uint8_t *base;
   int32_t *err() const { return reinterpret_cast<int32_t *>(base + lay.err); }
   int32_t *seqlen() const { return reinterpret_cast<int32_t *>(base + lay.seqlen); }
-  double2 *ea() const { return reinterpret_cast<double2 *>(base + lay.ea); }
+  float *w() const { return reinterpret_cast<float *>(base + lay.w); }
   float *raw() const { return reinterpret_cast<float *>(base + lay.raw); }
   int32_t *sel() const { return reinterpret_cast<int32_t *>(base + lay.sel); }
-  double *partials() const { return reinterpret_cast<double *>(base + lay.partials); }
 };
 
 const char *kStageNames[] = {"fold_kernel", "score_kernel", "unit_kernel"};
@@ -263,6 +251,7 @@ tria_status tria_score(const tria_config *cfg, const tria_stats *stats, const tr
   if ((s = check_config(cfg, true)) != TRIA_OK) return s;
   if ((s = check_cache(cfg, cache, false)) != TRIA_OK) return s;
   if (!cache->k || !aligned(cache->k, 16) || !cache->cur_pos) return TRIA_ERR_INVALID_ARG;
+  if ((s = check_key_rows(cfg, cache)) != TRIA_OK) return s;
   if ((s = check_stats(stats)) != TRIA_OK) return s;
   if (!score || (raw && !aligned(raw, 4))) return TRIA_ERR_INVALID_ARG;
   if ((s = check_ws(cfg, cache, ws, ws_bytes)) != TRIA_OK) return s;
@@ -271,20 +260,17 @@ tria_status tria_score(const tria_config *cfg, const tria_stats *stats, const tr
   float *rawp = raw ? raw : w.raw();
 
   static thread_local FoldParams fp;
-  fill_fold(fp, cfg, cache, w.seqlen(), w.ea(), w.err());
-  cudaError_t e = launch_fold(fp, cfg->head_dim / 2, st);
-  if (e != cudaSuccess) return TRIA_ERR_CUDA;
+  fill_fold(fp, cfg, stats, cache, w.seqlen(), w.w(), w.err());
   ScoreParams sp;
-  const int grid = fill_score(sp, cfg, stats, cache, w.ea(), rawp, w.partials(),
-                              w.lay.max_slots, w.err(), 0);
-  if (grid > 0) {
-    e = launch_score(sp, cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads, cfg->rope_layout, grid,
-                     st, true);
-    if (e != cudaSuccess) return TRIA_ERR_CUDA;
-  }
+  int grid = 0;
+  if (fill_score(sp, cfg, cache, w.w(), rawp, w.err(), 0, &grid) != cudaSuccess)
+    return TRIA_ERR_CUDA;
+  if (launch_fold(fp, st) != cudaSuccess) return TRIA_ERR_CUDA;
+  if (grid > 0 && launch_score(sp, cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads,
+                               cfg->rope_layout, grid, st, true) != cudaSuccess)
+    return TRIA_ERR_CUDA;
   UnitParams up;
   fill_unit(up, cfg, cache, kModeZmax);
-  link_unit_to_score(up, sp, w.partials(), score_tile_keys(cfg->head_dim));
   up.raw = rawp;
   up.score = score;
   up.seqlen = w.seqlen();
@@ -335,6 +321,7 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
   if ((s = check_config(cfg, true)) != TRIA_OK) return s;
   if ((s = check_cache(cfg, cache, true)) != TRIA_OK) return s;
   if (!cache->cur_pos) return TRIA_ERR_INVALID_ARG;
+  if ((s = check_key_rows(cfg, cache)) != TRIA_OK) return s;
   if ((s = check_stats(stats)) != TRIA_OK) return s;
   if (sel_out && !aligned(sel_out, 4)) return TRIA_ERR_INVALID_ARG;
   if ((s = check_ws(cfg, cache, ws, ws_bytes)) != TRIA_OK) return s;
@@ -349,20 +336,20 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
   };
 
   static thread_local FoldParams fp;
-  fill_fold(fp, cfg, cache, w.seqlen(), w.ea(), w.err());
-  if (!mark()) return TRIA_ERR_CUDA;
-  if (launch_fold(fp, cfg->head_dim / 2, st) != cudaSuccess) return TRIA_ERR_CUDA;
+  fill_fold(fp, cfg, stats, cache, w.seqlen(), w.w(), w.err());
   ScoreParams sp;
-  const int grid = fill_score(sp, cfg, stats, cache, w.ea(), w.raw(), w.partials(),
-                              w.lay.max_slots, w.err(), 1);
+  int grid = 0;
+  if (fill_score(sp, cfg, cache, w.w(), w.raw(), w.err(), 1, &grid) != cudaSuccess)
+    return TRIA_ERR_CUDA;
   const bool pdl = events == nullptr;  // stage events between kernels would defeat the overlap
+  if (!mark()) return TRIA_ERR_CUDA;
+  if (launch_fold(fp, st) != cudaSuccess) return TRIA_ERR_CUDA;
   if (!mark()) return TRIA_ERR_CUDA;
   if (grid > 0 && launch_score(sp, cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads,
                                cfg->rope_layout, grid, st, pdl) != cudaSuccess)
     return TRIA_ERR_CUDA;
   UnitParams up;
   fill_unit(up, cfg, cache, kModePrune);
-  link_unit_to_score(up, sp, w.partials(), score_tile_keys(cfg->head_dim));
   up.raw = w.raw();
   up.sel = sel_out ? sel_out : w.sel();
   up.write_short_sel = sel_out ? 1 : 0;

@@ -1,15 +1,20 @@
-// Fold of the future-offset average and the current position into one complex
-// factor per (sequence, RoPE pair).
+// Fold of the future-offset average, the current position and the calibrated
+// query statistics into one weight triple per (unit, query head, RoPE pair).
 //
 // The trigonometric term of the key score (romaanj.github.io review, "Method";
 // dimensionstp.github.io review, section 2-2) is
 //   S_trig = mean_delta sum_f |c_f||k_f| cos(w_f (cur + delta - p) + arg c_f - arg k_f).
 // With the pre-RoPE key k_f = ktilde_f e^{-i w_f p} the key's position p cancels
-// and the sum becomes Re sum_f conj(ktilde_f) * c_f * EA_f with
-//   EA_f = e^{i w_f cur} * (1/|O|) sum_{delta in O} e^{i w_f delta},
-// so the per-key work needs no position and no trigonometry.  EA is formed
-// here in float64 (angles reach ~1e5 rad); block f handles pair f.
-// Block 0 also snapshots and checks seq_len, so that every later kernel of
+// and the sum becomes Re sum_f conj(ktilde_f) * W_f with
+//   W_f  = c_f * EA_f,   EA_f = e^{i w_f cur} * (1/|O|) sum_{delta in O} e^{i w_f delta},
+// so the per-key work needs no position and no trigonometry.  The norm term's
+// weight is Nw_f = (1 - R_f) E|q_f| (section 3-2 (3)-(4)).
+//
+// Block (fp, y) handles the RoPE pairs f = 2fp, 2fp+1: it forms EA in float64
+// (angles reach ~1e5 rad) for every sequence, then writes, for a share y of
+// the (unit, head) pairs, the float32 weights
+//   w[unit][fp][h] = (Re W_2fp, Re W_2fp+1, Im W_2fp, Im W_2fp+1, Nw_2fp, Nw_2fp+1).
+// Block (0, 0) also snapshots and checks seq_len, so that every later kernel of
 // the call sees the lengths as they were at its start.
 #include "tria_internal.cuh"
 
@@ -17,40 +22,77 @@ namespace tria {
 
 __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldParams p) {
   dev::pdl_launch_dependents();  // the score kernel may start streaming keys now
-  const int f = blockIdx.x;
-  const double w = pow(p.theta, -2.0 * (double)f / (double)p.D);
-  double sc = 0.0, ss = 0.0;
+  const int fp = blockIdx.x;
+  const int F = p.D / 2;
+  __shared__ double red[4][8];
+  __shared__ double2 ea[TRIA_MAX_BATCH][2];
+  double w[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) w[q] = pow(p.theta, -2.0 * (double)(2 * fp + q) / (double)p.D);
+  double a[4] = {0.0, 0.0, 0.0, 0.0};  // (cos, sin) sums for the two pairs
   for (int j = threadIdx.x; j < p.n_offsets; j += blockDim.x) {
-    double s, c;
-    sincos(w * (double)p.offsets[j], &s, &c);
-    sc += c;
-    ss += s;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      double s, c;
+      sincos(w[q] * (double)p.offsets[j], &s, &c);
+      a[2 * q] += c;
+      a[2 * q + 1] += s;
+    }
   }
   // fixed-order block reduction (deterministic)
-  for (int o = 16; o > 0; o >>= 1) {
-    sc += __shfl_xor_sync(0xffffffffu, sc, o);
-    ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  }
-  __shared__ double red[2][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    for (int o = 16; o > 0; o >>= 1) a[i] += __shfl_xor_sync(0xffffffffu, a[i], o);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) { red[0][warp] = sc; red[1][warp] = ss; }
+  if (lane == 0)
+    for (int i = 0; i < 4; ++i) red[i][warp] = a[i];
   __syncthreads();
-  if (threadIdx.x == 0) {
-    double a = 0.0, b = 0.0;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) { a += red[0][i]; b += red[1][i]; }
-    red[0][0] = a / (double)p.n_offsets;
-    red[1][0] = b / (double)p.n_offsets;
+  double A[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    double s = 0.0;
+    for (int k = 0; k < (int)(blockDim.x >> 5); ++k) s += red[i][k];
+    A[i] = (p.flags & TRIA_NO_TRIG) ? 0.0 : s / (double)p.n_offsets;
   }
-  __syncthreads();
-  double ax = red[0][0], ay = red[1][0];
-  if (p.flags & TRIA_NO_TRIG) { ax = 0.0; ay = 0.0; }
-  const int F = p.D / 2;
   for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
-    double s, c;
-    sincos(w * (double)p.cur_pos[b], &s, &c);
-    p.ea[(size_t)b * F + f] = make_double2(c * ax - s * ay, c * ay + s * ax);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      double s, c;
+      sincos(w[q] * (double)p.cur_pos[b], &s, &c);
+      const double ax = A[2 * q], ay = A[2 * q + 1];
+      ea[b][q] = make_double2(c * ax - s * ay, c * ay + s * ax);
+    }
   }
-  if (f == 0) {
+  __syncthreads();
+
+  const int64_t units = (int64_t)p.L * p.Hkv * p.B;
+  const int64_t entries = units * p.G;
+  const int FP = F / 2;
+  for (int64_t e = (int64_t)blockIdx.y * blockDim.x + threadIdx.x; e < entries;
+       e += (int64_t)gridDim.y * blockDim.x) {
+    const int64_t unit = e / p.G;
+    const int h = (int)(e - unit * p.G);
+    const int b = (int)(unit % p.B);
+    const int64_t lg = unit / p.B;
+    const int l = (int)(lg / p.Hkv), g = (int)(lg % p.Hkv);
+    const size_t base = ((size_t)l * p.Hq + (size_t)g * p.G + h) * F + 2 * fp;
+    float wx[2], wy[2], nw[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const float2 c = p.centre[base + q];
+      const double2 e2 = ea[b][q];
+      wx[q] = (float)((double)c.x * e2.x - (double)c.y * e2.y);
+      wy[q] = (float)((double)c.x * e2.y + (double)c.y * e2.x);
+      const float r = (p.flags & TRIA_NO_CONC_WEIGHT) ? 0.0f : p.mrl[base + q];
+      nw[q] = (1.0f - r) * p.mean_norm[base + q];
+    }
+    float2 *out = reinterpret_cast<float2 *>(p.w + ((size_t)unit * FP + fp) * (6 * p.G) + 6 * h);
+    out[0] = make_float2(wx[0], wx[1]);
+    out[1] = make_float2(wy[0], wy[1]);
+    out[2] = make_float2(nw[0], nw[1]);
+  }
+
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
     for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
       int32_t T = p.seq_len[b];
       if (T < 0 || (int64_t)T > p.seg_cap[b]) {
@@ -62,8 +104,14 @@ __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldP
   }
 }
 
-cudaError_t launch_fold(const FoldParams &p, int F, cudaStream_t s) {
-  fold_kernel<<<F, 256, 0, s>>>(p);
+cudaError_t launch_fold(const FoldParams &p, cudaStream_t s) {
+  const int FP = p.D / 4;
+  const int64_t entries = (int64_t)p.L * p.Hkv * p.B * p.G;
+  // about 8 entries per thread, at most 64 blocks per pair
+  int64_t y = (entries + 2047) / 2048;
+  if (y < 1) y = 1;
+  if (y > 64) y = 64;
+  fold_kernel<<<dim3((unsigned)FP, (unsigned)y), 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -2,6 +2,7 @@
 // Device primitives are written directly in PTX for sm_100a.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -13,60 +14,59 @@ namespace tria {
 struct WsLayout {
   size_t err;       // int32 device error word (+ padding)
   size_t seqlen;    // int32 [B]   snapshot of seq_len taken at the start of a call
-  size_t ea;        // double2 [B][F]  e^{i w_f cur_b} * mean_delta e^{i w_f delta}
+  size_t w;         // float [L*Hkv*B][D/4][G][6]  folded weights (fold kernel)
   size_t raw;       // float [L][Hq][cap]  raw scores when the caller gives none
-  size_t score;     // float [L][Hkv][cap] group-max z-scores (tria_prune does not need it)
   size_t sel;       // int32 [L][Hkv][B][budget] selection scratch
-  size_t partials;  // double [L*Hkv*B][max_slots][G][2] per-CTA sums of s and s^2
-  int32_t max_slots;
   size_t total;
 };
 WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap_total);
 
 // ------------------------------------------------------------------ kernel parameters
-constexpr int kScoreConsumerWarps = 16;
+#ifndef TRIA_SCORE_WARPS
+#define TRIA_SCORE_WARPS 8
+#endif
+#ifndef TRIA_SCORE_KPT_CAP
+#define TRIA_SCORE_KPT_CAP 4
+#endif
+constexpr int kScoreConsumerWarps = TRIA_SCORE_WARPS;  // build-time tunables
+constexpr int kScoreKptCap = TRIA_SCORE_KPT_CAP;
 constexpr int kScoreThreads = (kScoreConsumerWarps + 1) * 32;
-constexpr int kScoreStages = 3;
-constexpr int kScoreTileBytes = 64 * 1024;   // bytes of K per pipeline stage
+constexpr int kScoreRingBytes = 192 * 1024;  // shared-memory ring of key chunks
 
 constexpr int kUnitThreads = 1024;
 constexpr int kUnitCluster = 8;
-constexpr int kUnitSmemSmall = 112 * 1024;  // smaller footprint (more clusters resident)
 constexpr int kUnitSmemLarge = 200 * 1024;  // one CTA per SM
 
 struct FoldParams {
   const int32_t *cur_pos;   // [B]
   const int32_t *seq_len;   // [B] caller's live lengths
   int32_t *seqlen_snap;     // [B] out
-  double2 *ea;              // [B][F] out
   int32_t *err;
+  const float2 *centre;     // [L][Hq][F]
+  const float *mean_norm;   // [L][Hq][F]
+  const float *mrl;         // [L][Hq][F]
+  float *w;                 // [L*Hkv*B][F/2][G][6] out
   double theta;
-  int32_t D, B, n_offsets;
+  int32_t D, B, L, Hkv, Hq, G, n_offsets;
   uint32_t flags;
   int64_t seg_cap[TRIA_MAX_BATCH];
   int32_t offsets[TRIA_MAX_OFFSETS];
 };
 
-struct ScoreParams {
-  const uint8_t *k;         // bf16 rows [L][Hkv][cap][D]
-  const float2 *centre;     // [L][Hq][F]
-  const float *mean_norm;   // [L][Hq][F]
-  const float *mrl;         // [L][Hq][F]
-  const double2 *ea;        // [B][F]  (written by the fold kernel)
+struct alignas(64) ScoreParams {
+  CUtensorMap tmap;         // K as a 2-D bf16 tensor [L*Hkv*cap][D], 128-byte swizzled boxes
+  const float *w;           // folded weights (written by the fold kernel)
   const int32_t *seq_len;   // [B] caller's live lengths (not modified during the call)
   float *raw;               // [L][Hq][cap]
-  double *partials;         // [units][max_slots][G][2]
   int32_t *err;
   int64_t cap;
-  int32_t max_slots;
   int32_t L, Hkv, Hq, B, budget;
   int32_t skip_short;       // 1: sequences with seq_len <= budget are not scored
-  int32_t no_conc_weight;   // ablation flag
-  int32_t tiles_per_row;    // tile_prefix[B]
-  int32_t tiles_per_cta;
-  int64_t total_tiles;
+  int32_t chunks_per_row;   // chunk_prefix[B]
+  int32_t chunks_per_cta;
+  int32_t total_chunks;     // < 2^31 (checked on the host)
   int64_t seg_start[TRIA_MAX_BATCH + 1];
-  int32_t tile_prefix[TRIA_MAX_BATCH + 1];
+  int32_t chunk_prefix[TRIA_MAX_BATCH + 1];
 };
 
 enum UnitMode : int32_t { kModeZmax = 0, kModeSelect = 1, kModeCompact = 2, kModePrune = 3 };
@@ -76,9 +76,6 @@ struct UnitParams {
   uint8_t *v;
   int32_t *pos;
   const float *raw;         // [L][Hq][cap]      (zmax, prune)
-  const double *partials;   // [units][max_slots][G][2] from the score kernel (zmax, prune)
-  int32_t max_slots, tiles_per_cta, tiles_per_row, tile_keys;
-  int32_t tile_prefix[TRIA_MAX_BATCH + 1];
   float *score;             // [L][Hkv][cap]     (zmax writes, select reads)
   int32_t *sel;             // [L][Hkv][B][budget]
   const int32_t *seqlen;    // [B] snapshot (zmax, select, prune)
@@ -93,14 +90,17 @@ struct UnitParams {
 };
 
 // ------------------------------------------------------------------ launchers (host)
-cudaError_t launch_fold(const FoldParams &p, int F, cudaStream_t s);
+cudaError_t launch_fold(const FoldParams &p, cudaStream_t s);
 cudaError_t launch_score(const ScoreParams &p, int D, int G, int layout, int grid,
                          cudaStream_t s, bool pdl);
 bool score_supported(int D, int G, int layout);
-int score_tile_keys(int D);
+int score_chunk_keys(int D, int G);
+// Encodes the tensor map of the key cache viewed as [rows][D] bf16.
+cudaError_t make_key_tensor_map(CUtensorMap *map, const void *k, int D, int64_t rows,
+                                int box_rows);
 cudaError_t launch_unit(const UnitParams &p, int units, cudaStream_t s, bool pdl);
 int unit_cluster_size();
-int unit_smem_bytes(int units, int64_t max_segment);
+int unit_smem_bytes();
 cudaError_t launch_calibrate(const void *q, int q_dtype, int64_t L, int64_t N, int64_t Hq,
                              int64_t D, int layout, float *centre, float *mean_norm, float *mrl,
                              cudaStream_t s);
@@ -135,6 +135,11 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+#ifndef TRIA_MBAR_HINT_NS
+#define TRIA_MBAR_HINT_NS 1000
+#endif
+constexpr uint32_t kMbarHintNs = TRIA_MBAR_HINT_NS;  // build-time tunable
+
 // One bounded try: returns true once the phase with the given parity has completed.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t done;
@@ -143,12 +148,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity), "r"(1000u)  // suspend hint: 1 us
+      : "r"(smem_addr(bar)), "r"(parity), "r"(kMbarHintNs)  // suspend-time hint
       : "memory");
   return done != 0;
 }
 
-// Waits with an iteration limit (about 2 s at the 1 us hint); false if it ran out.
+// Waits with an iteration limit (about 2 s at the 1 us hint, and never less than
+// the try's own time limit per iteration); false if it ran out.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
   for (uint32_t i = 0; i < 2000000u; ++i)
     if (mbar_try_wait(bar, parity)) return true;
@@ -161,6 +167,17 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           smem_addr(dst)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// 2-D tiled tensor load global -> shared (box given by the tensor map), completion
+// counted on an mbarrier; no multicast.  x is the innermost (element) coordinate.
+__device__ __forceinline__ void tma_load_2d(void *dst, const void *map, int32_t x, int32_t y,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
       : "memory");
 }
 

@@ -1,32 +1,40 @@
 // Per-unit stages of the prune step: one thread-block cluster per
-// (layer l, KV head g, sequence b).
+// (layer l, KV head g, sequence b); CTA r of the cluster owns the r-th slice of
+// the sequence's keys.
 //
 //   z-score + group max (romaanj.github.io review, "Method"; dimensionstp.github.io
 //     review, section 3-2 (6)): mu_h and the population sigma_h of the raw
 //     scores over the sequence's T live keys; z_h = (s_h - mu_h) / sigma_h
-//     (0 when sigma_h = 0); score = max_h z_h.  mu and sigma come from the
-//     float64 sums of s and s^2 the score kernel leaves per (CTA, head), added
-//     here in a fixed order, so the result is deterministic.
+//     (0 when sigma_h = 0); score = max_h z_h.  mu and sigma come from float64
+//     sums of s and s^2: each CTA sums its keys in a fixed order, and every CTA
+//     adds the cluster's partial sums in rank order, so all CTAs hold the same,
+//     deterministic statistics.
 //   selection (same sources, "prune back to budget"; section 3-2 (5)): the
 //     `budget` largest scores, ties to the lower slot, on order-preserving
-//     32-bit keys.  While the keys are computed, each is counted into a
-//     cluster-wide 12-bit histogram with remote shared-memory atomics (CTA q
-//     owns one eighth of the bins); after one barrier every CTA reads the whole
-//     histogram and names the bucket holding the budget-th key.  Usually that
-//     bucket is small: every CTA then gathers the bucket's keys from all peers
-//     (in slot order) and finishes the selection alone, exactly, so it also
-//     knows how many keys every peer keeps without another exchange.  A bucket
-//     too large to gather is refined by further cluster-wide rounds (12 then 8
-//     bits); if it is still large, its keys are all equal and the ties go to
-//     the lowest slots.
+//     32-bit keys.  While the keys are computed each CTA counts them into a
+//     local 4096-bin histogram (shared-memory atomics).  For z-scores the bins
+//     are a fixed grid of width 1/256 over [-8, 8) (a monotone function of the
+//     key), so the bin holding the budget-th key usually holds a few dozen keys;
+//     for arbitrary scores (tria_select) the bins are the top 12 key bits.  After
+//     one barrier every CTA reads the peers' 64 coarse counts, then the 64 fine
+//     counts of the coarse bin that holds the budget-th key, and so names its
+//     bin.  If that bucket is small, every CTA gathers its keys from all peers
+//     (in slot order) and resolves it alone (pairwise ranks, or local radix
+//     rounds for larger buckets), so it also knows how many keys every peer keeps
+//     without another exchange.  A bucket too large to gather is refined by
+//     cluster-wide rounds on the key bits (12, 12, 8; counts land in the owning
+//     CTA's slice through remote atomics); if it is still large its keys are all
+//     equal and the ties go to the lowest slots.
 //   compaction (eviction): kept rows of K, V and pos move in place to slots
 //     [0, kept).  A kept slot s_j always satisfies s_j >= j, so reading every
-//     source of a batch of destinations before any of them is written (one
-//     cluster barrier per batch) makes the in-place gather race-free: a
-//     destination row j can only be the source of a kept key with index <= j,
-//     which belongs to this batch or an earlier one.  Sources are staged in
-//     shared memory with 16-byte asynchronous copies; each CTA's destination
-//     rows are contiguous and go back with one bulk copy per tensor.
+//     source before any destination of the same batch is written (one cluster
+//     barrier in between) makes the in-place gather race-free.  Normally CTA q
+//     compacts the q-th eighth of the destinations in one batch: whoever emits a
+//     kept key stores its slot straight into q's shared-memory list, q stages the
+//     rows with 16-byte asynchronous copies and writes them back with one bulk
+//     copy per tensor after the barrier.  Larger budgets are compacted in batches
+//     in global destination order read from the selection list: every
+//     destination written in a batch precedes every source of the later batches.
 //
 // Cluster barriers are hardware barriers; there are no spin-waits.  The kernel
 // is launched as a programmatic dependent of the score kernel and waits for it
@@ -41,16 +49,22 @@ namespace tria {
 
 namespace {
 
-constexpr int kCtl = 24 * 1024;  // control region at the start of shared memory
+constexpr int kCtl = 32 * 1024;  // control region at the start of shared memory
 constexpr int kMaxG = 16;
 constexpr int kMaxCluster = 16;
 constexpr int kWarps = kUnitThreads / 32;
-constexpr int kBins = 4096;                   // cluster-wide histogram bins (12-bit digits)
+constexpr int kBins = 4096;                   // cluster-wide histogram bins
 constexpr int kSlice = kBins / kUnitCluster;  // bins each CTA of the cluster owns
+constexpr int kRounds = 3;                    // refinement rounds (12, 12, 8 key bits)
+constexpr int kCoarse = 64;                   // coarse bins of the first round (64 bins each)
 constexpr int kCandMax = 4096;                // bucket keys a CTA may gather
+constexpr int kDirectRank = 256;              // gathered buckets ranked pairwise
 constexpr int kLocalBins = 1024;              // bins of the rounds inside a gathered bucket
+constexpr int kOwnRows = 640;                 // destinations a CTA compacts in one batch
 
 struct Ctl {
+  double wsum[kWarps][2 * kMaxG];   // per-warp partial sums of s and s^2
+  double psum[2 * kMaxG];           // this CTA's partial sums (read by the peers)
   double sums[kMaxG][2];            // the unit's sums of s and s^2 per head
   float mu_hi[kMaxG], mu_lo[kMaxG];  // mean split into two floats (hi + lo)
   float inv_sigma[kMaxG];
@@ -60,8 +74,11 @@ struct Ctl {
   int32_t bc[8];                    // broadcast scalars
   int32_t gcnt[kMaxCluster][2];     // per peer: bucket keys above the threshold, equal to it
   int32_t scan[kWarps + 1];
+  int32_t src[kOwnRows];            // source slots of this CTA's share of the destinations
+  uint32_t coarse[kCoarse];         // this CTA's first-round counts per coarse bin
+  uint32_t gc[kUnitCluster][kCoarse];  // the cluster's coarse counts, then fine counts
   uint32_t lh[kLocalBins];          // histogram of the rounds inside a gathered bucket
-  uint32_t slice[3][kSlice];        // this CTA's slice of the cluster histogram, per round
+  uint32_t slice[kRounds][kSlice];  // this CTA's slice of the cluster histogram, per round
 };
 static_assert(sizeof(Ctl) <= kCtl, "control region too small");
 
@@ -105,6 +122,19 @@ __device__ __forceinline__ void cluster_hist_add(cg::cluster_group &cl, uint32_t
   }
 }
 
+// First-round bin of a z-score key: the float z it encodes on a grid of width
+// 1/256 over [-8, 8), clamped; non-decreasing in the key (NaN keys, which sit
+// at the ends of the key order, go to the end bins).
+__device__ __forceinline__ uint32_t fine_bin(uint32_t key) {
+  const uint32_t u = (key & 0x80000000u) ? (key & 0x7fffffffu) : ~key;
+  const float z = __uint_as_float(u);
+  if (z != z) return (key & 0x80000000u) ? (uint32_t)(kBins - 1) : 0u;
+  const float t = fmaf(z, 256.0f, 2048.0f);
+  if (!(t >= 0.0f)) return 0u;
+  if (t >= (float)(kBins - 1)) return (uint32_t)(kBins - 1);
+  return (uint32_t)t;
+}
+
 // Finds, in a histogram of `nbins` counts ordered by increasing key, the bin
 // holding the krem-th largest counted key.  Every thread returns the bin, the
 // number of counted keys above it and the bin's own count (block-wide).
@@ -139,10 +169,42 @@ __device__ __forceinline__ void find_bin(const uint32_t *tot, int nbins, int kre
   __syncthreads();
 }
 
+// One warp: in the counts cnt[q][i] of CL peers over 64 bins ordered by
+// increasing key, the bin holding the krem-th largest counted key, the number
+// of counted keys above it and its own count (returned to every lane).
+__device__ __forceinline__ void warp_find_bin64(const uint32_t *cnt, int krem, int *bin, int *above,
+                                                int *count) {
+  const int lane = threadIdx.x & 31;
+  const int bh = 63 - 2 * lane, bl = 62 - 2 * lane;  // this lane's bins, higher first
+  int ch = 0, cl_ = 0;
+#pragma unroll
+  for (int q = 0; q < kUnitCluster; ++q) {
+    ch += (int)cnt[q * 64 + bh];
+    cl_ += (int)cnt[q * 64 + bl];
+  }
+  const int s = ch + cl_;
+  int incl = s;  // keys in this lane's bins and in all higher bins
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  const int higher = incl - s;
+  const bool mine = higher < krem && krem <= incl;
+  const uint32_t who = __ballot_sync(0xffffffffu, mine);
+  const int src = who ? __ffs(who) - 1 : 0;
+  int b = bh, a = higher, c = ch;
+  if (higher + ch < krem) { b = bl; a = higher + ch; c = cl_; }
+  *bin = __shfl_sync(0xffffffffu, b, src);
+  *above = __shfl_sync(0xffffffffu, a, src);
+  *count = __shfl_sync(0xffffffffu, c, src);
+}
+
 // Peer whose range [off[q], off[q+1]) holds index i (off has CL+1 entries).
-__device__ __forceinline__ int owner_of(const int32_t *off, int CL, int i) {
+__device__ __forceinline__ int owner_of(const int32_t *off, int i) {
   int q = 0;
-  while (q + 1 < CL && off[q + 1] <= i) ++q;
+#pragma unroll
+  for (int k = 1; k < kUnitCluster; ++k) q += off[k] <= i;
   return q;
 }
 
@@ -169,14 +231,30 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
-__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Stages rows src[0..m) of K and V (ROW bytes each) and of pos into shared memory
+// with 16-byte (4-byte for pos) asynchronous copies, and waits for them.
+__device__ __forceinline__ void stage_rows(const int32_t *src, int m, const uint8_t *kg,
+                                           const uint8_t *vg, const int32_t *pg, uint8_t *sk,
+                                           uint8_t *sv, int32_t *sp, int ROW, int vlog2) {
+  const int VPR = ROW >> 4;
+  for (int it = threadIdx.x; it < (m << (vlog2 + 1)); it += blockDim.x) {
+    const int jj = it >> (vlog2 + 1), w = it & ((2 << vlog2) - 1);
+    const size_t s = (size_t)src[jj];
+    if (w < VPR) cp_async16(sk + (size_t)jj * ROW + 16 * w, kg + s * ROW + 16 * w);
+    else cp_async16(sv + (size_t)jj * ROW + 16 * (w - VPR), vg + s * ROW + 16 * (w - VPR));
+  }
+  for (int jj = threadIdx.x; jj < m; jj += blockDim.x) cp_async4(sp + jj, pg + src[jj]);
+  cp_async_wait_all();
+  fence_proxy_async_smem();  // the staged rows are read back by bulk copies
+}
 
 }  // namespace
 
 template <int G>
 __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_constant__ UnitParams p) {
   cg::cluster_group cl = cg::this_cluster();
-  const int CL = (int)cl.num_blocks();
+  constexpr int CL = kUnitCluster;
   const int r = (int)cl.block_rank();
   const int64_t unit = blockIdx.x / CL;
   const int b = (int)(unit % p.B);
@@ -193,10 +271,19 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
   const size_t data_bytes = (size_t)p.smem_bytes - kCtl;
   int32_t *sel = p.sel + (row * p.B + b) * (int64_t)p.budget;
 
+  const int ROW = 2 * p.D;                    // bytes per K or V row
+  const int vlog2 = 31 - __clz(ROW >> 4);     // log2 of 16-byte vectors per row
+  const int64_t rbase = row * p.cap + seg;
+  uint8_t *kg = p.k + (size_t)rbase * ROW;
+  uint8_t *vg = p.v + (size_t)rbase * ROW;
+  int32_t *pg = p.pos + rbase;
+
   // prologue (overlaps the score kernel's tail): clear the histogram slices of all
-  // rounds, and make sure every peer has before anyone counts into them
-  for (int i = tid; i < 3 * kSlice; i += nthr) (&c.slice[0][0])[i] = 0u;
-  cl.sync();
+  // rounds; the first cluster barrier below makes every peer's clearing visible
+  // before anyone counts into them
+  for (int i = tid; i < kRounds * kSlice; i += nthr) (&c.slice[0][0])[i] = 0u;
+  const bool zmodes = p.mode == kModeZmax || p.mode == kModePrune;
+  if (!zmodes) cl.sync();
   dev::pdl_wait();
 
   int kept = 0;
@@ -252,62 +339,102 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     const int n = (int)(hi - lo);
     const int nmax = (int)((T + CL - 1) / CL);
     const int nmax4 = (nmax + 3) & ~3;
-    // data region: zkey[nmax4] | tot[kBins] | cand_key[cap] | cand_slot[cap]
+    // data region: zkey[nmax4] | tot[kBins] | ... | cand_key[cand_cap] (at the end)
     const size_t fixed = (size_t)nmax4 * 4 + (size_t)kBins * 4;
-    const int cand_cap = fixed + 8ull * 256 <= data_bytes
-                             ? (int)min((size_t)kCandMax, (data_bytes - fixed) / 8) : 0;
+    const int cand_cap = fixed + 4ull * 256 <= data_bytes
+                             ? (int)min((size_t)kCandMax, (data_bytes - fixed) / 4) : 0;
     if (cand_cap == 0) {
       if (r == 0 && tid == 0) dev::set_error(p.err, TRIA_DEVERR_SEGMENT_BIG);
       return;  // every CTA of the cluster takes this branch (same T)
     }
     uint32_t *zkey = reinterpret_cast<uint32_t *>(data);
-    uint32_t *tot = zkey + nmax4;  // [kBins] the cluster histogram, read back
-    uint32_t *cand_key = tot + kBins;
-    int32_t *cand_slot = reinterpret_cast<int32_t *>(cand_key + cand_cap);
+    uint32_t *tot = zkey + nmax4;  // [kBins] this CTA's first-round histogram, later scratch
+    uint32_t *cand_key = reinterpret_cast<uint32_t *>(data + data_bytes) - cand_cap;
+    for (int i = tid; i < kBins; i += nthr) tot[i] = 0u;
+    __syncthreads();
+    // the first round bins z-scores on a fixed grid, arbitrary scores by their top bits
+    const bool fine = zmodes;
 
-    if (p.mode == kModeZmax || p.mode == kModePrune) {
+    if (zmodes) {
       // ---------------------------------------------------- z-score statistics
-      // The score kernel left float64 sums of s and s^2 per (CTA, head) for this
-      // unit; the CTAs that scored it are those whose tile runs meet its live tiles.
-      {
-        const int64_t first_tile = row * p.tiles_per_row + p.tile_prefix[b];
-        const int64_t live_tiles = ((int64_t)T + p.tile_keys - 1) / p.tile_keys;
-        const int64_t c0 = first_tile / p.tiles_per_cta;
-        const int64_t c1 = (first_tile + live_tiles - 1) / p.tiles_per_cta;
-        const int nv = (int)(c1 - c0 + 1) * 2 * G;
-        const double *pu = p.partials + unit * (int64_t)p.max_slots * (2 * G);
-        double *tmp = reinterpret_cast<double *>(data);  // scratch before the keys exist
-        for (int i = tid; i < nv; i += nthr) tmp[i] = pu[i];
-        __syncthreads();
-        if (tid < 2 * G) {
-          double a = 0.0;
-          for (int i = tid; i < nv; i += 2 * G) a += tmp[i];  // fixed order
-          c.sums[tid >> 1][tid & 1] = a;
-        }
-        __syncthreads();
-        if (tid < G) {
-          const double m = c.sums[tid][0] / (double)T;
-          const double var = c.sums[tid][1] / (double)T - m * m;
-          c.mu_hi[tid] = (float)m;
-          c.mu_lo[tid] = (float)(m - (double)c.mu_hi[tid]);
-          c.inv_sigma[tid] = var > 0.0 ? (float)(1.0 / sqrt(var)) : 0.0f;
-        }
-        __syncthreads();
-      }
-      // ---------------------------------------------------- z and group max
+      // float64 sums of s and s^2 over this CTA's keys (fixed order: each thread
+      // its keys in index order, then warps by a fixed shuffle tree, then warps in
+      // order), published for the peers, then the peers' sums added in rank order.
       const float *rawu = p.raw + ((int64_t)l * p.Hq + (int64_t)g * G) * p.cap + seg + lo;
-      float *score = p.score + row * p.cap + seg + lo;
-      float mh[G], ml[G], is[G];
-#pragma unroll
-      for (int j = 0; j < G; ++j) { mh[j] = c.mu_hi[j]; ml[j] = c.mu_lo[j]; is[j] = c.inv_sigma[j]; }
       constexpr int U = G <= 4 ? 4 : (G <= 8 ? 2 : 1);  // keys per thread per round of loads
-      for (int i0 = tid; i0 < n; i0 += U * nthr) {
-        float v[U][G];
+      const bool one_round = n <= U * nthr;            // values stay in registers
+      float v[U][G];
+      auto load = [&](int i0) {
 #pragma unroll
         for (int u = 0; u < U; ++u)
 #pragma unroll
           for (int j = 0; j < G; ++j)
             v[u][j] = i0 + u * nthr < n ? rawu[(int64_t)j * p.cap + i0 + u * nthr] : 0.0f;
+      };
+      double s1[G], s2[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) { s1[j] = 0.0; s2[j] = 0.0; }
+      auto accumulate = [&](int i0) {
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (i0 + u * nthr < n) {
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+              const double x = (double)v[u][j];
+              s1[j] += x;
+              s2[j] = fma(x, x, s2[j]);
+            }
+          }
+      };
+      if (one_round) {
+        load(tid);
+        accumulate(tid);
+      } else {
+        for (int i0 = tid; i0 < n; i0 += U * nthr) {
+          load(i0);
+          accumulate(i0);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          s1[j] += __shfl_xor_sync(0xffffffffu, s1[j], o);
+          s2[j] += __shfl_xor_sync(0xffffffffu, s2[j], o);
+        }
+      }
+      const int warp = tid >> 5;
+      if ((tid & 31) == 0) {
+#pragma unroll
+        for (int j = 0; j < G; ++j) { c.wsum[warp][2 * j] = s1[j]; c.wsum[warp][2 * j + 1] = s2[j]; }
+      }
+      __syncthreads();
+      if (tid < 2 * G) {
+        double a = 0.0;
+        for (int w = 0; w < kWarps; ++w) a += c.wsum[w][tid];
+        c.psum[tid] = a;
+      }
+      cl.sync();  // partial sums published; histogram slices cleared cluster-wide
+      if (tid < 2 * G) {
+        double a = 0.0;
+        for (int q = 0; q < CL; ++q) a += cl.map_shared_rank(&c.psum[0], q)[tid];
+        c.sums[tid >> 1][tid & 1] = a;
+      }
+      __syncthreads();
+      if (tid < G) {
+        const double m = c.sums[tid][0] / (double)T;
+        const double var = c.sums[tid][1] / (double)T - m * m;
+        c.mu_hi[tid] = (float)m;
+        c.mu_lo[tid] = (float)(m - (double)c.mu_hi[tid]);
+        c.inv_sigma[tid] = var > 0.0 ? (float)(1.0 / sqrt(var)) : 0.0f;
+      }
+      __syncthreads();
+      // ---------------------------------------------------- z and group max
+      float *score = p.score + row * p.cap + seg + lo;
+      float mh[G], ml[G], is[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) { mh[j] = c.mu_hi[j]; ml[j] = c.mu_lo[j]; is[j] = c.inv_sigma[j]; }
+      auto zround = [&](int i0) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int i = i0 + u * nthr;
@@ -320,52 +447,112 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
             } else {
               const uint32_t key = dev::order_key(zf);
               zkey[i] = key;
-              cluster_hist_add(cl, &c.slice[0][0], key >> 20, 9);
+              atomicAdd(&tot[fine_bin(key)], 1u);
             }
           }
         }
+      };
+      if (one_round) {
+        zround(tid);
+      } else {
+        for (int i0 = tid; i0 < n; i0 += U * nthr) {
+          load(i0);
+          zround(i0);
+        }
       }
-      if (p.mode == kModeZmax) return;
+      if (p.mode == kModeZmax) {
+        cl.sync();  // no CTA retires while a peer may still read its partial sums
+        return;
+      }
     } else {
       const float *score = p.score + row * p.cap + seg + lo;
       for (int i = tid; i < n; i += nthr) {
         const uint32_t key = dev::order_key(score[i]);
         zkey[i] = key;
-        cluster_hist_add(cl, &c.slice[0][0], key >> 20, 9);
+        atomicAdd(&tot[key >> 20], 1u);
       }
     }
 
     // ------------------------------------------------------------ threshold
-    // Cluster-wide histogram rounds on digits [31:20], [19:8], [7:0] of the keys,
-    // until the bucket of the krem-th largest key is small enough to gather (or
-    // the key is fully known).  Round r counts into slice[r] of the owners.
-    uint32_t prefix = 0, mask = 0;
+    // Round 0: the cluster's counts of the first-round bins, coarse then fine.
+    __syncthreads();  // local histogram complete
+    {
+      const int warp = tid >> 5, lane = tid & 31;
+      if (warp < kCoarse / 2) {  // warp w sums the fine bins of coarse bins 2w, 2w+1
+        const int cb = 2 * warp + (lane >> 4);
+        const int f0 = cb * 64 + (lane & 15) * 4;
+        uint32_t sum = tot[f0] + tot[f0 + 1] + tot[f0 + 2] + tot[f0 + 3];
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if ((lane & 15) == 0) c.coarse[cb] = sum;
+      }
+    }
+    cl.sync();  // every CTA's first-round histogram is complete
+    uint32_t prefix = 0, mask = 0, bin0 = 0;
     int krem = p.budget, bucket = 0;
-    int shift = 20, dbits = 12;
-    for (int round = 0;; ++round) {
+    int top = fine ? 32 : 20;  // bits below `top` are not fixed by prefix/mask
+    {
+      // coarse bin holding the krem-th largest key, then its fine bin
+      if (tid < CL * kCoarse)
+        c.gc[tid / kCoarse][tid % kCoarse] = cl.map_shared_rank(&c.coarse[0], tid / kCoarse)[tid % kCoarse];
+      __syncthreads();
+      if (tid < 32) {
+        int bin, above, cnt;
+        warp_find_bin64(&c.gc[0][0], krem, &bin, &above, &cnt);
+        if (tid == 0) { c.bc[0] = bin; c.bc[1] = above; }
+      }
+      __syncthreads();
+      const int cbin = c.bc[0];
+      krem -= c.bc[1];
+      __syncthreads();
+      if (tid < CL * kCoarse)
+        c.gc[tid / kCoarse][tid % kCoarse] =
+            cl.map_shared_rank(tot, tid / kCoarse)[cbin * 64 + tid % kCoarse];
+      __syncthreads();
+      if (tid < 32) {
+        int bin, above, cnt;
+        warp_find_bin64(&c.gc[0][0], krem, &bin, &above, &cnt);
+        if (tid == 0) { c.bc[0] = cbin * 64 + bin; c.bc[1] = above; c.bc[2] = cnt; }
+      }
+      __syncthreads();
+      const int bin = c.bc[0];
+      krem -= c.bc[1];
+      bucket = c.bc[2];
+      __syncthreads();
+      if (fine) {
+        bin0 = (uint32_t)bin;
+      } else {
+        prefix = (uint32_t)bin << 20;
+        mask = 0xfff00000u;
+      }
+    }
+    auto in_bucket = [&](uint32_t key) -> bool {
+      return (!fine || fine_bin(key) == bin0) && ((key & mask) == prefix);
+    };
+    // Refinement rounds: the next key-bit digit of the bucket's keys, counted into
+    // slice[round] of the owning CTAs, until the bucket is small enough to gather
+    // or the key is fully known.  (`tot` is rewritten only after the first barrier
+    // below, when every peer has finished reading this CTA's histogram.)
+    for (int round = 0; bucket > cand_cap && top > 0; ++round) {
+      const int dshift = top >= 12 ? top - 12 : 0;
+      const int dbits = top - dshift;
       const int nb = 1 << dbits;
       const int per_log2 = dbits - 3;  // bins per owner: nb / 8
+      for (int i = tid; i < n; i += nthr) {
+        const uint32_t key = zkey[i];
+        if (in_bucket(key))
+          cluster_hist_add(cl, &c.slice[round][0], (key >> dshift) & (nb - 1), per_log2);
+      }
       cl.sync();  // every count of this round has landed
       for (int i = tid; i < nb; i += nthr)
         tot[i] = cl.map_shared_rank(&c.slice[round][0], i >> per_log2)[i & ((1 << per_log2) - 1)];
       __syncthreads();
       int bin, above;
       find_bin(tot, nb, krem, c.bc, c.scan, &bin, &above, &bucket);
-      prefix |= (uint32_t)bin << shift;
-      mask |= (uint32_t)(nb - 1) << shift;
       krem -= above;
-      if (bucket <= cand_cap || shift == 0) break;
-      // refine: the next digit of the bucket's keys, into the next round's slices
-      const int nshift = shift >= 12 ? shift - 12 : 0;
-      const int nbits = shift - nshift;
-      for (int i = tid; i < n; i += nthr) {
-        const uint32_t key = zkey[i];
-        if ((key & mask) == prefix)
-          cluster_hist_add(cl, &c.slice[round + 1][0], (key >> nshift) & ((1u << nbits) - 1),
-                           nbits - 3);
-      }
-      shift = nshift;
-      dbits = nbits;
+      prefix |= (uint32_t)bin << dshift;
+      mask |= (uint32_t)(nb - 1) << dshift;
+      top = dshift;
     }
     // Keys above the bucket are kept, keys below dropped; of the bucket's keys the
     // krem largest are kept (ties: lowest slots).  Each thread owns a contiguous
@@ -374,9 +561,12 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     const int a0 = min(n, tid * RL), a1 = min(n, a0 + RL);
     int above_local = 0, in_local = 0;
     for (int i = a0; i < a1; ++i) {
-      const uint32_t mk = zkey[i] & mask;
-      above_local += mk > prefix;
-      in_local += mk == prefix;
+      const uint32_t key = zkey[i];
+      const uint32_t fb = fine ? fine_bin(key) : 0u;
+      const bool same_bin = !fine || fb == bin0;
+      const bool in = same_bin && (key & mask) == prefix;
+      in_local += in;
+      above_local += (fine && fb > bin0) || (same_bin && (key & mask) > prefix);
     }
     const bool gather = bucket <= cand_cap;
     int tot_pk;
@@ -385,11 +575,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       int o = x_pk & 0xffff;
       for (int i = a0; i < a1; ++i) {
         const uint32_t key = zkey[i];
-        if ((key & mask) == prefix) {
-          cand_key[o] = key;
-          cand_slot[o] = (int32_t)(lo + i);
-          ++o;
-        }
+        if (in_bucket(key)) cand_key[o++] = key;
       }
     }
     if (tid == 0) { c.cnt[0] = tot_pk >> 16; c.cnt[1] = tot_pk & 0xffff; }
@@ -414,36 +600,53 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       const int C = c.off[CL];
       uint32_t *gkey = tot;  // [C], C <= cand_cap <= kBins
       for (int i = tid; i < C; i += nthr) {
-        const int q = owner_of(c.off, CL, i);
+        const int q = owner_of(c.off, i);
         gkey[i] = cl.map_shared_rank(cand_key, q)[i - c.off[q]];
       }
       __syncthreads();
-      // the low bits below the bucket prefix, by 10-bit local rounds
-      int rshift = shift, rkrem = krem;
-      uint32_t rprefix = prefix, rmask = mask;
-      while (rshift > 0) {
-        const int nshift = rshift >= 10 ? rshift - 10 : 0;
-        const int nbits = rshift - nshift;
-        for (int i = tid; i < (1 << nbits); i += nthr) c.lh[i] = 0;
-        __syncthreads();
-        for (int i = tid; i < C; i += nthr) {
-          const uint32_t key = gkey[i];
-          if ((key & rmask) == rprefix) atomicAdd(&c.lh[(key >> nshift) & ((1u << nbits) - 1)], 1u);
+      if (C <= kDirectRank) {
+        // pairwise ranks (larger keys first, then lower slots): the key of rank
+        // krem-1 is the threshold
+        if (tid < C) {
+          const uint32_t key = gkey[tid];
+          int rank = 0;
+          for (int j = 0; j < C; ++j) {
+            const uint32_t kj = gkey[j];
+            rank += (kj > key) | ((kj == key) & (j < tid));
+          }
+          if (rank == krem - 1) c.bc[6] = (int32_t)key;
         }
         __syncthreads();
-        int bin, above, cnt;
-        find_bin(c.lh, 1 << nbits, rkrem, c.bc, c.scan, &bin, &above, &cnt);
-        rprefix |= (uint32_t)bin << nshift;
-        rmask |= (uint32_t)((1 << nbits) - 1) << nshift;
-        rkrem -= above;
-        rshift = nshift;
+        thr = (uint32_t)c.bc[6];
+        k_eq = -1;  // from the counts below
+      } else {
+        // the low bits below the bucket's fixed bits, by 10-bit local rounds
+        int rshift = top, rkrem = krem;
+        uint32_t rprefix = prefix, rmask = mask;
+        while (rshift > 0) {
+          const int nshift = rshift >= 10 ? rshift - 10 : 0;
+          const int nbits = rshift - nshift;
+          for (int i = tid; i < (1 << nbits); i += nthr) c.lh[i] = 0;
+          __syncthreads();
+          for (int i = tid; i < C; i += nthr) {
+            const uint32_t key = gkey[i];
+            if ((key & rmask) == rprefix) atomicAdd(&c.lh[(key >> nshift) & ((1u << nbits) - 1)], 1u);
+          }
+          __syncthreads();
+          int bin, above, cnt;
+          find_bin(c.lh, 1 << nbits, rkrem, c.bc, c.scan, &bin, &above, &cnt);
+          rprefix |= (uint32_t)bin << nshift;
+          rmask |= (uint32_t)((1 << nbits) - 1) << nshift;
+          rkrem -= above;
+          rshift = nshift;
+        }
+        thr = rprefix;
+        k_eq = rkrem;
       }
-      thr = rprefix;
-      k_eq = rkrem;
       // per peer: bucket keys above thr and equal to thr
       for (int i = tid; i < C; i += nthr) {
         const uint32_t key = gkey[i];
-        if (key >= thr) atomicAdd(&c.gcnt[owner_of(c.off, CL, i)][key == thr ? 1 : 0], 1);
+        if (key >= thr) atomicAdd(&c.gcnt[owner_of(c.off, i)][key == thr ? 1 : 0], 1);
       }
       __syncthreads();
     } else {
@@ -456,17 +659,29 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     // ------------------------------------------------------------ emit kept slots
     // CTA q keeps its keys above the bucket, its bucket keys above thr, and those
     // of its keys equal to thr whose cluster-wide rank in slot order is < k_eq.
+    // Destination share of each CTA when the unit is compacted in one batch.
+    const int per = (p.budget + CL - 1) / CL;
+    const bool balanced = p.mode == kModePrune &&
+                          per <= (int)min((size_t)kOwnRows, data_bytes / (2 * (size_t)ROW + 4));
     if (tid == 0) {
+      int keq = k_eq;
+      if (keq < 0) {
+        int gt = 0;
+        for (int q = 0; q < CL; ++q) gt += c.gcnt[q][0];
+        keq = krem - gt;
+      }
       int eqb = 0, base = 0;
       for (int q = 0; q < CL; ++q) {
         const int qe = c.gcnt[q][1];
-        const int take = max(0, min(qe, k_eq - eqb));
+        const int take = max(0, min(qe, keq - eqb));
         if (q == r) { c.bc[4] = base; c.bc[5] = eqb; }
         eqb += qe;
         base += c.peer[q][0] + c.gcnt[q][0] + take;
       }
+      c.bc[3] = keq;
     }
     __syncthreads();
+    k_eq = c.bc[3];
     {
       int gt = 0, eq = 0;
       for (int i = a0; i < a1; ++i) {
@@ -484,29 +699,50 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
         bool keep = key > thr;
         if (key == thr) { keep = er < k_eq; ++er; }
         if (keep) {
-          if (o < p.budget) sel[o] = (int32_t)(lo + i);
+          if (o < p.budget) {
+            const int32_t slot = (int32_t)(lo + i);
+            sel[o] = slot;
+            if (balanced) {  // straight into the list of the CTA that compacts destination o
+              const int q = o / per;
+              cl.map_shared_rank(&c.src[0], q)[o - q * per] = slot;
+            }
+          }
           ++o;
         }
       }
     }
-    cl.sync();  // selection list complete and visible; peers' shared memory no longer read
+    cl.sync();  // selection lists complete and visible; peers' keys are no longer read
     if (p.mode == kModeSelect) return;
+    if (balanced) {
+      // ------------------------------------- one batch: this CTA's share of destinations
+      const int j0 = r * per;
+      const int m = max(0, min(per, p.budget - j0));
+      uint8_t *sk = data;
+      uint8_t *sv = data + (size_t)per * ROW;
+      int32_t *sp = reinterpret_cast<int32_t *>(data + 2 * (size_t)per * ROW);
+      stage_rows(c.src, m, kg, vg, pg, sk, sv, sp, ROW, vlog2);
+      __syncthreads();
+      cl.sync();  // every source row of the unit has been read
+      if (tid == 0 && m > 0) {
+        bulk_s2g(kg + (size_t)j0 * ROW, sk, (uint32_t)m * ROW);
+        bulk_s2g(vg + (size_t)j0 * ROW, sv, (uint32_t)m * ROW);
+        bulk_commit();
+      }
+      for (int jj = tid; jj < m; jj += nthr) pg[j0 + jj] = sp[jj];
+      if (tid == 0) bulk_wait_read0();  // shared memory stays valid until the copies read it
+      if (r == 0 && tid == 0 && l == 0 && g == 0) p.seq_len_out[b] = p.budget;
+      return;
+    }
     kept = p.budget;
   }
 
-  // -------------------------------------------------------------- in-place compaction
-  const int ROW = 2 * p.D;   // bytes per K or V row
-  const int VPR = ROW / 16;  // 16-byte vectors per row
+  // -------------------------------------------------------------- batched compaction
   const int cap_rows = (int)(data_bytes / (2 * (size_t)ROW + 8));
   // Batch bt covers the destinations [bt * CL * cap_rows, (bt + 1) * CL * cap_rows) of the
   // whole cluster (CTA r takes the r-th chunk), so every destination written in a batch
   // precedes every destination, and hence every source, of the batches after it.
   const int64_t per_batch = (int64_t)CL * cap_rows;
   const int batches = (int)((kept + per_batch - 1) / per_batch);
-  const int64_t rbase = row * p.cap + seg;
-  uint8_t *kg = p.k + (size_t)rbase * ROW;
-  uint8_t *vg = p.v + (size_t)rbase * ROW;
-  int32_t *pg = p.pos + rbase;
   uint8_t *sk = data;                                                     // [cap_rows][ROW]
   uint8_t *sv = data + (size_t)cap_rows * ROW;                            // [cap_rows][ROW]
   int32_t *sp = reinterpret_cast<int32_t *>(data + 2 * (size_t)cap_rows * ROW);  // [cap_rows]
@@ -524,15 +760,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     }
     if (bad) dev::set_error(p.err, TRIA_DEVERR_SELECTION);
     __syncthreads();
-    for (int it = tid; it < nb * 2 * VPR; it += nthr) {
-      const int jj = it / (2 * VPR), w = it - jj * 2 * VPR;
-      const size_t s = (size_t)ss[jj];
-      if (w < VPR) cp_async16(sk + (size_t)jj * ROW + 16 * w, kg + s * ROW + 16 * w);
-      else cp_async16(sv + (size_t)jj * ROW + 16 * (w - VPR), vg + s * ROW + 16 * (w - VPR));
-    }
-    for (int jj = tid; jj < nb; jj += nthr) cp_async4(sp + jj, pg + ss[jj]);
-    cp_async_wait_all();
-    fence_proxy_async_smem();  // the staged rows are read back by bulk copies
+    stage_rows(ss, nb, kg, vg, pg, sk, sv, sp, ROW, vlog2);
     __syncthreads();
     cl.sync();  // every source row of this batch has been read, cluster-wide
     if (tid == 0 && nb > 0) {
@@ -544,7 +772,6 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     if (tid == 0) bulk_wait_read0();  // the staging buffers may be reused by the next batch
     __syncthreads();
   }
-  if (tid == 0) bulk_wait0();
   if (r == 0 && tid == 0 && l == 0 && g == 0) p.seq_len_out[b] = kept;
 }
 
@@ -557,9 +784,8 @@ static void configure_unit() {
   cudaFuncSetAttribute(unit_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kUnitSmemLarge);
 }
 
-int unit_smem_bytes(int units, int64_t max_segment) {
-  (void)units;
-  (void)max_segment;  // the large size holds the keys of a TRIA_MAX_SEGMENT segment per CTA
+int unit_smem_bytes() {
+  // the large size holds the keys of a TRIA_MAX_SEGMENT segment per CTA
   static bool configured[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && !configured[dev]) {

@@ -11,18 +11,42 @@ namespace tria {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+ScoreGrid score_grid(const tria_config &cfg, const int64_t *seq_start) {
+  ScoreGrid g{};
+  const int G = cfg.n_kv_heads > 0 ? cfg.n_q_heads / cfg.n_kv_heads : 1;
+  g.chunk_keys = score_chunk_keys(cfg.head_dim, G);
+  const int ch = g.chunk_keys > 0 ? g.chunk_keys : 1;
+  int64_t acc = 0, most = 0;
+  for (int b = 0; b < cfg.batch; ++b) {
+    const int64_t n = (seq_start[b + 1] - seq_start[b] + ch - 1) / ch;
+    acc += n;
+    if (n > most) most = n;
+  }
+  g.chunks_per_row = (int)acc;
+  g.total = (int64_t)cfg.num_layers * cfg.n_kv_heads * acc;
+  if (g.total == 0) return g;
+  int64_t grid = device_sm_count();
+  if (grid > g.total) grid = g.total;
+  g.chunks_per_cta = (int)((g.total + grid - 1) / grid);
+  g.grid = (int)((g.total + g.chunks_per_cta - 1) / g.chunks_per_cta);
+  g.max_slots = (int)((most + g.chunks_per_cta - 1) / g.chunks_per_cta + 1);
+  return g;
+}
+
 WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap) {
-  (void)seq_start;
   WsLayout w{};
   const size_t F = (size_t)cfg.head_dim / 2;
   const size_t units = (size_t)cfg.num_layers * cfg.n_kv_heads * cfg.batch;
   const size_t G = cfg.n_kv_heads > 0 ? (size_t)(cfg.n_q_heads / cfg.n_kv_heads) : 1;
+  w.max_slots = score_grid(cfg, seq_start).max_slots;
   size_t o = 0;
   w.err = o;      o += 256;
   w.seqlen = o;   o = align_up(o + 4ull * cfg.batch, 256);
   w.w = o;        o = align_up(o + 4ull * units * (F / 2) * G * 6, 256);
   w.raw = o;      o = align_up(o + 4ull * cfg.num_layers * cfg.n_q_heads * (size_t)cap, 256);
   w.sel = o;      o = align_up(o + 4ull * units * cfg.budget, 256);
+  w.partials = o;
+  o = align_up(o + 16ull * units * (size_t)w.max_slots * kScoreConsumerWarps * G, 256);
   w.total = o;
   return w;
 }
@@ -139,13 +163,16 @@ void fill_fold(FoldParams &fp, const tria_config *cfg, const tria_stats *st,
 
 // Builds the score kernel parameters; *grid receives the grid size (0: nothing to launch).
 cudaError_t fill_score(ScoreParams &sp, const tria_config *cfg, const tria_cache *c,
-                       const float *w, float *raw, int32_t *err, int skip_short, int *grid) {
+                       const float *w, float *raw, double *partials, int32_t *err, int skip_short,
+                       int *grid) {
   std::memset(&sp, 0, sizeof sp);
-  const int G = cfg->n_q_heads / cfg->n_kv_heads;
-  const int ch = score_chunk_keys(cfg->head_dim, G);
+  const ScoreGrid sg = score_grid(*cfg, c->seq_start);
+  const int ch = sg.chunk_keys;
   sp.w = w;
   sp.seq_len = c->seq_len;
   sp.raw = raw;
+  sp.partials = partials;
+  sp.max_slots = sg.max_slots;
   sp.err = err;
   sp.cap = c->cap_total;
   sp.L = cfg->num_layers;
@@ -161,20 +188,25 @@ cudaError_t fill_score(ScoreParams &sp, const tria_config *cfg, const tria_cache
     if (b < cfg->batch) acc += (int32_t)((c->seq_start[b + 1] - c->seq_start[b] + ch - 1) / ch);
   }
   sp.chunks_per_row = acc;
-  const int64_t total = (int64_t)cfg->num_layers * cfg->n_kv_heads * acc;
   *grid = 0;
-  if (total > INT32_MAX - 64) return cudaErrorInvalidValue;  // excluded by check_key_rows
-  sp.total_chunks = (int32_t)total;
-  if (total == 0) return cudaSuccess;
-  int64_t g = device_sm_count();
-  if (g > total) g = total;
-  sp.chunks_per_cta = (int32_t)((total + g - 1) / g);
-  g = (total + sp.chunks_per_cta - 1) / sp.chunks_per_cta;
+  if (sg.total > INT32_MAX - 64) return cudaErrorInvalidValue;  // excluded by check_key_rows
+  sp.total_chunks = (int32_t)sg.total;
+  sp.chunks_per_cta = sg.chunks_per_cta;
+  if (sg.total == 0) return cudaSuccess;
   const int64_t rows = (int64_t)cfg->num_layers * cfg->n_kv_heads * c->cap_total;
   cudaError_t e = make_key_tensor_map(&sp.tmap, c->k, cfg->head_dim, rows, ch);
   if (e != cudaSuccess) return e;
-  *grid = (int)g;
+  *grid = sg.grid;
   return cudaSuccess;
+}
+
+// The unit kernel finds the score kernel's partial sums through its chunk decomposition.
+void link_unit_to_score(UnitParams &up, const ScoreParams &sp) {
+  up.partials = sp.partials;
+  up.max_slots = sp.max_slots;
+  up.chunks_per_cta = sp.chunks_per_cta > 0 ? sp.chunks_per_cta : 1;
+  up.chunks_per_row = sp.chunks_per_row;
+  for (int b = 0; b <= TRIA_MAX_BATCH; ++b) up.chunk_prefix[b] = sp.chunk_prefix[b];
 }
 
 void fill_unit(UnitParams &up, const tria_config *cfg, const tria_cache *c, int mode) {
@@ -201,6 +233,7 @@ struct Ws {
   int32_t *err() const { return reinterpret_cast<int32_t *>(base + lay.err); }
   int32_t *seqlen() const { return reinterpret_cast<int32_t *>(base + lay.seqlen); }
   float *w() const { return reinterpret_cast<float *>(base + lay.w); }
+  double *partials() const { return reinterpret_cast<double *>(base + lay.partials); }
   float *raw() const { return reinterpret_cast<float *>(base + lay.raw); }
   int32_t *sel() const { return reinterpret_cast<int32_t *>(base + lay.sel); }
 };
@@ -263,7 +296,7 @@ tria_status tria_score(const tria_config *cfg, const tria_stats *stats, const tr
   fill_fold(fp, cfg, stats, cache, w.seqlen(), w.w(), w.err());
   ScoreParams sp;
   int grid = 0;
-  if (fill_score(sp, cfg, cache, w.w(), rawp, w.err(), 0, &grid) != cudaSuccess)
+  if (fill_score(sp, cfg, cache, w.w(), rawp, w.partials(), w.err(), 0, &grid) != cudaSuccess)
     return TRIA_ERR_CUDA;
   if (launch_fold(fp, st) != cudaSuccess) return TRIA_ERR_CUDA;
   if (grid > 0 && launch_score(sp, cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads,
@@ -271,6 +304,7 @@ tria_status tria_score(const tria_config *cfg, const tria_stats *stats, const tr
     return TRIA_ERR_CUDA;
   UnitParams up;
   fill_unit(up, cfg, cache, kModeZmax);
+  link_unit_to_score(up, sp);
   up.raw = rawp;
   up.score = score;
   up.seqlen = w.seqlen();
@@ -339,7 +373,7 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
   fill_fold(fp, cfg, stats, cache, w.seqlen(), w.w(), w.err());
   ScoreParams sp;
   int grid = 0;
-  if (fill_score(sp, cfg, cache, w.w(), w.raw(), w.err(), 1, &grid) != cudaSuccess)
+  if (fill_score(sp, cfg, cache, w.w(), w.raw(), w.partials(), w.err(), 1, &grid) != cudaSuccess)
     return TRIA_ERR_CUDA;
   const bool pdl = events == nullptr;  // stage events between kernels would defeat the overlap
   if (!mark()) return TRIA_ERR_CUDA;
@@ -350,6 +384,7 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
     return TRIA_ERR_CUDA;
   UnitParams up;
   fill_unit(up, cfg, cache, kModePrune);
+  link_unit_to_score(up, sp);
   up.raw = w.raw();
   up.sel = sel_out ? sel_out : w.sel();
   up.write_short_sel = sel_out ? 1 : 0;

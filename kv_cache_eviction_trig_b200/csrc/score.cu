@@ -18,8 +18,9 @@
 // whole keys: it reads its rows from the swizzled boxes (conflict-free across
 // the warp), widens bf16 pairs to float, forms |k_f| and accumulates all G
 // heads with the paired FP32 FMA of sm_100 (__ffma2_rn on two RoPE pairs at a
-// time).  The folded weights are the same for every lane, so they are read as
-// broadcast loads that stay in L1.  No cross-lane reduction and no
+// time).  The folded weights of a unit (3 KB at D = 128, G = 4) are brought
+// into one of two shared-memory weight slots by a bulk copy when the producer
+// reaches the unit, and read as broadcasts.  No cross-lane reduction and no
 // synchronisation between consumer warps are needed.
 #include <cudaTypedefs.h>
 
@@ -42,11 +43,13 @@ struct ScoreShape {
   static constexpr int BOXB = CH * 128;                            // bytes per box region
   static constexpr int CB = CH * 2 * D;                            // bytes per chunk
   static constexpr int NW = kScoreConsumerWarps;
-  static constexpr int NSLOT = kScoreRingBytes / CB < 24 ? kScoreRingBytes / CB : 24;
+  static constexpr int WB = FP * G * 24;                           // weight bytes per unit
+  static constexpr int NSLOT0 = (kScoreRingBytes - 2 * WB) / CB;
+  static constexpr int NSLOT = NSLOT0 < 24 ? NSLOT0 : 24;
   static constexpr bool OK = (D == 64 || D == 128 || D == 256) &&
                              (G == 1 || G == 2 || G == 4 || G == 8 || G == 16) && NSLOT > NW;
-  static constexpr size_t SMEM =
-      1024 + (size_t)NSLOT * CB + (size_t)NSLOT * 16 + 2ull * NSLOT * 8 + 4ull * TRIA_MAX_BATCH;
+  static constexpr size_t SMEM = 1024 + (size_t)NSLOT * CB + 2ull * WB + (size_t)NSLOT * 16 +
+                                 2ull * NSLOT * 8 + 2ull * 8 + 4ull * TRIA_MAX_BATCH + 32 * 20;
 };
 
 __device__ __forceinline__ float sqrt_approx(float x) {
@@ -93,6 +96,21 @@ __device__ __forceinline__ void load_pairs(const uint8_t *chunk, int r, int c8, 
   }
 }
 
+// Row, sequence and first key of chunk c (chunks are laid out row by row, and
+// within a row sequence by sequence).
+__device__ __forceinline__ void chunk_coords(const ScoreParams &p, int c, int &row, int &b,
+                                             int &j) {
+  row = c / p.chunks_per_row;
+  const int rem = c - row * p.chunks_per_row;
+  int lo = 0, hi = p.B;  // largest lo with chunk_prefix[lo] <= rem
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.chunk_prefix[mid] <= rem) lo = mid; else hi = mid;
+  }
+  b = lo;
+  j = rem - p.chunk_prefix[lo];  // chunk index within the segment
+}
+
 // acc += wx * x + wy * y + wn * n, two RoPE pairs at a time.
 __device__ __forceinline__ void fma3(float2 &acc, float2 wx, float2 wy, float2 wn, float2 x,
                                      float2 y, float2 n) {
@@ -108,12 +126,17 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   constexpr int F = S::F, FP = S::FP, KPT = S::KPT, CH = S::CH, CB = S::CB, NW = S::NW;
   constexpr int NSLOT = S::NSLOT;
 
+  constexpr int WB = S::WB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *ring = smem_raw + ((1024u - (dev::smem_addr(smem_raw) & 1023u)) & 1023u);
-  int4 *desc = reinterpret_cast<int4 *>(ring + (size_t)NSLOT * CB);  // per slot: row, b, key0, n
+  uint8_t *wring = ring + (size_t)NSLOT * CB;                        // [2][WB] weight slots
+  int4 *desc = reinterpret_cast<int4 *>(wring + 2 * WB);  // per slot: row, b | wslot, key0, n
   uint64_t *full = reinterpret_cast<uint64_t *>(desc + NSLOT);
   uint64_t *empty = full + NSLOT;
-  int32_t *live = reinterpret_cast<int32_t *>(empty + NSLOT);  // [B] keys to score per sequence
+  uint64_t *wfull = empty + NSLOT;                         // [2] weight slot loaded
+  int32_t *live = reinterpret_cast<int32_t *>(wfull + 2);  // [B] keys to score per sequence
+  int4 *tab = reinterpret_cast<int4 *>(live + TRIA_MAX_BATCH);  // [32] chunk descriptors
+  int32_t *taby = reinterpret_cast<int32_t *>(tab + 32);          // [32] their tensor rows
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -121,49 +144,128 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       dev::mbar_init(&full[s], 1);
       dev::mbar_init(&empty[s], 1);
     }
+    dev::mbar_init(&wfull[0], 1);
+    dev::mbar_init(&wfull[1], 1);
     dev::fence_mbar_init();
+  }
+  for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+    int32_t T = p.seq_len[b];
+    if (T < 0 || (int64_t)T > p.seg_start[b + 1] - p.seg_start[b]) T = 0;  // flagged by the fold
+    if (p.skip_short && T <= p.budget) T = 0;
+    live[b] = T;
   }
   __syncthreads();
   if (threadIdx.x == 0) dev::pdl_launch_dependents();
+  const int c0 = blockIdx.x * p.chunks_per_cta;
+  const int c1 = min(c0 + p.chunks_per_cta, p.total_chunks);
+  // The first unit with live chunks: its weights are copied by the consumers
+  // themselves straight from L2 (not queued behind the key stream) into slot 0.
+  int first_unit = -1;
+  for (int c = c0; c < c1; ++c) {
+    int row, b, jc;
+    chunk_coords(p, c, row, b, jc);
+    if (live[b] > jc * CH) { first_unit = row * p.B + b; break; }
+    c += max(0, (p.chunk_prefix[b + 1] - p.chunk_prefix[b]) - jc - 1);  // skip the dead rest
+  }
 
   if (warp == NW) {
     // ---------------------------------------------------------------- producer
-    for (int b = lane; b < p.B; b += 32) {
-      int32_t T = p.seq_len[b];
-      if (T < 0 || (int64_t)T > p.seg_start[b + 1] - p.seg_start[b]) T = 0;  // flagged by the fold
-      if (p.skip_short && T <= p.budget) T = 0;
-      live[b] = T;
-    }
-    __syncwarp();
-    if (lane == 0) {
-      const int c0 = blockIdx.x * p.chunks_per_cta;
-      const int c1 = min(c0 + p.chunks_per_cta, p.total_chunks);
-      uint32_t q = 0;
-      bool failed = false;
-      for (int c = c0; c < c1 && !failed; ++c) {
-        const int row = c / p.chunks_per_row;
-        const int rem = c - row * p.chunks_per_row;
-        int lo = 0, hi = p.B;  // largest b with chunk_prefix[b] <= rem
-        while (hi - lo > 1) {
-          const int mid = (lo + hi) >> 1;
-          if (p.chunk_prefix[mid] <= rem) lo = mid; else hi = mid;
-        }
-        const int key0 = (rem - p.chunk_prefix[lo]) * CH;
-        const int n = min(max(live[lo] - key0, 0), CH);
-        if (n == 0) continue;
-        const uint32_t s = q % NSLOT, use = q / NSLOT;
-        if (use > 0 && !dev::mbar_wait(&empty[s], (use - 1) & 1)) {
-          failed = true;
-          break;
-        }
-        desc[s] = make_int4(row, lo, key0, n);
-        dev::mbar_arrive_expect_tx(&full[s], CB);
-        const int32_t y = (int32_t)((int64_t)row * p.cap + p.seg_start[lo] + key0);
-#pragma unroll
-        for (int bx = 0; bx < S::NBOX; ++bx)
-          dev::tma_load_2d(ring + (size_t)s * CB + bx * S::BOXB, &p.tmap, bx * 64, y, &full[s]);
-        ++q;
+    // lane 0's state: slot positions, weight slots
+    uint32_t q = 0;
+    bool failed = false;
+    int64_t cur_unit = first_unit;  // its weights were put in slot 0 by the consumers
+    int wslot = 0;
+    bool prefilled = first_unit >= 0;  // the current unit's weights came from the consumers
+    uint32_t wuse[2] = {0, 0};    // bulk fills of each weight slot so far (barrier phases)
+    int64_t wlast[2] = {-1, -1};  // last chunk position that read each weight slot
+    // Weight fills wait for the fold kernel; the first ones are held back until the
+    // ring is full, so the first key chunks stream in while the fold runs.
+    bool folded = false;
+    int npend = 0;
+    int pend_slot[2] = {0, 0};
+    int64_t pend_unit[2] = {0, 0};
+    auto flush = [&]() {
+      if (npend == 0) return;
+      if (!folded) {
+        dev::pdl_wait();  // the weights come from the fold kernel
+        folded = true;
       }
+      for (int i = 0; i < npend; ++i) {
+        dev::mbar_arrive_expect_tx(&wfull[pend_slot[i]], WB);
+        dev::bulk_g2s(wring + pend_slot[i] * WB,
+                      reinterpret_cast<const uint8_t *>(p.w) + pend_unit[i] * WB, WB,
+                      &wfull[pend_slot[i]]);
+      }
+      npend = 0;
+    };
+    // The 32 lanes describe 32 chunks at a time in parallel; lane 0 then issues them.
+    for (int cg0 = c0; cg0 < c1; cg0 += 32) {
+      {
+        const int c = cg0 + lane;
+        int row = 0, lo = 0, key0 = 0, n = 0;
+        if (c < c1) {
+          int jc;
+          chunk_coords(p, c, row, lo, jc);
+          key0 = jc * CH;
+          n = min(max(live[lo] - key0, 0), CH);
+        }
+        tab[lane] = make_int4(row, lo, key0, n);
+        taby[lane] = (int32_t)((int64_t)row * p.cap + p.seg_start[lo] + key0);
+      }
+      __syncwarp();
+      if (lane == 0 && !failed) {
+        const int cnt = min(32, c1 - cg0);
+        for (int i = 0; i < cnt; ++i) {
+          const int4 e = tab[i];
+          const int row = e.x, lo = e.y, key0 = e.z, n = e.w;
+          if (n == 0) continue;
+          const uint32_t s = q % NSLOT, use = q / NSLOT;
+          if (use > 0 && !dev::mbar_wait(&empty[s], (use - 1) & 1)) {
+            failed = true;
+            break;
+          }
+          const int64_t unit = (int64_t)row * p.B + lo;
+          if (unit != cur_unit) {
+            // the unit's weights go to the other weight slot, once every chunk that read
+            // that slot's previous weights has been released (all positions up to
+            // q - NSLOT are: the waits above covered them)
+            const int j = wslot ^ 1;
+            if (wlast[j] >= 0) {
+              flush();  // the chunks awaited below need their weights
+              for (int64_t pp = (int64_t)q - NSLOT + 1; pp <= wlast[j] && !failed; ++pp) {
+                // pp > q - NSLOT: position pp's slot was not reused yet, so the parity is its own
+                if (pp >= 0) failed = !dev::mbar_wait(&empty[pp % NSLOT], (uint32_t)(pp / NSLOT) & 1);
+              }
+              if (failed) break;
+            }
+            pend_slot[npend] = j;
+            pend_unit[npend] = unit;
+            ++npend;
+            if (folded) flush();
+            ++wuse[j];
+            wslot = j;
+            cur_unit = unit;
+            prefilled = false;
+          }
+          wlast[wslot] = q;
+          // weight tag: 4 for the consumers' own fill, else slot | phase parity << 1
+          const int wtag = prefilled ? 4 : (wslot | (int)(((wuse[wslot] - 1) & 1) << 1));
+          desc[s] = make_int4(row, lo | (wtag << 16), key0, n);
+          dev::mbar_arrive_expect_tx(&full[s], CB);
+          const int32_t y = taby[i];
+#pragma unroll
+          for (int bx = 0; bx < S::NBOX; ++bx)
+            dev::tma_load_2d(ring + (size_t)s * CB + bx * S::BOXB, &p.tmap, bx * 64, y, &full[s]);
+          ++q;
+          if (q >= (uint32_t)NSLOT) flush();  // the ring is full: wait for the fold now
+        }
+      }
+      failed = __shfl_sync(0xffffffffu, failed, 0);
+      if (failed) break;
+      __syncwarp();  // lane 0 has read the table
+    }
+    if (lane == 0) {
+      if (!failed) flush();
       // one end marker per consumer warp
       for (int t = 0; t < NW && !failed; ++t) {
         const uint32_t s = q % NSLOT, use = q / NSLOT;
@@ -187,7 +289,55 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   }
 
   // ------------------------------------------------------------------ consumers
-  dev::pdl_wait();  // the folded weights come from the fold kernel
+  int wseen = -1;  // weight slot and fill parity last waited for
+  // float64 sums of s and s^2 of this lane's keys for the current unit; each warp
+  // writes one entry per unit its CTA's chunk run meets (zeros where it had none)
+  const int u_first = [&] {
+    int row, b, j;
+    chunk_coords(p, c0, row, b, j);
+    return row * p.B + b;
+  }();
+  const int u_last = [&] {
+    int row, b, j;
+    chunk_coords(p, max(c1 - 1, c0), row, b, j);
+    return row * p.B + b;
+  }();
+  double s1[G], s2[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) { s1[h] = 0.0; s2[h] = 0.0; }
+  auto write_unit = [&](int u, bool zero) {
+    double v[2 * G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      double a = zero ? 0.0 : s1[h], b2 = zero ? 0.0 : s2[h];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        b2 += __shfl_xor_sync(0xffffffffu, b2, o);
+      }
+      v[2 * h] = a;
+      v[2 * h + 1] = b2;
+    }
+    const int row = u / p.B, b = u - row * p.B;
+    if (p.chunk_prefix[b + 1] == p.chunk_prefix[b]) return;  // an empty segment: never read
+    const int slot = (int)blockIdx.x - (row * p.chunks_per_row + p.chunk_prefix[b]) / p.chunks_per_cta;
+    if (slot < 0 || slot >= p.max_slots) return;
+    double *dst = p.partials + (((int64_t)u * p.max_slots + slot) * NW + warp) * (2 * G);
+    if (lane < 2 * G) {
+#pragma unroll
+      for (int i = 0; i < 2 * G; ++i)
+        if (lane == i) dst[i] = v[i];
+    }
+  };
+  if (first_unit >= 0) {
+    dev::pdl_wait();  // the weights come from the fold kernel
+    const uint4 *src = reinterpret_cast<const uint4 *>(reinterpret_cast<const uint8_t *>(p.w) +
+                                                       (int64_t)first_unit * WB);
+    for (int i = threadIdx.x; i < WB / 16; i += NW * 32) reinterpret_cast<uint4 *>(wring)[i] = src[i];
+    dev::named_barrier(1, NW * 32);
+    wseen = 4;  // the tag of these weights
+  }
+  int cur = -1, next_unwritten = u_first;
   for (uint32_t q = warp;; q += NW) {
     const uint32_t s = q % NSLOT, use = q / NSLOT;
     // the slot's previous chunk was released, so the parity below is this use's
@@ -198,9 +348,28 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     }
     const int4 d = desc[s];
     if (d.w < 0) break;
-    const int row = d.x, b = d.y, key0 = d.z, n = d.w;
-    const int64_t unit = (int64_t)row * p.B + b;
-    const float *wu = p.w + (size_t)unit * FP * 6 * G;
+    const int row = d.x, b = d.y & 0xffff, key0 = d.z, n = d.w;
+    const int unit = row * p.B + b;
+    if (unit != cur) {
+      if (cur >= 0) {
+        write_unit(cur, false);
+        next_unwritten = cur + 1;
+      }
+      for (int u = next_unwritten; u < unit; ++u) write_unit(u, true);
+      next_unwritten = unit;
+      cur = unit;
+#pragma unroll
+      for (int h = 0; h < G; ++h) { s1[h] = 0.0; s2[h] = 0.0; }
+    }
+    const int wtag = d.y >> 16;  // weight slot | fill parity << 1, or 4: slot 0 by the consumers
+    if (wtag != wseen) {
+      if (!dev::mbar_wait(&wfull[wtag & 1], (uint32_t)(wtag >> 1))) {
+        if (lane == 0) dev::set_error(p.err, TRIA_DEVERR_TIMEOUT);
+        break;
+      }
+      wseen = wtag;
+    }
+    const float *wu = reinterpret_cast<const float *>(wring + (wtag & 1) * WB);
     const uint8_t *chunk = ring + (size_t)s * CB;
 
     float2 acc[KPT][G];
@@ -254,11 +423,23 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       const int r = lane + 32 * k;
       if (r < n) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) rawp[(size_t)h * p.cap + r] = acc[k][h].x + acc[k][h].y;
+        for (int h = 0; h < G; ++h) {
+          const float v = acc[k][h].x + acc[k][h].y;
+          rawp[(size_t)h * p.cap + r] = v;
+          s1[h] += (double)v;
+          s2[h] = fma((double)v, (double)v, s2[h]);
+        }
       }
     }
     __syncwarp();
     if (lane == 0) dev::mbar_arrive(&empty[s]);
+  }
+  if (c0 < c1) {
+    if (cur >= 0) {
+      write_unit(cur, false);
+      next_unwritten = cur + 1;
+    }
+    for (int u = next_unwritten; u <= u_last; ++u) write_unit(u, true);
   }
 }
 

@@ -17,9 +17,23 @@ struct WsLayout {
   size_t w;         // float [L*Hkv*B][D/4][G][6]  folded weights (fold kernel)
   size_t raw;       // float [L][Hq][cap]  raw scores when the caller gives none
   size_t sel;       // int32 [L][Hkv][B][budget] selection scratch
+  size_t partials;  // double [L*Hkv*B][max_slots][score warps][G][2] sums of s and s^2
+  int32_t max_slots;
   size_t total;
 };
 WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap_total);
+
+// How the score kernel's grid divides the key chunks (a function of the shapes,
+// seq_start and the current device's SM count).
+struct ScoreGrid {
+  int chunk_keys;       // keys per chunk
+  int chunks_per_row;   // chunks of one (layer, KV head) row over all sequences
+  int64_t total;        // chunks over all rows
+  int chunks_per_cta;
+  int grid;
+  int max_slots;        // most CTAs whose chunk runs meet one unit
+};
+ScoreGrid score_grid(const tria_config &cfg, const int64_t *seq_start);
 
 // ------------------------------------------------------------------ kernel parameters
 #ifndef TRIA_SCORE_WARPS
@@ -31,9 +45,12 @@ WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap
 constexpr int kScoreConsumerWarps = TRIA_SCORE_WARPS;  // build-time tunables
 constexpr int kScoreKptCap = TRIA_SCORE_KPT_CAP;
 constexpr int kScoreThreads = (kScoreConsumerWarps + 1) * 32;
-constexpr int kScoreRingBytes = 192 * 1024;  // shared-memory ring of key chunks
+constexpr int kScoreRingBytes = 204 * 1024;  // shared memory for key chunks and weights
 
-constexpr int kUnitThreads = 1024;
+#ifndef TRIA_UNIT_THREADS
+#define TRIA_UNIT_THREADS 1024
+#endif
+constexpr int kUnitThreads = TRIA_UNIT_THREADS;  // build-time tunable: 256, 512 or 1024
 constexpr int kUnitCluster = 8;
 constexpr int kUnitSmemLarge = 200 * 1024;  // one CTA per SM
 
@@ -58,6 +75,8 @@ struct alignas(64) ScoreParams {
   const float *w;           // folded weights (written by the fold kernel)
   const int32_t *seq_len;   // [B] caller's live lengths (not modified during the call)
   float *raw;               // [L][Hq][cap]
+  double *partials;         // per (unit, slot, warp): float64 sums of s and s^2 per head
+  int32_t max_slots;
   int32_t *err;
   int64_t cap;
   int32_t L, Hkv, Hq, B, budget;
@@ -76,6 +95,9 @@ struct UnitParams {
   uint8_t *v;
   int32_t *pos;
   const float *raw;         // [L][Hq][cap]      (zmax, prune)
+  const double *partials;   // the score kernel's per-(unit, slot, warp) sums (zmax, prune)
+  int32_t max_slots, chunks_per_cta, chunks_per_row;
+  int32_t chunk_prefix[TRIA_MAX_BATCH + 1];
   float *score;             // [L][Hkv][cap]     (zmax writes, select reads)
   int32_t *sel;             // [L][Hkv][B][budget]
   const int32_t *seqlen;    // [B] snapshot (zmax, select, prune)

@@ -6,9 +6,9 @@
 //     review, section 3-2 (6)): mu_h and the population sigma_h of the raw
 //     scores over the sequence's T live keys; z_h = (s_h - mu_h) / sigma_h
 //     (0 when sigma_h = 0); score = max_h z_h.  mu and sigma come from float64
-//     sums of s and s^2: each CTA sums its keys in a fixed order, and every CTA
-//     adds the cluster's partial sums in rank order, so all CTAs hold the same,
-//     deterministic statistics.
+//     sums of s and s^2 that the score kernel leaves per (CTA, warp); every CTA
+//     adds them in the same fixed order, so all CTAs hold the same, deterministic
+//     statistics without exchanging anything.
 //   selection (same sources, "prune back to budget"; section 3-2 (5)): the
 //     `budget` largest scores, ties to the lower slot, on order-preserving
 //     32-bit keys.  While the keys are computed each CTA counts them into a
@@ -58,13 +58,11 @@ constexpr int kSlice = kBins / kUnitCluster;  // bins each CTA of the cluster ow
 constexpr int kRounds = 3;                    // refinement rounds (12, 12, 8 key bits)
 constexpr int kCoarse = 64;                   // coarse bins of the first round (64 bins each)
 constexpr int kCandMax = 4096;                // bucket keys a CTA may gather
-constexpr int kDirectRank = 256;              // gathered buckets ranked pairwise
+constexpr int kDirectRank = kUnitThreads < 256 ? kUnitThreads : 256;  // buckets ranked pairwise
 constexpr int kLocalBins = 1024;              // bins of the rounds inside a gathered bucket
 constexpr int kOwnRows = 640;                 // destinations a CTA compacts in one batch
 
 struct Ctl {
-  double wsum[kWarps][2 * kMaxG];   // per-warp partial sums of s and s^2
-  double psum[2 * kMaxG];           // this CTA's partial sums (read by the peers)
   double sums[kMaxG][2];            // the unit's sums of s and s^2 per head
   float mu_hi[kMaxG], mu_lo[kMaxG];  // mean split into two floats (hi + lo)
   float inv_sigma[kMaxG];
@@ -357,11 +355,12 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
 
     if (zmodes) {
       // ---------------------------------------------------- z-score statistics
-      // float64 sums of s and s^2 over this CTA's keys (fixed order: each thread
-      // its keys in index order, then warps by a fixed shuffle tree, then warps in
-      // order), published for the peers, then the peers' sums added in rank order.
+      // The score kernel left, per (CTA slot, warp), float64 sums of s and s^2 of the
+      // unit's keys; every CTA of the cluster adds them in the same fixed order
+      // (strided lanes, then a shuffle tree), so all hold identical statistics.
       const float *rawu = p.raw + ((int64_t)l * p.Hq + (int64_t)g * G) * p.cap + seg + lo;
-      constexpr int U = G <= 4 ? 4 : (G <= 8 ? 2 : 1);  // keys per thread per round of loads
+      // keys per thread per round of loads (U * G raw values in registers)
+      constexpr int U = (16384 / kUnitThreads) / (G > 4 ? G : 4) > 0 ? (16384 / kUnitThreads) / (G > 4 ? G : 4) : 1;
       const bool one_round = n <= U * nthr;            // values stay in registers
       float v[U][G];
       auto load = [&](int i0) {
@@ -371,64 +370,31 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
           for (int j = 0; j < G; ++j)
             v[u][j] = i0 + u * nthr < n ? rawu[(int64_t)j * p.cap + i0 + u * nthr] : 0.0f;
       };
-      double s1[G], s2[G];
+      if (one_round) load(tid);  // in flight while the sums are added
+      {
+        const int64_t first = (int64_t)row * p.chunks_per_row + p.chunk_prefix[b];
+        const int nch = p.chunk_prefix[b + 1] - p.chunk_prefix[b];
+        const int slots = (int)((first + nch - 1) / p.chunks_per_cta - first / p.chunks_per_cta) + 1;
+        const int entries = slots * kScoreConsumerWarps;
+        const double *pu = p.partials + unit * (int64_t)p.max_slots * kScoreConsumerWarps * (2 * G);
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int col = warp; col < 2 * G; col += kWarps) {
+          double a = 0.0;
+          for (int e = lane; e < entries; e += 32) a += pu[(int64_t)e * (2 * G) + col];
 #pragma unroll
-      for (int j = 0; j < G; ++j) { s1[j] = 0.0; s2[j] = 0.0; }
-      auto accumulate = [&](int i0) {
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-          if (i0 + u * nthr < n) {
-#pragma unroll
-            for (int j = 0; j < G; ++j) {
-              const double x = (double)v[u][j];
-              s1[j] += x;
-              s2[j] = fma(x, x, s2[j]);
-            }
-          }
-      };
-      if (one_round) {
-        load(tid);
-        accumulate(tid);
-      } else {
-        for (int i0 = tid; i0 < n; i0 += U * nthr) {
-          load(i0);
-          accumulate(i0);
+          for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+          if (lane == 0) c.sums[col >> 1][col & 1] = a;
         }
-      }
-#pragma unroll
-      for (int j = 0; j < G; ++j) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          s1[j] += __shfl_xor_sync(0xffffffffu, s1[j], o);
-          s2[j] += __shfl_xor_sync(0xffffffffu, s2[j], o);
+        __syncthreads();
+        if (tid < G) {
+          const double m = c.sums[tid][0] / (double)T;
+          const double var = c.sums[tid][1] / (double)T - m * m;
+          c.mu_hi[tid] = (float)m;
+          c.mu_lo[tid] = (float)(m - (double)c.mu_hi[tid]);
+          c.inv_sigma[tid] = var > 0.0 ? (float)(1.0 / sqrt(var)) : 0.0f;
         }
+        __syncthreads();
       }
-      const int warp = tid >> 5;
-      if ((tid & 31) == 0) {
-#pragma unroll
-        for (int j = 0; j < G; ++j) { c.wsum[warp][2 * j] = s1[j]; c.wsum[warp][2 * j + 1] = s2[j]; }
-      }
-      __syncthreads();
-      if (tid < 2 * G) {
-        double a = 0.0;
-        for (int w = 0; w < kWarps; ++w) a += c.wsum[w][tid];
-        c.psum[tid] = a;
-      }
-      cl.sync();  // partial sums published; histogram slices cleared cluster-wide
-      if (tid < 2 * G) {
-        double a = 0.0;
-        for (int q = 0; q < CL; ++q) a += cl.map_shared_rank(&c.psum[0], q)[tid];
-        c.sums[tid >> 1][tid & 1] = a;
-      }
-      __syncthreads();
-      if (tid < G) {
-        const double m = c.sums[tid][0] / (double)T;
-        const double var = c.sums[tid][1] / (double)T - m * m;
-        c.mu_hi[tid] = (float)m;
-        c.mu_lo[tid] = (float)(m - (double)c.mu_hi[tid]);
-        c.inv_sigma[tid] = var > 0.0 ? (float)(1.0 / sqrt(var)) : 0.0f;
-      }
-      __syncthreads();
       // ---------------------------------------------------- z and group max
       float *score = p.score + row * p.cap + seg + lo;
       float mh[G], ml[G], is[G];
@@ -460,10 +426,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
           zround(i0);
         }
       }
-      if (p.mode == kModeZmax) {
-        cl.sync();  // no CTA retires while a peer may still read its partial sums
-        return;
-      }
+      if (p.mode == kModeZmax) return;
     } else {
       const float *score = p.score + row * p.cap + seg + lo;
       for (int i = tid; i < n; i += nthr) {
@@ -478,8 +441,8 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     __syncthreads();  // local histogram complete
     {
       const int warp = tid >> 5, lane = tid & 31;
-      if (warp < kCoarse / 2) {  // warp w sums the fine bins of coarse bins 2w, 2w+1
-        const int cb = 2 * warp + (lane >> 4);
+      for (int w2 = warp; w2 < kCoarse / 2; w2 += kWarps) {  // coarse bins 2*w2, 2*w2+1
+        const int cb = 2 * w2 + (lane >> 4);
         const int f0 = cb * 64 + (lane & 15) * 4;
         uint32_t sum = tot[f0] + tot[f0 + 1] + tot[f0 + 2] + tot[f0 + 3];
 #pragma unroll
@@ -493,8 +456,8 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     int top = fine ? 32 : 20;  // bits below `top` are not fixed by prefix/mask
     {
       // coarse bin holding the krem-th largest key, then its fine bin
-      if (tid < CL * kCoarse)
-        c.gc[tid / kCoarse][tid % kCoarse] = cl.map_shared_rank(&c.coarse[0], tid / kCoarse)[tid % kCoarse];
+      for (int i = tid; i < CL * kCoarse; i += nthr)
+        c.gc[i / kCoarse][i % kCoarse] = cl.map_shared_rank(&c.coarse[0], i / kCoarse)[i % kCoarse];
       __syncthreads();
       if (tid < 32) {
         int bin, above, cnt;
@@ -505,9 +468,8 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       const int cbin = c.bc[0];
       krem -= c.bc[1];
       __syncthreads();
-      if (tid < CL * kCoarse)
-        c.gc[tid / kCoarse][tid % kCoarse] =
-            cl.map_shared_rank(tot, tid / kCoarse)[cbin * 64 + tid % kCoarse];
+      for (int i = tid; i < CL * kCoarse; i += nthr)
+        c.gc[i / kCoarse][i % kCoarse] = cl.map_shared_rank(tot, i / kCoarse)[cbin * 64 + i % kCoarse];
       __syncthreads();
       if (tid < 32) {
         int bin, above, cnt;
@@ -663,22 +625,35 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     const int per = (p.budget + CL - 1) / CL;
     const bool balanced = p.mode == kModePrune &&
                           per <= (int)min((size_t)kOwnRows, data_bytes / (2 * (size_t)ROW + 4));
-    if (tid == 0) {
+    if (tid < 32) {
+      // lane q < CL: peer q's keys equal to thr before it (eqb), the ones it keeps
+      // (take), and the first output index of its kept keys (base)
+      const int q = tid;
+      const int gt = q < CL ? c.gcnt[q][0] : 0, qe = q < CL ? c.gcnt[q][1] : 0;
+      const int ab = q < CL ? c.peer[q][0] : 0;
       int keq = k_eq;
       if (keq < 0) {
-        int gt = 0;
-        for (int q = 0; q < CL; ++q) gt += c.gcnt[q][0];
-        keq = krem - gt;
+        int tgt = gt;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) tgt += __shfl_xor_sync(0xffffffffu, tgt, o);
+        keq = krem - tgt;
       }
-      int eqb = 0, base = 0;
-      for (int q = 0; q < CL; ++q) {
-        const int qe = c.gcnt[q][1];
-        const int take = max(0, min(qe, keq - eqb));
-        if (q == r) { c.bc[4] = base; c.bc[5] = eqb; }
-        eqb += qe;
-        base += c.peer[q][0] + c.gcnt[q][0] + take;
+      int eqi = qe;  // inclusive prefix of equal keys
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, eqi, o);
+        if (q >= o) eqi += t;
       }
-      c.bc[3] = keq;
+      const int eqb = eqi - qe;
+      const int kq = ab + gt + max(0, min(qe, keq - eqb));
+      int ki = kq;  // inclusive prefix of kept keys
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, ki, o);
+        if (q >= o) ki += t;
+      }
+      if (q == r) { c.bc[4] = ki - kq; c.bc[5] = eqb; }
+      if (q == 0) c.bc[3] = keq;
     }
     __syncthreads();
     k_eq = c.bc[3];

@@ -13,7 +13,9 @@ from typing import Optional, Sequence
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libtria.so")
+# TRIA_LIB may name another build of the same library (for example one built with
+# different tuning constants); by default the in-tree build is loaded.
+LIB_PATH = os.environ.get("TRIA_LIB") or os.path.join(_HERE, "libtria.so")
 
 OK = 0
 ERR_INVALID_ARG = 1

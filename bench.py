@@ -123,57 +123,90 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def _cpu_baseline(wl, seconds_target=12.0):
-    """The oracle, as it stands, on the host cores: a bounded sample of the
-    workload (every query head of every KV head of layer 0, sequence 0, on the
-    first n keys; budget scaled by n/T)."""
-    import oracle
-    from tests import common  # the oracle's numpy marshalling helpers
+def rank_workload(index: int, rank: int):
+    """The workload a rank prunes: the same shapes on every rank, its own draw
+    (seed + 1000 * rank) so that ranks never share inputs."""
+    wl = workloads.workload(index)
+    return workloads.workload(index, seed=wl.seed + 1000 * rank) if rank else wl
 
-    T = wl.seq_lens[0]
-    per_key_cos = wl.group * len(wl.offsets) * (wl.head_dim // 2)
-    threads = oracle.num_threads()
-    # about 20 ns per cosine term per thread; aim at ~seconds_target of wall time
-    n = int(seconds_target * threads / (per_key_cos * 20e-9 * wl.n_kv_heads))
-    n = max(64, min(T, n))
-    sub = workloads.custom("cpu-sample", L=1, B=1, Hq=wl.n_q_heads, Hkv=wl.n_kv_heads,
-                           D=wl.head_dim, theta=wl.rope_theta,
-                           budget=max(1, wl.budget * n // T), offsets=wl.offsets,
-                           seq_lens=[n], seed=wl.seed, nu=wl.kv_noise,
-                           position_mode=wl.position_mode, rope_layout=wl.rope_layout,
-                           n_calib=wl.n_calib)
-    sub.position_span = lambda t, _T=T: wl.position_span(_T)
-    data = workloads.generate(sub)
-    stats = common.stats_fp32(data["q_calib"], wl.rope_layout)
-    prob = common.problem(sub, data, stats)
-    v = common.bf16_bits(data["v"])
-    t0 = time.perf_counter()
-    oracle.prune(prob, v)
-    dt = time.perf_counter() - t0
-    keys = n * wl.n_kv_heads
-    return {"value": keys / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"layer 0, all {wl.n_kv_heads} KV heads x {wl.group} query heads, "
-                      f"first {n} of {T} keys, budget {sub.budget}; {dt:.1f} s wall"}
+
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of a list of floats over all ranks (identity with one
+    process); every rank receives the result."""
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+class OracleSample:
+    """The oracle, as it stands, on the host cores, over a bounded sample of the
+    workload: every query head of every KV head of layer 0, sequence 0, on the
+    first n keys (budget scaled by n/T), n sized for about `seconds` of wall time."""
+
+    def __init__(self, wl, seconds):
+        import oracle
+        from tests import common  # the oracle's numpy marshalling helpers
+
+        self.oracle = oracle
+        T = wl.seq_lens[0]
+        per_key_cos = wl.group * len(wl.offsets) * (wl.head_dim // 2)
+        self.threads = oracle.num_threads()
+        # about 20 ns per cosine term per thread
+        n = int(seconds * self.threads / (per_key_cos * 20e-9 * wl.n_kv_heads))
+        n = max(64, min(T, n))
+        sub = workloads.custom("cpu-sample", L=1, B=1, Hq=wl.n_q_heads, Hkv=wl.n_kv_heads,
+                               D=wl.head_dim, theta=wl.rope_theta,
+                               budget=max(1, wl.budget * n // T), offsets=wl.offsets,
+                               seq_lens=[n], seed=wl.seed, nu=wl.kv_noise,
+                               position_mode=wl.position_mode, rope_layout=wl.rope_layout,
+                               n_calib=wl.n_calib)
+        sub.position_span = lambda t, _T=T: wl.position_span(_T)
+        data = workloads.generate(sub)
+        stats = common.stats_fp32(data["q_calib"], wl.rope_layout)
+        self.prob = common.problem(sub, data, stats)
+        self.v = common.bf16_bits(data["v"])
+        self.keys = n * wl.n_kv_heads
+        self.desc = (f"layer 0, all {wl.n_kv_heads} KV heads x {wl.group} query heads, "
+                     f"first {n} of {T} keys, budget {sub.budget}")
+
+    def run(self):
+        """Seconds of one oracle prune of the sample."""
+        t0 = time.perf_counter()
+        self.oracle.prune(self.prob, self.v)
+        return time.perf_counter() - t0
+
+
+def _cpu_baseline(wl, seconds_target=12.0):
+    s = OracleSample(wl, seconds_target)
+    dt = s.run()
+    return {"value": s.keys / dt, "unit": UNIT, "cores": s.threads, "kind": "oracle",
+            "sample": f"{s.desc}; {dt:.1f} s wall"}
 
 
 def run_reference(args):
     rank, world, _ = _rank_env()
     if rank != 0:
-        return
+        return  # the oracle runs once, on rank 0's host
     wl = workloads.workload(args.workload)
-    vals = []
+    # each step is a bounded sample, sized so that the whole run takes a few minutes
+    per_step = max(0.2, min(args.ref_seconds, 150.0 / (args.steps + args.warmup)))
+    sample = OracleSample(wl, per_step)
+    times = []
     for i in range(args.warmup + args.steps):
-        cb = _cpu_baseline(wl, seconds_target=args.ref_seconds)
+        dt = sample.run()
         if i >= args.warmup:
-            vals.append(cb["value"])
-    value = statistics.median(vals)
-    cb["value"] = value
+            times.append(dt)
+    value = sample.keys / statistics.median(times)
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(times) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; the oracle on a bounded sample of the workload)",
         "config": dict(wl.describe(), l2="n/a (host)"),
-        "cpu_baseline": cb,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": sample.threads, "kind": "oracle",
+                         "sample": f"{sample.desc}; median of {args.steps} runs"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
@@ -185,8 +218,7 @@ def run_ours(args):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
-    wl = workloads.workload(args.workload)
-    wl = workloads.workload(args.workload, seed=wl.seed + 1000 * rank) if rank else wl
+    wl = rank_workload(args.workload, rank)
 
     data = workloads.generate(wl, device=dev)
     cfg = tria.Config.from_workload(wl)
@@ -289,11 +321,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in eev)
 
-    if world > 1:
-        t = torch.tensor([total_ms, e2e_ms] + avg_kern, device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
-        avg_kern = [float(x) for x in t[2:]]
+    red = max_over_ranks([total_ms, e2e_ms] + avg_kern, device=dev)
+    total_ms, e2e_ms, avg_kern = red[0], red[1], red[2:]
 
     keys = wl.keys_scored
     value = keys * world / (total_ms / 1e3 / args.steps)

@@ -63,33 +63,50 @@ __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
   return make_float2(dev::bf16lo(w), dev::bf16hi(w));
 }
 
-// 16-byte chunk `c` (0..7) of row `r` of a 128-byte-swizzled box region.
-__device__ __forceinline__ uint4 lds_swizzled(const uint8_t *box, int r, int c) {
-  return *reinterpret_cast<const uint4 *>(box + r * 128 + ((c ^ (r & 7)) << 4));
-}
+// Row r of a chunk lives in the 128-byte-swizzled box regions the TMA wrote:
+// 16-byte unit u of the row's 128 bytes in a box is stored at unit u ^ (r & 7).
 
-// The x and y words of RoPE pairs 8*c8 .. 8*c8+7 of row r: x pairs (f, f+1) in xw[j]
-// for f = 8*c8 + 2j, likewise y.
-template <int D, int CH, int LAYOUT>
-__device__ __forceinline__ void load_pairs(const uint8_t *chunk, int r, int c8, uint32_t (&xw)[4],
-                                           uint32_t (&yw)[4]) {
+// The x and y words of RoPE pairs 2*JU*it .. 2*JU*it + 2*JU-1 of row r: x pairs (f, f+1)
+// in xw[j] for f = 2*JU*it + 2j, likewise y (JU = 4, 2 or 1 words per load).
+template <int D, int CH, int LAYOUT, int JU>
+__device__ __forceinline__ void load_pairs(const uint8_t *chunk, int r, int it, uint32_t (&xw)[JU],
+                                           uint32_t (&yw)[JU]) {
   constexpr int F = D / 2;
   constexpr int BOXB = CH * 128;
   if constexpr (LAYOUT == TRIA_ROPE_HALF_SPLIT) {
-    const int dx = 8 * c8, dy = F + 8 * c8;  // first element of the x and y runs
-    const uint4 a = lds_swizzled(chunk + (dx >> 6) * BOXB, r, (dx & 63) >> 3);
-    const uint4 b = lds_swizzled(chunk + (dy >> 6) * BOXB, r, (dy & 63) >> 3);
-    xw[0] = a.x; xw[1] = a.y; xw[2] = a.z; xw[3] = a.w;
-    yw[0] = b.x; yw[1] = b.y; yw[2] = b.z; yw[3] = b.w;
+    const int dx = 2 * JU * it, dy = F + 2 * JU * it;  // first element of the x and y runs
+    const uint8_t *ax = chunk + (dx >> 6) * BOXB + r * 128 + ((((dx & 63) >> 3) ^ (r & 7)) << 4) + (dx & 7) * 2;
+    const uint8_t *ay = chunk + (dy >> 6) * BOXB + r * 128 + ((((dy & 63) >> 3) ^ (r & 7)) << 4) + (dy & 7) * 2;
+    if constexpr (JU == 4) {
+      const uint4 a = *reinterpret_cast<const uint4 *>(ax), b = *reinterpret_cast<const uint4 *>(ay);
+      xw[0] = a.x; xw[1] = a.y; xw[2] = a.z; xw[3] = a.w;
+      yw[0] = b.x; yw[1] = b.y; yw[2] = b.z; yw[3] = b.w;
+    } else if constexpr (JU == 2) {
+      const uint2 a = *reinterpret_cast<const uint2 *>(ax), b = *reinterpret_cast<const uint2 *>(ay);
+      xw[0] = a.x; xw[1] = a.y;
+      yw[0] = b.x; yw[1] = b.y;
+    } else {
+      xw[0] = *reinterpret_cast<const uint32_t *>(ax);
+      yw[0] = *reinterpret_cast<const uint32_t *>(ay);
+    }
   } else {
     // interleaved: word q holds (x_q, y_q); regroup into x and y pairs
-    const int d0 = 16 * c8;
-    const uint8_t *box = chunk + (d0 >> 6) * BOXB;
-    const uint4 a = lds_swizzled(box, r, (d0 & 63) >> 3);
-    const uint4 b = lds_swizzled(box, r, ((d0 & 63) >> 3) + 1);
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const int d0 = 4 * JU * it;
+    const uint8_t *a0 = chunk + (d0 >> 6) * BOXB + r * 128 + ((((d0 & 63) >> 3) ^ (r & 7)) << 4) + (d0 & 7) * 2;
+    uint32_t w[2 * JU];
+    if constexpr (JU == 4) {
+      const uint8_t *a1 = chunk + (d0 >> 6) * BOXB + r * 128 + (((((d0 & 63) >> 3) + 1) ^ (r & 7)) << 4);
+      const uint4 a = *reinterpret_cast<const uint4 *>(a0), b = *reinterpret_cast<const uint4 *>(a1);
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    } else if constexpr (JU == 2) {
+      const uint4 a = *reinterpret_cast<const uint4 *>(a0);
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    } else {
+      const uint2 a = *reinterpret_cast<const uint2 *>(a0);
+      w[0] = a.x; w[1] = a.y;
+    }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < JU; ++i) {
       xw[i] = __byte_perm(w[2 * i], w[2 * i + 1], 0x5410);  // (x_2i, x_2i+1)
       yw[i] = __byte_perm(w[2 * i], w[2 * i + 1], 0x7632);  // (y_2i, y_2i+1)
     }
@@ -148,28 +165,37 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     dev::mbar_init(&wfull[1], 1);
     dev::fence_mbar_init();
   }
-  for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
-    int32_t T = p.seq_len[b];
-    if (T < 0 || (int64_t)T > p.seg_start[b + 1] - p.seg_start[b]) T = 0;  // flagged by the fold
-    if (p.skip_short && T <= p.budget) T = 0;
-    live[b] = T;
-  }
   __syncthreads();
   if (threadIdx.x == 0) dev::pdl_launch_dependents();
   const int c0 = blockIdx.x * p.chunks_per_cta;
   const int c1 = min(c0 + p.chunks_per_cta, p.total_chunks);
   // The first unit with live chunks: its weights are copied by the consumers
   // themselves straight from L2 (not queued behind the key stream) into slot 0.
-  int first_unit = -1;
-  for (int c = c0; c < c1; ++c) {
-    int row, b, jc;
-    chunk_coords(p, c, row, b, jc);
-    if (live[b] > jc * CH) { first_unit = row * p.B + b; break; }
-    c += max(0, (p.chunk_prefix[b + 1] - p.chunk_prefix[b]) - jc - 1);  // skip the dead rest
-  }
+  auto find_first_unit = [&]() {
+    for (int c = c0; c < c1; ++c) {
+      int row, b, jc;
+      chunk_coords(p, c, row, b, jc);
+      if (live[b] > jc * CH) return row * p.B + b;
+      c += max(0, (p.chunk_prefix[b + 1] - p.chunk_prefix[b]) - jc - 1);  // skip the dead rest
+    }
+    return -1;
+  };
+  // Named barriers: 1 the consumers among themselves; 2 the consumers' warm-up is
+  // done (the producer may start the key stream); 3 the producer's live lengths are
+  // written (the consumers may read them).
 
   if (warp == NW) {
     // ---------------------------------------------------------------- producer
+    for (int b = lane; b < p.B; b += 32) {
+      int32_t T = p.seq_len[b];
+      if (T < 0 || (int64_t)T > p.seg_start[b + 1] - p.seg_start[b]) T = 0;  // flagged by the fold
+      if (p.skip_short && T <= p.budget) T = 0;
+      live[b] = T;
+    }
+    __syncwarp();
+    __threadfence_block();
+    dev::named_barrier_arrive(3, (NW + 1) * 32);
+    const int first_unit = find_first_unit();
     // lane 0's state: slot positions, weight slots
     uint32_t q = 0;
     bool failed = false;
@@ -198,6 +224,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       }
       npend = 0;
     };
+    // The consumers first run their chunk code once (see below); the key stream
+    // starts after that, so their instruction fetches do not queue behind it.
+    dev::named_barrier(2, (NW + 1) * 32);
     // The 32 lanes describe 32 chunks at a time in parallel; lane 0 then issues them.
     for (int cg0 = c0; cg0 < c1; cg0 += 32) {
       {
@@ -292,16 +321,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   int wseen = -1;  // weight slot and fill parity last waited for
   // float64 sums of s and s^2 of this lane's keys for the current unit; each warp
   // writes one entry per unit its CTA's chunk run meets (zeros where it had none)
-  const int u_first = [&] {
-    int row, b, j;
-    chunk_coords(p, c0, row, b, j);
-    return row * p.B + b;
-  }();
-  const int u_last = [&] {
-    int row, b, j;
-    chunk_coords(p, max(c1 - 1, c0), row, b, j);
-    return row * p.B + b;
-  }();
+  int u_first = 0, u_last = -1, first_unit = -1;  // set after the warm-up
   double s1[G], s2[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) { s1[h] = 0.0; s2[h] = 0.0; }
@@ -329,45 +349,50 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         if (lane == i) dst[i] = v[i];
     }
   };
-  if (first_unit >= 0) {
-    dev::pdl_wait();  // the weights come from the fold kernel
-    const uint4 *src = reinterpret_cast<const uint4 *>(reinterpret_cast<const uint8_t *>(p.w) +
-                                                       (int64_t)first_unit * WB);
-    for (int i = threadIdx.x; i < WB / 16; i += NW * 32) reinterpret_cast<uint4 *>(wring)[i] = src[i];
-    dev::named_barrier(1, NW * 32);
-    wseen = 4;  // the tag of these weights
-  }
-  int cur = -1, next_unwritten = u_first;
-  for (uint32_t q = warp;; q += NW) {
-    const uint32_t s = q % NSLOT, use = q / NSLOT;
-    // the slot's previous chunk was released, so the parity below is this use's
-    if ((use > 0 && !dev::mbar_wait(&empty[s], (use - 1) & 1)) ||
-        !dev::mbar_wait(&full[s], use & 1)) {
-      if (lane == 0) dev::set_error(p.err, TRIA_DEVERR_TIMEOUT);
-      break;
-    }
-    const int4 d = desc[s];
-    if (d.w < 0) break;
-    const int row = d.x, b = d.y & 0xffff, key0 = d.z, n = d.w;
-    const int unit = row * p.B + b;
-    if (unit != cur) {
-      if (cur >= 0) {
-        write_unit(cur, false);
-        next_unwritten = cur + 1;
-      }
-      for (int u = next_unwritten; u < unit; ++u) write_unit(u, true);
-      next_unwritten = unit;
-      cur = unit;
-#pragma unroll
-      for (int h = 0; h < G; ++h) { s1[h] = 0.0; s2[h] = 0.0; }
-    }
-    const int wtag = d.y >> 16;  // weight slot | fill parity << 1, or 4: slot 0 by the consumers
-    if (wtag != wseen) {
-      if (!dev::mbar_wait(&wfull[wtag & 1], (uint32_t)(wtag >> 1))) {
+  int cur = -1, next_unwritten = 0;
+  // The first pass is a warm-up: one inner iteration and the epilogue of the chunk
+  // code on whatever the ring holds, storing nothing (n = 0), so that the code is
+  // fetched before the key stream saturates the memory system.
+  bool warm = true;
+#pragma unroll 1
+  for (uint32_t q = warp;;) {
+    uint32_t s = 0;
+    int row = 0, b = 0, key0 = 0, n = 0, wtag = 0;
+    if (!warm) {
+      s = q % NSLOT;
+      const uint32_t use = q / NSLOT;
+      // the slot's previous chunk was released, so the parity below is this use's
+      if ((use > 0 && !dev::mbar_wait(&empty[s], (use - 1) & 1)) ||
+          !dev::mbar_wait(&full[s], use & 1)) {
         if (lane == 0) dev::set_error(p.err, TRIA_DEVERR_TIMEOUT);
         break;
       }
-      wseen = wtag;
+      const int4 d = desc[s];
+      if (d.w < 0) break;
+      row = d.x;
+      b = d.y & 0xffff;
+      key0 = d.z;
+      n = d.w;
+      const int unit = row * p.B + b;
+      if (unit != cur) {
+        if (cur >= 0) {
+          write_unit(cur, false);
+          next_unwritten = cur + 1;
+        }
+        for (int u = next_unwritten; u < unit; ++u) write_unit(u, true);
+        next_unwritten = unit;
+        cur = unit;
+#pragma unroll
+        for (int h = 0; h < G; ++h) { s1[h] = 0.0; s2[h] = 0.0; }
+      }
+      wtag = d.y >> 16;  // weight slot | fill parity << 1, or 4: slot 0 by the consumers
+      if (wtag != wseen) {
+        if (!dev::mbar_wait(&wfull[wtag & 1], (uint32_t)(wtag >> 1))) {
+          if (lane == 0) dev::set_error(p.err, TRIA_DEVERR_TIMEOUT);
+          break;
+        }
+        wseen = wtag;
+      }
     }
     const float *wu = reinterpret_cast<const float *>(wring + (wtag & 1) * WB);
     const uint8_t *chunk = ring + (size_t)s * CB;
@@ -378,14 +403,16 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 #pragma unroll
       for (int h = 0; h < G; ++h) acc[k][h] = make_float2(0.0f, 0.0f);
 
+    constexpr int JU = kScoreJu;
+    const int iters = warm ? 1 : FP / JU;
 #pragma unroll 1
-    for (int c8 = 0; c8 < F / 8; ++c8) {
-      uint32_t xw[KPT][4], yw[KPT][4];
+    for (int it = 0; it < iters; ++it) {
+      uint32_t xw[KPT][JU], yw[KPT][JU];
 #pragma unroll
-      for (int k = 0; k < KPT; ++k) load_pairs<D, CH, LAYOUT>(chunk, lane + 32 * k, c8, xw[k], yw[k]);
+      for (int k = 0; k < KPT; ++k) load_pairs<D, CH, LAYOUT, JU>(chunk, lane + 32 * k, it, xw[k], yw[k]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float *wf = wu + (size_t)(4 * c8 + j) * 6 * G;
+      for (int j = 0; j < JU; ++j) {
+        const float *wf = wu + (size_t)(JU * it + j) * 6 * G;
         float2 X[KPT], Y[KPT], N[KPT];
 #pragma unroll
         for (int k = 0; k < KPT; ++k) {
@@ -431,8 +458,33 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
       }
     }
+    if (warm) {
+      warm = false;
+      dev::named_barrier_arrive(2, (NW + 1) * 32);  // the producer may start the stream
+      {
+        int row, b, j;
+        chunk_coords(p, c0, row, b, j);
+        u_first = row * p.B + b;
+        chunk_coords(p, max(c1 - 1, c0), row, b, j);
+        u_last = row * p.B + b;
+        next_unwritten = u_first;
+      }
+      dev::named_barrier(3, (NW + 1) * 32);  // the live lengths are written
+      first_unit = find_first_unit();
+      if (first_unit >= 0) {
+        dev::pdl_wait();  // the weights come from the fold kernel
+        const uint4 *src = reinterpret_cast<const uint4 *>(reinterpret_cast<const uint8_t *>(p.w) +
+                                                           (int64_t)first_unit * WB);
+        for (int i = threadIdx.x; i < WB / 16; i += NW * 32)
+          reinterpret_cast<uint4 *>(wring)[i] = src[i];
+        dev::named_barrier(1, NW * 32);
+        wseen = 4;  // the tag of these weights
+      }
+      continue;
+    }
     __syncwarp();
     if (lane == 0) dev::mbar_arrive(&empty[s]);
+    q += NW;
   }
   if (c0 < c1) {
     if (cur >= 0) {

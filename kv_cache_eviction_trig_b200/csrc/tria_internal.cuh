@@ -44,8 +44,12 @@ ScoreGrid score_grid(const tria_config &cfg, const int64_t *seq_start);
 #endif
 constexpr int kScoreConsumerWarps = TRIA_SCORE_WARPS;  // build-time tunables
 constexpr int kScoreKptCap = TRIA_SCORE_KPT_CAP;
+#ifndef TRIA_SCORE_JU
+#define TRIA_SCORE_JU 4
+#endif
+constexpr int kScoreJu = TRIA_SCORE_JU;  // pairs of RoPE pairs per inner iteration: 1, 2 or 4
 constexpr int kScoreThreads = (kScoreConsumerWarps + 1) * 32;
-constexpr int kScoreRingBytes = 204 * 1024;  // shared memory for key chunks and weights
+constexpr int kScoreRingBytes = 220 * 1024;  // shared memory for key chunks and weights
 
 #ifndef TRIA_UNIT_THREADS
 #define TRIA_UNIT_THREADS 1024
@@ -205,6 +209,11 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *map, int32_t 
 
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Arrives at a named barrier without waiting for it.
+__device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t threads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // bf16 pair in one 32-bit word -> two floats (exact widening).

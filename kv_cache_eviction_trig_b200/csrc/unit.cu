@@ -61,6 +61,7 @@ constexpr int kCandMax = 4096;                // bucket keys a CTA may gather
 constexpr int kDirectRank = kUnitThreads < 256 ? kUnitThreads : 256;  // buckets ranked pairwise
 constexpr int kLocalBins = 1024;              // bins of the rounds inside a gathered bucket
 constexpr int kOwnRows = 640;                 // destinations a CTA compacts in one batch
+constexpr int kKeptMax = 3072;                // kept keys of one CTA listed for the compactors
 
 struct Ctl {
   double sums[kMaxG][2];            // the unit's sums of s and s^2 per head
@@ -73,6 +74,9 @@ struct Ctl {
   int32_t gcnt[kMaxCluster][2];     // per peer: bucket keys above the threshold, equal to it
   int32_t scan[kWarps + 1];
   int32_t src[kOwnRows];            // source slots of this CTA's share of the destinations
+  int32_t base[kMaxCluster];        // per peer: first output index of its kept keys
+  int32_t keptq[kMaxCluster];       // per peer: its kept keys
+  int32_t kept_src[kKeptMax];       // slots of this CTA's kept keys, in output order
   uint32_t coarse[kCoarse];         // this CTA's first-round counts per coarse bin
   uint32_t gc[kUnitCluster][kCoarse];  // the cluster's coarse counts, then fine counts
   uint32_t lh[kLocalBins];          // histogram of the rounds inside a gathered bucket
@@ -318,7 +322,26 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       return;
     }
   } else {
-    const int32_t T = p.seqlen[b];
+    const int32_t T = p.seqlen[b];  // issued first: the loads below do not need it
+    if (zmodes) {
+      // The score kernel left, per (CTA slot, warp), float64 sums of s and s^2 of the
+      // unit's keys; every CTA of the cluster adds them in the same fixed order
+      // (strided lanes, then a shuffle tree), so all hold identical statistics.  They
+      // do not depend on the live length, so their loads overlap its load.
+      const int64_t first = (int64_t)row * p.chunks_per_row + p.chunk_prefix[b];
+      const int nch = p.chunk_prefix[b + 1] - p.chunk_prefix[b];
+      const int slots = nch > 0 ? (int)((first + nch - 1) / p.chunks_per_cta - first / p.chunks_per_cta) + 1 : 0;
+      const int entries = slots * kScoreConsumerWarps;
+      const double *pu = p.partials + unit * (int64_t)p.max_slots * kScoreConsumerWarps * (2 * G);
+      const int warp = tid >> 5, lane = tid & 31;
+      for (int col = warp; col < 2 * G; col += kWarps) {
+        double a = 0.0;
+        for (int e = lane; e < entries; e += 32) a += pu[(int64_t)e * (2 * G) + col];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) c.sums[col >> 1][col & 1] = a;
+      }
+    }
     if (T < 0 || (int64_t)T > seg_cap) {
       if (r == 0 && tid == 0) dev::set_error(p.err, TRIA_DEVERR_SEQ_LEN);
       return;  // same decision in every CTA of the cluster
@@ -337,18 +360,22 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     const int n = (int)(hi - lo);
     const int nmax = (int)((T + CL - 1) / CL);
     const int nmax4 = (nmax + 3) & ~3;
-    // data region: zkey[nmax4] | tot[kBins] | ... | cand_key[cand_cap] (at the end)
-    const size_t fixed = (size_t)nmax4 * 4 + (size_t)kBins * 4;
-    const int cand_cap = fixed + 4ull * 256 <= data_bytes
-                             ? (int)min((size_t)kCandMax, (data_bytes - fixed) / 4) : 0;
+    // data region: zkey[nmax4] | tot[kBins] | gslot[kCandMax] | ... |
+    //              cand_key[cand_cap] cand_slot[cand_cap] (at the end)
+    const size_t fixed = (size_t)nmax4 * 4 + (size_t)kBins * 4 + (size_t)kCandMax * 4;
+    const int cand_cap = fixed + 8ull * 256 <= data_bytes
+                             ? (int)min((size_t)kCandMax, (data_bytes - fixed) / 8) : 0;
     if (cand_cap == 0) {
       if (r == 0 && tid == 0) dev::set_error(p.err, TRIA_DEVERR_SEGMENT_BIG);
       return;  // every CTA of the cluster takes this branch (same T)
     }
     uint32_t *zkey = reinterpret_cast<uint32_t *>(data);
     uint32_t *tot = zkey + nmax4;  // [kBins] this CTA's first-round histogram, later scratch
-    uint32_t *cand_key = reinterpret_cast<uint32_t *>(data + data_bytes) - cand_cap;
+    int32_t *gslot = reinterpret_cast<int32_t *>(tot + kBins);  // [kCandMax] gathered slots
+    uint32_t *cand_key = reinterpret_cast<uint32_t *>(data + data_bytes) - 2 * cand_cap;
+    int32_t *cand_slot = reinterpret_cast<int32_t *>(cand_key + cand_cap);
     for (int i = tid; i < kBins; i += nthr) tot[i] = 0u;
+    if (tid < 2) c.cnt[tid] = 0;
     __syncthreads();
     // the first round bins z-scores on a fixed grid, arbitrary scores by their top bits
     const bool fine = zmodes;
@@ -370,22 +397,9 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
           for (int j = 0; j < G; ++j)
             v[u][j] = i0 + u * nthr < n ? rawu[(int64_t)j * p.cap + i0 + u * nthr] : 0.0f;
       };
-      if (one_round) load(tid);  // in flight while the sums are added
+      if (one_round) load(tid);  // in flight while mu and sigma are formed
       {
-        const int64_t first = (int64_t)row * p.chunks_per_row + p.chunk_prefix[b];
-        const int nch = p.chunk_prefix[b + 1] - p.chunk_prefix[b];
-        const int slots = (int)((first + nch - 1) / p.chunks_per_cta - first / p.chunks_per_cta) + 1;
-        const int entries = slots * kScoreConsumerWarps;
-        const double *pu = p.partials + unit * (int64_t)p.max_slots * kScoreConsumerWarps * (2 * G);
-        const int warp = tid >> 5, lane = tid & 31;
-        for (int col = warp; col < 2 * G; col += kWarps) {
-          double a = 0.0;
-          for (int e = lane; e < entries; e += 32) a += pu[(int64_t)e * (2 * G) + col];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-          if (lane == 0) c.sums[col >> 1][col & 1] = a;
-        }
-        __syncthreads();
+        // c.sums were written before the live length was read (a barrier since)
         if (tid < G) {
           const double m = c.sums[tid][0] / (double)T;
           const double var = c.sums[tid][1] / (double)T - m * m;
@@ -517,30 +531,33 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       top = dshift;
     }
     // Keys above the bucket are kept, keys below dropped; of the bucket's keys the
-    // krem largest are kept (ties: lowest slots).  Each thread owns a contiguous
-    // run of this CTA's keys, so runs in thread order are in slot order.
+    // krem largest are kept (ties: lowest slots).  Each CTA counts its keys above the
+    // bucket and lists its bucket keys with their slots (in any order).
+    const bool gather = bucket <= cand_cap;
+    {
+      int above_local = 0;
+      for (int i = tid; i < n; i += nthr) {
+        const uint32_t key = zkey[i];
+        const uint32_t fb = fine ? fine_bin(key) : 0u;
+        const bool same_bin = !fine || fb == bin0;
+        if (same_bin && (key & mask) == prefix) {
+          const int pos = atomicAdd(&c.cnt[1], 1);
+          if (gather && pos < cand_cap) {
+            cand_key[pos] = key;
+            cand_slot[pos] = (int32_t)(lo + i);
+          }
+        } else {
+          above_local += (fine && fb > bin0) || (same_bin && (key & mask) > prefix);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) above_local += __shfl_xor_sync(0xffffffffu, above_local, o);
+      if ((tid & 31) == 0 && above_local) atomicAdd(&c.cnt[0], above_local);
+    }
+    // Each thread also owns a contiguous run of this CTA's keys, so runs in thread
+    // order are in slot order (used when the kept keys are emitted).
     const int RL = (n + nthr - 1) / nthr;
     const int a0 = min(n, tid * RL), a1 = min(n, a0 + RL);
-    int above_local = 0, in_local = 0;
-    for (int i = a0; i < a1; ++i) {
-      const uint32_t key = zkey[i];
-      const uint32_t fb = fine ? fine_bin(key) : 0u;
-      const bool same_bin = !fine || fb == bin0;
-      const bool in = same_bin && (key & mask) == prefix;
-      in_local += in;
-      above_local += (fine && fb > bin0) || (same_bin && (key & mask) > prefix);
-    }
-    const bool gather = bucket <= cand_cap;
-    int tot_pk;
-    const int x_pk = block_excl_scan((above_local << 16) | in_local, c.scan, &tot_pk);  // n < 65536
-    if (gather) {
-      int o = x_pk & 0xffff;
-      for (int i = a0; i < a1; ++i) {
-        const uint32_t key = zkey[i];
-        if (in_bucket(key)) cand_key[o++] = key;
-      }
-    }
-    if (tid == 0) { c.cnt[0] = tot_pk >> 16; c.cnt[1] = tot_pk & 0xffff; }
     cl.sync();  // counts and bucket lists complete
     if (tid < CL) {
       const Ctl *peer = cl.map_shared_rank(&c, tid);
@@ -564,6 +581,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       for (int i = tid; i < C; i += nthr) {
         const int q = owner_of(c.off, i);
         gkey[i] = cl.map_shared_rank(cand_key, q)[i - c.off[q]];
+        gslot[i] = cl.map_shared_rank(cand_slot, q)[i - c.off[q]];
       }
       __syncthreads();
       if (C <= kDirectRank) {
@@ -571,10 +589,11 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
         // krem-1 is the threshold
         if (tid < C) {
           const uint32_t key = gkey[tid];
+          const int32_t slot = gslot[tid];
           int rank = 0;
           for (int j = 0; j < C; ++j) {
             const uint32_t kj = gkey[j];
-            rank += (kj > key) | ((kj == key) & (j < tid));
+            rank += (kj > key) | ((kj == key) & (gslot[j] < slot));
           }
           if (rank == krem - 1) c.bc[6] = (int32_t)key;
         }
@@ -623,8 +642,8 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     // of its keys equal to thr whose cluster-wide rank in slot order is < k_eq.
     // Destination share of each CTA when the unit is compacted in one batch.
     const int per = (p.budget + CL - 1) / CL;
-    const bool balanced = p.mode == kModePrune &&
-                          per <= (int)min((size_t)kOwnRows, data_bytes / (2 * (size_t)ROW + 4));
+    const bool balanced_fit = p.mode == kModePrune &&
+                              per <= (int)min((size_t)kOwnRows, data_bytes / (2 * (size_t)ROW + 4));
     if (tid < 32) {
       // lane q < CL: peer q's keys equal to thr before it (eqb), the ones it keeps
       // (take), and the first output index of its kept keys (base)
@@ -653,10 +672,13 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
         if (q >= o) ki += t;
       }
       if (q == r) { c.bc[4] = ki - kq; c.bc[5] = eqb; }
-      if (q == 0) c.bc[3] = keq;
+      if (q < CL) { c.base[q] = ki - kq; c.keptq[q] = kq; }
+      const int most = __reduce_max_sync(0xffffffffu, q < CL ? kq : 0);
+      if (q == 0) { c.bc[3] = keq; c.bc[7] = most; }
     }
     __syncthreads();
     k_eq = c.bc[3];
+    const bool balanced = balanced_fit && c.bc[7] <= kKeptMax;
     {
       int gt = 0, eq = 0;
       for (int i = a0; i < a1; ++i) {
@@ -677,10 +699,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
           if (o < p.budget) {
             const int32_t slot = (int32_t)(lo + i);
             sel[o] = slot;
-            if (balanced) {  // straight into the list of the CTA that compacts destination o
-              const int q = o / per;
-              cl.map_shared_rank(&c.src[0], q)[o - q * per] = slot;
-            }
+            if (balanced) c.kept_src[o - c.bc[4]] = slot;  // read by the compacting CTAs
           }
           ++o;
         }
@@ -692,6 +711,14 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       // ------------------------------------- one batch: this CTA's share of destinations
       const int j0 = r * per;
       const int m = max(0, min(per, p.budget - j0));
+      for (int jj = tid; jj < m; jj += nthr) {
+        const int j = j0 + jj;
+        int q = 0;  // the peer whose kept keys include output index j
+#pragma unroll
+        for (int k = 1; k < kUnitCluster; ++k) q += c.base[k] <= j;
+        c.src[jj] = cl.map_shared_rank(&c.kept_src[0], q)[j - c.base[q]];
+      }
+      __syncthreads();
       uint8_t *sk = data;
       uint8_t *sv = data + (size_t)per * ROW;
       int32_t *sp = reinterpret_cast<int32_t *>(data + 2 * (size_t)per * ROW);

@@ -159,6 +159,8 @@ void fill_fold(FoldParams &fp, const tria_config *cfg, const tria_stats *st,
   fp.flags = cfg->flags;
   for (int b = 0; b < cfg->batch; ++b) fp.seg_cap[b] = c->seq_start[b + 1] - c->seq_start[b];
   std::memcpy(fp.offsets, cfg->offsets, sizeof(int32_t) * cfg->n_offsets);
+  for (int f = 0; f < cfg->head_dim / 2 && f < 128; ++f)
+    fp.omega[f] = std::pow(cfg->rope_theta, -2.0 * (double)f / (double)cfg->head_dim);
 }
 
 // Builds the score kernel parameters; *grid receives the grid size (0: nothing to launch).

@@ -10,8 +10,9 @@
 // so the per-key work needs no position and no trigonometry.  The norm term's
 // weight is Nw_f = (1 - R_f) E|q_f| (section 3-2 (3)-(4)).
 //
-// Block (fp, y) handles the RoPE pairs f = 2fp, 2fp+1: it forms EA in float64
-// (angles reach ~1e5 rad) for every sequence, then writes, for a share y of
+// Block (fp, y) handles the RoPE pairs f = 2fp, 2fp+1 (w_f comes from the host,
+// in double precision): it forms EA in float64 (angles reach ~1e5 rad) for every
+// sequence, then writes, for a share y of
 // the (unit, head) pairs, the float32 weights
 //   w[unit][fp][h] = (Re W_2fp, Re W_2fp+1, Im W_2fp, Im W_2fp+1, Nw_2fp, Nw_2fp+1).
 // Block (0, 0) also snapshots and checks seq_len, so that every later kernel of
@@ -20,15 +21,38 @@
 
 namespace tria {
 
+static_assert(TRIA_MAX_BATCH <= 256, "the fold handles one sequence per thread of a block");
+
 __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldParams p) {
   dev::pdl_launch_dependents();  // the score kernel may start streaming keys now
   const int fp = blockIdx.x;
   const int F = p.D / 2;
   __shared__ double red[4][8];
   __shared__ double2 ea[TRIA_MAX_BATCH][2];
-  double w[2];
+  // Loads that do not depend on the trigonometry are issued first.
+  const int64_t units = (int64_t)p.L * p.Hkv * p.B;
+  const int64_t entries = units * p.G;
+  const int64_t e0 = (int64_t)blockIdx.y * blockDim.x + threadIdx.x;
+  float2 c0[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float r0[2] = {0.f, 0.f}, m0[2] = {0.f, 0.f};
+  if (e0 < entries) {
+    const int64_t unit = e0 / p.G;
+    const int h = (int)(e0 - unit * p.G);
+    const int64_t lg = unit / p.B;
+    const int l = (int)(lg / p.Hkv), g = (int)(lg % p.Hkv);
+    const size_t base0 = ((size_t)l * p.Hq + (size_t)g * p.G + h) * F + 2 * fp;
 #pragma unroll
-  for (int q = 0; q < 2; ++q) w[q] = pow(p.theta, -2.0 * (double)(2 * fp + q) / (double)p.D);
+    for (int q = 0; q < 2; ++q) {
+      c0[q] = p.centre[base0 + q];
+      r0[q] = p.mrl[base0 + q];
+      m0[q] = p.mean_norm[base0 + q];
+    }
+  }
+  const int32_t cur = threadIdx.x < p.B ? p.cur_pos[threadIdx.x] : 0;
+  const bool snap = blockIdx.x == 0 && blockIdx.y == 0 && (int)threadIdx.x < p.B;
+  const int32_t t_in = snap ? p.seq_len[threadIdx.x] : 0;
+  // w_f = theta^(-2f/D), evaluated on the host in double precision
+  const double w[2] = {p.omega[2 * fp], p.omega[2 * fp + 1]};
   double a[4] = {0.0, 0.0, 0.0, 0.0};  // (cos, sin) sums for the two pairs
   for (int j = threadIdx.x; j < p.n_offsets; j += blockDim.x) {
 #pragma unroll
@@ -55,21 +79,19 @@ __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldP
     A[i] = (p.flags & TRIA_NO_TRIG) ? 0.0 : s / (double)p.n_offsets;
   }
   for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+    const int32_t cb = b == (int)threadIdx.x ? cur : p.cur_pos[b];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       double s, c;
-      sincos(w[q] * (double)p.cur_pos[b], &s, &c);
+      sincos(w[q] * (double)cb, &s, &c);
       const double ax = A[2 * q], ay = A[2 * q + 1];
       ea[b][q] = make_double2(c * ax - s * ay, c * ay + s * ax);
     }
   }
   __syncthreads();
 
-  const int64_t units = (int64_t)p.L * p.Hkv * p.B;
-  const int64_t entries = units * p.G;
   const int FP = F / 2;
-  for (int64_t e = (int64_t)blockIdx.y * blockDim.x + threadIdx.x; e < entries;
-       e += (int64_t)gridDim.y * blockDim.x) {
+  for (int64_t e = e0; e < entries; e += (int64_t)gridDim.y * blockDim.x) {
     const int64_t unit = e / p.G;
     const int h = (int)(e - unit * p.G);
     const int b = (int)(unit % p.B);
@@ -79,12 +101,13 @@ __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldP
     float wx[2], wy[2], nw[2];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-      const float2 c = p.centre[base + q];
+      const bool pre = e == e0;  // the first entry's inputs were loaded up front
+      const float2 c = pre ? c0[q] : p.centre[base + q];
       const double2 e2 = ea[b][q];
       wx[q] = (float)((double)c.x * e2.x - (double)c.y * e2.y);
       wy[q] = (float)((double)c.x * e2.y + (double)c.y * e2.x);
-      const float r = (p.flags & TRIA_NO_CONC_WEIGHT) ? 0.0f : p.mrl[base + q];
-      nw[q] = (1.0f - r) * p.mean_norm[base + q];
+      const float r = (p.flags & TRIA_NO_CONC_WEIGHT) ? 0.0f : (pre ? r0[q] : p.mrl[base + q]);
+      nw[q] = (1.0f - r) * (pre ? m0[q] : p.mean_norm[base + q]);
     }
     float2 *out = reinterpret_cast<float2 *>(p.w + ((size_t)unit * FP + fp) * (6 * p.G) + 6 * h);
     out[0] = make_float2(wx[0], wx[1]);
@@ -92,15 +115,13 @@ __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldP
     out[2] = make_float2(nw[0], nw[1]);
   }
 
-  if (blockIdx.x == 0 && blockIdx.y == 0) {
-    for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
-      int32_t T = p.seq_len[b];
-      if (T < 0 || (int64_t)T > p.seg_cap[b]) {
-        dev::set_error(p.err, TRIA_DEVERR_SEQ_LEN);
-        T = 0;
-      }
-      p.seqlen_snap[b] = T;
+  if (snap) {  // B <= TRIA_MAX_BATCH = blockDim.x: one sequence per thread
+    int32_t T = t_in;
+    if (T < 0 || (int64_t)T > p.seg_cap[threadIdx.x]) {
+      dev::set_error(p.err, TRIA_DEVERR_SEQ_LEN);
+      T = 0;
     }
+    p.seqlen_snap[threadIdx.x] = T;
   }
 }
 

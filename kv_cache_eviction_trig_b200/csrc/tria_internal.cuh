@@ -72,6 +72,7 @@ struct FoldParams {
   uint32_t flags;
   int64_t seg_cap[TRIA_MAX_BATCH];
   int32_t offsets[TRIA_MAX_OFFSETS];
+  double omega[128];        // w_f = theta^(-2f/D), f < D/2
 };
 
 struct alignas(64) ScoreParams {

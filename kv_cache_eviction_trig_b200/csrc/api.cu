@@ -225,8 +225,14 @@ void fill_unit(UnitParams &up, const tria_config *cfg, const tria_cache *c, int 
   up.D = cfg->head_dim;
   up.budget = cfg->budget;
   up.mode = mode;
-  for (int b = 0; b <= cfg->batch; ++b) up.seg_start[b] = c->seq_start[b];
+  int64_t most = 0;
+  for (int b = 0; b <= cfg->batch; ++b) {
+    up.seg_start[b] = c->seq_start[b];
+    if (b < cfg->batch && c->seq_start[b + 1] - c->seq_start[b] > most)
+      most = c->seq_start[b + 1] - c->seq_start[b];
+  }
   up.smem_bytes = unit_smem_bytes();
+  up.cluster = unit_cluster_size((int64_t)cfg->num_layers * cfg->n_kv_heads * cfg->batch, most);
 }
 
 struct Ws {

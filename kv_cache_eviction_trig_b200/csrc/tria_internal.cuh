@@ -56,6 +56,7 @@ constexpr int kScoreRingBytes = 220 * 1024;  // shared memory for key chunks and
 #endif
 constexpr int kUnitThreads = TRIA_UNIT_THREADS;  // build-time tunable: 256, 512 or 1024
 constexpr int kUnitCluster = 8;
+constexpr int kUnitClustersAtOnce = 15;  // 8-CTA clusters of 200 KB resident at once on a B200
 constexpr int kUnitSmemLarge = 200 * 1024;  // one CTA per SM
 
 struct FoldParams {
@@ -113,6 +114,7 @@ struct UnitParams {
   int32_t mode;
   int32_t write_short_sel;  // prune: also write identity lists for sequences not pruned
   int32_t smem_bytes;       // dynamic shared memory of the launch
+  int32_t cluster;          // CTAs per unit (1 or kUnitCluster)
   int64_t seg_start[TRIA_MAX_BATCH + 1];
 };
 
@@ -126,7 +128,8 @@ int score_chunk_keys(int D, int G);
 cudaError_t make_key_tensor_map(CUtensorMap *map, const void *k, int D, int64_t rows,
                                 int box_rows);
 cudaError_t launch_unit(const UnitParams &p, int units, cudaStream_t s, bool pdl);
-int unit_cluster_size();
+// CTAs per unit: 8 (one cluster) for few units, 1 for many units whose segments fit.
+int unit_cluster_size(int64_t units, int64_t max_segment);
 int unit_smem_bytes();
 cudaError_t launch_calibrate(const void *q, int q_dtype, int64_t L, int64_t N, int64_t Hq,
                              int64_t D, int layout, float *centre, float *mean_norm, float *mrl,

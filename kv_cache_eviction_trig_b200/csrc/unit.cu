@@ -174,13 +174,14 @@ __device__ __forceinline__ void find_bin(const uint32_t *tot, int nbins, int kre
 // One warp: in the counts cnt[q][i] of CL peers over 64 bins ordered by
 // increasing key, the bin holding the krem-th largest counted key, the number
 // of counted keys above it and its own count (returned to every lane).
+template <int CL>
 __device__ __forceinline__ void warp_find_bin64(const uint32_t *cnt, int krem, int *bin, int *above,
                                                 int *count) {
   const int lane = threadIdx.x & 31;
   const int bh = 63 - 2 * lane, bl = 62 - 2 * lane;  // this lane's bins, higher first
   int ch = 0, cl_ = 0;
 #pragma unroll
-  for (int q = 0; q < kUnitCluster; ++q) {
+  for (int q = 0; q < CL; ++q) {
     ch += (int)cnt[q * 64 + bh];
     cl_ += (int)cnt[q * 64 + bl];
   }
@@ -203,10 +204,11 @@ __device__ __forceinline__ void warp_find_bin64(const uint32_t *cnt, int krem, i
 }
 
 // Peer whose range [off[q], off[q+1]) holds index i (off has CL+1 entries).
+template <int CL>
 __device__ __forceinline__ int owner_of(const int32_t *off, int i) {
   int q = 0;
 #pragma unroll
-  for (int k = 1; k < kUnitCluster; ++k) q += off[k] <= i;
+  for (int k = 1; k < CL; ++k) q += off[k] <= i;
   return q;
 }
 
@@ -253,10 +255,10 @@ __device__ __forceinline__ void stage_rows(const int32_t *src, int m, const uint
 
 }  // namespace
 
-template <int G>
+template <int G, int CL>
 __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_constant__ UnitParams p) {
+  static_assert(CL == 1 || CL == kUnitCluster, "a unit is one CTA or one full cluster");
   cg::cluster_group cl = cg::this_cluster();
-  constexpr int CL = kUnitCluster;
   const int r = (int)cl.block_rank();
   const int64_t unit = blockIdx.x / CL;
   const int b = (int)(unit % p.B);
@@ -475,7 +477,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       __syncthreads();
       if (tid < 32) {
         int bin, above, cnt;
-        warp_find_bin64(&c.gc[0][0], krem, &bin, &above, &cnt);
+        warp_find_bin64<CL>(&c.gc[0][0], krem, &bin, &above, &cnt);
         if (tid == 0) { c.bc[0] = bin; c.bc[1] = above; }
       }
       __syncthreads();
@@ -487,7 +489,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       __syncthreads();
       if (tid < 32) {
         int bin, above, cnt;
-        warp_find_bin64(&c.gc[0][0], krem, &bin, &above, &cnt);
+        warp_find_bin64<CL>(&c.gc[0][0], krem, &bin, &above, &cnt);
         if (tid == 0) { c.bc[0] = cbin * 64 + bin; c.bc[1] = above; c.bc[2] = cnt; }
       }
       __syncthreads();
@@ -513,16 +515,28 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       const int dshift = top >= 12 ? top - 12 : 0;
       const int dbits = top - dshift;
       const int nb = 1 << dbits;
-      const int per_log2 = dbits - 3;  // bins per owner: nb / 8
-      for (int i = tid; i < n; i += nthr) {
-        const uint32_t key = zkey[i];
-        if (in_bucket(key))
-          cluster_hist_add(cl, &c.slice[round][0], (key >> dshift) & (nb - 1), per_log2);
+      if constexpr (CL == 1) {
+        // one CTA holds the whole unit: count straight into `tot` (its first-round
+        // counts are no longer needed)
+        for (int i = tid; i < nb; i += nthr) tot[i] = 0u;
+        __syncthreads();
+        for (int i = tid; i < n; i += nthr) {
+          const uint32_t key = zkey[i];
+          if (in_bucket(key)) atomicAdd(&tot[(key >> dshift) & (nb - 1)], 1u);
+        }
+        __syncthreads();
+      } else {
+        const int per_log2 = dbits - 3;  // bins per owner: nb / 8
+        for (int i = tid; i < n; i += nthr) {
+          const uint32_t key = zkey[i];
+          if (in_bucket(key))
+            cluster_hist_add(cl, &c.slice[round][0], (key >> dshift) & (nb - 1), per_log2);
+        }
+        cl.sync();  // every count of this round has landed
+        for (int i = tid; i < nb; i += nthr)
+          tot[i] = cl.map_shared_rank(&c.slice[round][0], i >> per_log2)[i & ((1 << per_log2) - 1)];
+        __syncthreads();
       }
-      cl.sync();  // every count of this round has landed
-      for (int i = tid; i < nb; i += nthr)
-        tot[i] = cl.map_shared_rank(&c.slice[round][0], i >> per_log2)[i & ((1 << per_log2) - 1)];
-      __syncthreads();
       int bin, above;
       find_bin(tot, nb, krem, c.bc, c.scan, &bin, &above, &bucket);
       krem -= above;
@@ -579,7 +593,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       const int C = c.off[CL];
       uint32_t *gkey = tot;  // [C], C <= cand_cap <= kBins
       for (int i = tid; i < C; i += nthr) {
-        const int q = owner_of(c.off, i);
+        const int q = owner_of<CL>(c.off, i);
         gkey[i] = cl.map_shared_rank(cand_key, q)[i - c.off[q]];
         gslot[i] = cl.map_shared_rank(cand_slot, q)[i - c.off[q]];
       }
@@ -627,7 +641,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       // per peer: bucket keys above thr and equal to thr
       for (int i = tid; i < C; i += nthr) {
         const uint32_t key = gkey[i];
-        if (key >= thr) atomicAdd(&c.gcnt[owner_of(c.off, i)][key == thr ? 1 : 0], 1);
+        if (key >= thr) atomicAdd(&c.gcnt[owner_of<CL>(c.off, i)][key == thr ? 1 : 0], 1);
       }
       __syncthreads();
     } else {
@@ -715,7 +729,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
         const int j = j0 + jj;
         int q = 0;  // the peer whose kept keys include output index j
 #pragma unroll
-        for (int k = 1; k < kUnitCluster; ++k) q += c.base[k] <= j;
+        for (int k = 1; k < CL; ++k) q += c.base[k] <= j;
         c.src[jj] = cl.map_shared_rank(&c.kept_src[0], q)[j - c.base[q]];
       }
       __syncthreads();
@@ -779,38 +793,51 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
 
 // Launch configuration: 8-CTA clusters of 1024 threads, one CTA per SM
 // (portable cluster size; 15 clusters are resident at once on a B200).
-int unit_cluster_size() { return kUnitCluster; }
-
-template <int G>
+template <int G, int CL>
 static void configure_unit() {
-  cudaFuncSetAttribute(unit_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kUnitSmemLarge);
+  cudaFuncSetAttribute(unit_kernel<G, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       kUnitSmemLarge);
 }
 
 int unit_smem_bytes() {
-  // the large size holds the keys of a TRIA_MAX_SEGMENT segment per CTA
+  // the large size holds the keys of a TRIA_MAX_SEGMENT segment per CTA of a cluster
   static bool configured[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && !configured[dev]) {
-    configure_unit<1>();
-    configure_unit<2>();
-    configure_unit<4>();
-    configure_unit<8>();
-    configure_unit<16>();
+    configure_unit<1, 1>();
+    configure_unit<2, 1>();
+    configure_unit<4, 1>();
+    configure_unit<8, 1>();
+    configure_unit<16, 1>();
+    configure_unit<1, kUnitCluster>();
+    configure_unit<2, kUnitCluster>();
+    configure_unit<4, kUnitCluster>();
+    configure_unit<8, kUnitCluster>();
+    configure_unit<16, kUnitCluster>();
     configured[dev] = true;
   }
   return kUnitSmemLarge;
 }
 
-cudaError_t launch_unit(const UnitParams &p, int units, cudaStream_t s, bool pdl) {
-  const int cs = kUnitCluster;
+int unit_cluster_size(int64_t units, int64_t max_segment) {
+  // Few units: a cluster of CTAs per unit (latency).  Many units: one CTA per unit
+  // (more units at once), when a CTA's shared memory holds a whole segment's keys:
+  // zkey + first-round histogram + gathered slots + a minimal bucket list.
+  const int64_t data = kUnitSmemLarge - kCtl;
+  const bool fits = 4 * ((max_segment + 3) & ~3ll) + 4ll * kBins + 4ll * kCandMax + 8ll * 256 <= data;
+  return (units > kUnitClustersAtOnce && fits) ? 1 : kUnitCluster;
+}
+
+template <int CL>
+static cudaError_t launch_unit_cl(const UnitParams &p, int units, cudaStream_t s, bool pdl) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)units * cs, 1, 1);
+  cfg.gridDim = dim3((unsigned)units * CL, 1, 1);
   cfg.blockDim = dim3(kUnitThreads, 1, 1);
   cfg.dynamicSmemBytes = p.smem_bytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.x = CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -820,13 +847,18 @@ cudaError_t launch_unit(const UnitParams &p, int units, cudaStream_t s, bool pdl
   // the group size only shapes the z-score stage
   const int G = (p.mode == kModeZmax || p.mode == kModePrune) ? p.G : 1;
   switch (G) {
-    case 1: return cudaLaunchKernelEx(&cfg, unit_kernel<1>, p);
-    case 2: return cudaLaunchKernelEx(&cfg, unit_kernel<2>, p);
-    case 4: return cudaLaunchKernelEx(&cfg, unit_kernel<4>, p);
-    case 8: return cudaLaunchKernelEx(&cfg, unit_kernel<8>, p);
-    case 16: return cudaLaunchKernelEx(&cfg, unit_kernel<16>, p);
+    case 1: return cudaLaunchKernelEx(&cfg, unit_kernel<1, CL>, p);
+    case 2: return cudaLaunchKernelEx(&cfg, unit_kernel<2, CL>, p);
+    case 4: return cudaLaunchKernelEx(&cfg, unit_kernel<4, CL>, p);
+    case 8: return cudaLaunchKernelEx(&cfg, unit_kernel<8, CL>, p);
+    case 16: return cudaLaunchKernelEx(&cfg, unit_kernel<16, CL>, p);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_unit(const UnitParams &p, int units, cudaStream_t s, bool pdl) {
+  return p.cluster == 1 ? launch_unit_cl<1>(p, units, s, pdl)
+                        : launch_unit_cl<kUnitCluster>(p, units, s, pdl);
 }
 
 }  // namespace tria

@@ -261,11 +261,13 @@ def test_compact_in_place_is_bit_exact(kind):
 
 
 @pytest.mark.parametrize("kind", ["last", "alternating", "random"])
-@pytest.mark.parametrize("D,budget,T", [(128, 3500, 4000), (256, 2000, 2500)])
-def test_compact_many_units_multi_batch(kind, D, budget, T):
-    """Budgets larger than one cluster can stage at once (about 2900 rows of
-    D=128, 1400 of D=256) are compacted in several cluster-wide batches."""
-    wl = small("compact-multi", L=2, Hq=32, Hkv=8, B=1, D=D, seq_lens=[T], budget=budget)
+@pytest.mark.parametrize("L,D,budget,T", [(2, 128, 3500, 4000), (2, 256, 2000, 2500),
+                                          (1, 128, 3500, 4000)])
+def test_compact_many_units_multi_batch(kind, L, D, budget, T):
+    """Budgets larger than a unit's CTAs can stage at once are compacted in several
+    batches: 16 units (one CTA each; about 330 rows of D=128 or 166 of D=256 per batch)
+    and 8 units (one 8-CTA cluster each; about 2600 rows of D=128 per batch)."""
+    wl = small("compact-multi", L=L, Hq=32, Hkv=8, B=1, D=D, seq_lens=[T], budget=budget)
     case = Case(wl)
     rng = np.random.default_rng(11)
     sel = np.stack([np.stack([np.stack([_adversarial_sel(kind, T, wl.budget, rng)
@@ -386,3 +388,45 @@ def test_repeated_prune_is_stable():
     torch.cuda.synchronize()
     for n, t in snap.items():
         assert torch.equal(case.dev[n], t)
+
+
+# Problems with more than 15 units run one CTA per unit instead of one 8-CTA cluster.
+
+def test_prune_edge_lengths_one_cta_per_unit():
+    """40 units (L2 x Hkv4 x B5): T = 0, < budget, = budget, budget + 1 and long."""
+    wl = small("edges-1cta", L=2, B=5, Hq=8, Hkv=4, seq_lens=[0, 50, 100, 101, 900], budget=100,
+               slack=3)
+    case = Case(wl)
+    ref = oracle.prune(case.prob, common.bf16_bits(case.host["v"]))
+    sel = torch.full((2, 4, 5, 100), -7, dtype=torch.int32, device="cuda")
+    tria.tria_prune(case.cfg, case.stats, case.cache, case.ws, sel_out=sel)
+    torch.cuda.synchronize()
+    assert tria.tria_get_device_error(case.ws) == 0
+    assert case.dev["seq_len"].cpu().tolist() == [0, 50, 100, 100, 100]
+    gsel = sel.cpu().numpy()
+    check_selection(gsel, ref["sel"], ref["raw"], ref["score"], case)
+    check_compacted(case, gsel, [0, 50, 100, 100, 100])
+
+
+def test_score_one_cta_per_unit():
+    case = Case(small("score-1cta", L=2, B=3, Hq=8, Hkv=4, seq_lens=[700, 129, 2000], budget=64,
+                      offsets=[2 ** i for i in range(12)]))
+    ref_raw = oracle.raw_scores(case.prob)
+    _, ref_score = oracle.zmax(case.prob, ref_raw)
+    gpu_raw, gpu_score = case.gpu_score()
+    check_raw(gpu_raw, ref_raw, case)
+    check_score(gpu_score, ref_raw, ref_score, case)
+
+
+def test_select_on_identical_scores_one_cta_per_unit():
+    case = Case(small("select-1cta", L=2, B=2, Hq=8, Hkv=4, seq_lens=[1500, 333], budget=200))
+    wl = case.wl
+    rng = np.random.default_rng(9)
+    score = rng.normal(size=(wl.num_layers, wl.n_kv_heads, wl.cap_total)).astype(np.float32)
+    score[..., ::5] = score[..., 2:3]          # many exact ties
+    score[..., 1::7] = -0.0
+    sel = torch.full((wl.num_layers, wl.n_kv_heads, wl.batch, wl.budget), -7, dtype=torch.int32,
+                     device="cuda")
+    tria.tria_select(case.cfg, case.cache, torch.from_numpy(score).cuda(), sel, case.ws)
+    ref = oracle.select(case.prob, score.astype(np.float64))
+    np.testing.assert_array_equal(sel.cpu().numpy(), ref)

@@ -53,6 +53,7 @@ constexpr int kCtl = 32 * 1024;  // control region at the start of shared memory
 constexpr int kMaxG = 16;
 constexpr int kMaxCluster = 16;
 constexpr int kWarps = kUnitThreads / 32;
+static_assert(kWarps >= 1 && kWarps <= 32, "one lane per warp in the emit prefix");
 constexpr int kBins = 4096;                   // cluster-wide histogram bins
 constexpr int kSlice = kBins / kUnitCluster;  // bins each CTA of the cluster owns
 constexpr int kRounds = 3;                    // refinement rounds (12, 12, 8 key bits)
@@ -73,6 +74,7 @@ struct Ctl {
   int32_t bc[8];                    // broadcast scalars
   int32_t gcnt[kMaxCluster][2];     // per peer: bucket keys above the threshold, equal to it
   int32_t scan[kWarps + 1];
+  int32_t wgt[kWarps], weq[kWarps];  // per warp: its run's keys above and equal to thr
   int32_t src[kOwnRows];            // source slots of this CTA's share of the destinations
   int32_t base[kMaxCluster];        // per peer: first output index of its kept keys
   int32_t keptq[kMaxCluster];       // per peer: its kept keys
@@ -568,10 +570,6 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       for (int o = 16; o > 0; o >>= 1) above_local += __shfl_xor_sync(0xffffffffu, above_local, o);
       if ((tid & 31) == 0 && above_local) atomicAdd(&c.cnt[0], above_local);
     }
-    // Each thread also owns a contiguous run of this CTA's keys, so runs in thread
-    // order are in slot order (used when the kept keys are emitted).
-    const int RL = (n + nthr - 1) / nthr;
-    const int a0 = min(n, tid * RL), a1 = min(n, a0 + RL);
     cl.sync();  // counts and bucket lists complete
     if (tid < CL) {
       const Ctl *peer = cl.map_shared_rank(&c, tid);
@@ -694,29 +692,44 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     k_eq = c.bc[3];
     const bool balanced = balanced_fit && c.bc[7] <= kKeptMax;
     {
+      // Warp w owns a contiguous run of this CTA's keys (runs in warp order are in
+      // slot order); its lanes read consecutive keys, so the shared-memory reads are
+      // free of bank conflicts, and ballots order the kept keys inside each step.
+      const int warp = tid >> 5, lane = tid & 31;
+      const int WL = ((n + kWarps - 1) / kWarps + 31) & ~31;
+      const int w0 = min(n, warp * WL), w1 = min(n, w0 + WL);
       int gt = 0, eq = 0;
-      for (int i = a0; i < a1; ++i) {
+      for (int i = w0 + lane; i < w1; i += 32) {
         const uint32_t key = zkey[i];
         gt += key > thr;
         eq += key == thr;
       }
-      int tot2;
-      const int x2 = block_excl_scan((gt << 16) | eq, c.scan, &tot2);
-      const int eq_x = x2 & 0xffff;
+      gt = __reduce_add_sync(0xffffffffu, gt);
+      eq = __reduce_add_sync(0xffffffffu, eq);
+      if (lane == 0) { c.wgt[warp] = gt; c.weq[warp] = eq; }
+      __syncthreads();
+      // keys above thr and keys equal to thr in the runs of the warps before this one
+      const int gt_x = __reduce_add_sync(0xffffffffu, lane < warp ? c.wgt[lane] : 0);
+      const int eq_x = __reduce_add_sync(0xffffffffu, lane < warp ? c.weq[lane] : 0);
       int er = c.bc[5] + eq_x;  // cluster-wide rank of this run's first key equal to thr
-      int o = c.bc[4] + (x2 >> 16) + max(0, min(eq_x, k_eq - c.bc[5]));
-      for (int i = a0; i < a1; ++i) {
-        const uint32_t key = zkey[i];
-        bool keep = key > thr;
-        if (key == thr) { keep = er < k_eq; ++er; }
-        if (keep) {
-          if (o < p.budget) {
-            const int32_t slot = (int32_t)(lo + i);
-            sel[o] = slot;
-            if (balanced) c.kept_src[o - c.bc[4]] = slot;  // read by the compacting CTAs
-          }
-          ++o;
+      int o = c.bc[4] + gt_x + max(0, min(eq_x, k_eq - c.bc[5]));
+      const uint32_t below = (1u << lane) - 1u;
+      for (int i0 = w0; i0 < w1; i0 += 32) {
+        const int i = i0 + lane;
+        const bool in = i < w1;
+        const uint32_t key = in ? zkey[i] : 0u;
+        const bool is_eq = in && key == thr;
+        const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
+        const bool keep = in && (key > thr || (is_eq && er + __popc(eqm & below) < k_eq));
+        const uint32_t km = __ballot_sync(0xffffffffu, keep);
+        const int oi = o + __popc(km & below);
+        if (keep && oi < p.budget) {
+          const int32_t slot = (int32_t)(lo + i);
+          sel[oi] = slot;
+          if (balanced) c.kept_src[oi - c.bc[4]] = slot;  // read by the compacting CTAs
         }
+        o += __popc(km);
+        er += __popc(eqm);
       }
     }
     cl.sync();  // selection lists complete and visible; peers' keys are no longer read

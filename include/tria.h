@@ -81,6 +81,7 @@ typedef enum {
 #define TRIA_DEVERR_SELECTION 2    /* tria_compact: selection not ascending / out of range: unit skipped */
 #define TRIA_DEVERR_TIMEOUT 4      /* a bounded wait on an mbarrier ran out: results invalid */
 #define TRIA_DEVERR_SEGMENT_BIG 8  /* a live sequence exceeded the kernel's per-unit capacity */
+#define TRIA_DEVERR_SEGMENT_FULL 16 /* tria_append: no free slot in a segment: that sequence skipped */
 
 /* Host-side description of the prune problem, copied by value. */
 typedef struct {
@@ -95,6 +96,12 @@ typedef struct {
   const int32_t *offsets; /* HOST [n_offsets] future query offsets, each >= 1 */
   int32_t n_offsets;
   uint32_t flags;       /* 0, or TRIA_NO_TRIG / TRIA_NO_CONC_WEIGHT */
+  int32_t prune_window; /* >= 0.  tria_prune / tria_prune_noalloc prune a sequence only
+                           once seq_len >= budget + max(prune_window, 1) (a decode loop
+                           that calls tria_prune after every tria_append then prunes each
+                           sequence back to budget every prune_window decoded tokens);
+                           0 or 1: every sequence with seq_len > budget.  Other calls
+                           ignore it. */
 } tria_config;
 
 /* The cache.  Device pointers except seq_start. */
@@ -103,7 +110,8 @@ typedef struct {
   void *v;                 /* DEVICE bf16 [L][Hkv][cap_total][D], 16-byte aligned */
   int32_t *pos;            /* DEVICE int32 [L][Hkv][cap_total], 16-byte aligned */
   int32_t *seq_len;        /* DEVICE int32 [B], live keys per sequence (in/out) */
-  const int32_t *cur_pos;  /* DEVICE int32 [B], position of each sequence's newest token */
+  int32_t *cur_pos;        /* DEVICE int32 [B], position of each sequence's newest token
+                              (read by the scoring calls, advanced by tria_append) */
   const int64_t *seq_start;/* HOST int64 [B+1], nondecreasing, seq_start[B] <= cap_total */
   int64_t cap_total;       /* slots per (layer, KV head) row */
 } tria_cache;
@@ -159,12 +167,30 @@ tria_status tria_compact(const tria_config *cfg, const tria_cache *cache, const 
                          void *ws, size_t ws_bytes, void *stream);
 
 /* The whole prune step in one call: score, z-score + group max, select and
- * compact every (layer, KV head, sequence) with seq_len > budget; shorter
- * sequences are left untouched.  seq_len is read once at the start and
- * rewritten at the end.  If sel_out is not NULL it receives the selection
- * as tria_select would write it (for units that were pruned). */
+ * compact every (layer, KV head, sequence) with seq_len > budget (and
+ * seq_len >= budget + cfg->prune_window); other sequences are left untouched.
+ * seq_len is read once at the start and rewritten at the end.  If sel_out is
+ * not NULL it receives the selection as tria_select would write it for the
+ * sequences that were pruned and for those with seq_len <= budget; the rows of
+ * sequences held back by prune_window are not written. */
 tria_status tria_prune(const tria_config *cfg, const tria_stats *stats, const tria_cache *cache,
                        int32_t *sel_out, void *ws, size_t ws_bytes, void *stream);
+
+/* The decode-loop step before the prune (romaanj.github.io review, "Background":
+ * every decoded token is appended to the cache; dimensionstp.github.io review,
+ * section 3-2 (5), window-based pruning).  k_new and v_new are DEVICE bf16
+ * [L][Hkv][B][D], 16-byte aligned: the new token of every sequence.  For every
+ * (layer, KV head, sequence) the token's K and V rows go to slot
+ * seq_start[b] + seq_len[b] and its position cur_pos[b] + 1 to pos; then
+ * seq_len[b] and cur_pos[b] advance by one.  A sequence whose segment has no
+ * free slot (seq_len[b] == segment capacity) is left unchanged and sets
+ * TRIA_DEVERR_SEGMENT_FULL; one with seq_len[b] out of range sets
+ * TRIA_DEVERR_SEQ_LEN.  Two kernel launches, no host synchronisation: a decode
+ * step (tria_append, then tria_prune with cfg->prune_window) can be captured in
+ * a CUDA graph and replayed.  ws as for the other calls (only its error word is
+ * used). */
+tria_status tria_append(const tria_config *cfg, const tria_cache *cache, const void *k_new,
+                        const void *v_new, void *ws, size_t ws_bytes, void *stream);
 
 /* tria_prune with a cudaEvent_t (as void*) recorded on `stream` before each
  * of its kernels and after the last: events[0..n_stages].  Returns the number

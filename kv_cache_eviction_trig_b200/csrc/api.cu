@@ -83,6 +83,7 @@ tria_status check_config(const tria_config *cfg, bool scoring) {
   if (cfg->budget < 1) return TRIA_ERR_INVALID_ARG;
   if (cfg->budget > TRIA_MAX_SEGMENT) return TRIA_ERR_UNSUPPORTED;
   if (cfg->n_q_heads / cfg->n_kv_heads > 16) return TRIA_ERR_UNSUPPORTED;
+  if (cfg->prune_window < 0) return TRIA_ERR_INVALID_ARG;
   if (scoring) {
     if (!(cfg->rope_theta > 1.0) || !std::isfinite(cfg->rope_theta)) return TRIA_ERR_INVALID_ARG;
     if (!cfg->offsets || cfg->n_offsets < 1) return TRIA_ERR_INVALID_ARG;
@@ -137,6 +138,13 @@ tria_status check_ws(const tria_config *cfg, const tria_cache *c, void *ws, size
 
 tria_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TRIA_OK : TRIA_ERR_CUDA; }
 
+// The shortest live length the prune acts on: budget + max(prune_window, 1).
+int32_t prune_from(const tria_config *cfg) {
+  const int64_t w = cfg->prune_window > 1 ? cfg->prune_window : 1;
+  const int64_t t = (int64_t)cfg->budget + w;
+  return t < INT32_MAX ? (int32_t)t : INT32_MAX;
+}
+
 void fill_fold(FoldParams &fp, const tria_config *cfg, const tria_stats *st,
                const tria_cache *c, int32_t *seqlen_snap, float *w, int32_t *err) {
   std::memset(&fp, 0, sizeof fp);
@@ -181,7 +189,7 @@ cudaError_t fill_score(ScoreParams &sp, const tria_config *cfg, const tria_cache
   sp.Hkv = cfg->n_kv_heads;
   sp.Hq = cfg->n_q_heads;
   sp.B = cfg->batch;
-  sp.budget = cfg->budget;
+  sp.prune_from = prune_from(cfg);
   sp.skip_short = skip_short;
   int32_t acc = 0;
   for (int b = 0; b <= cfg->batch; ++b) {
@@ -224,6 +232,7 @@ void fill_unit(UnitParams &up, const tria_config *cfg, const tria_cache *c, int 
   up.G = cfg->n_q_heads / cfg->n_kv_heads;
   up.D = cfg->head_dim;
   up.budget = cfg->budget;
+  up.prune_from = prune_from(cfg);
   up.mode = mode;
   int64_t most = 0;
   for (int b = 0; b <= cfg->batch; ++b) {
@@ -353,6 +362,35 @@ tria_status tria_compact(const tria_config *cfg, const tria_cache *cache, const 
   up.err = w.err();
   return cuda_status(launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch,
                                  static_cast<cudaStream_t>(stream), false));
+}
+
+tria_status tria_append(const tria_config *cfg, const tria_cache *cache, const void *k_new,
+                        const void *v_new, void *ws, size_t ws_bytes, void *stream) {
+  tria_status s;
+  if ((s = check_config(cfg, false)) != TRIA_OK) return s;
+  if ((s = check_cache(cfg, cache, true)) != TRIA_OK) return s;
+  if (!cache->cur_pos) return TRIA_ERR_INVALID_ARG;
+  if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return TRIA_ERR_INVALID_ARG;
+  if (cfg->head_dim > 256) return TRIA_ERR_UNSUPPORTED;
+  if ((s = check_ws(cfg, cache, ws, ws_bytes)) != TRIA_OK) return s;
+  const Ws w{ws_layout(*cfg, cache->seq_start, cache->cap_total), static_cast<uint8_t *>(ws)};
+  AppendParams ap;
+  std::memset(&ap, 0, sizeof ap);
+  ap.k_new = static_cast<const uint8_t *>(k_new);
+  ap.v_new = static_cast<const uint8_t *>(v_new);
+  ap.k = static_cast<uint8_t *>(cache->k);
+  ap.v = static_cast<uint8_t *>(cache->v);
+  ap.pos = cache->pos;
+  ap.seq_len = cache->seq_len;
+  ap.cur_pos = cache->cur_pos;
+  ap.err = w.err();
+  ap.cap = cache->cap_total;
+  ap.L = cfg->num_layers;
+  ap.Hkv = cfg->n_kv_heads;
+  ap.B = cfg->batch;
+  ap.D = cfg->head_dim;
+  for (int b = 0; b <= cfg->batch; ++b) ap.seg_start[b] = cache->seq_start[b];
+  return cuda_status(launch_append(ap, static_cast<cudaStream_t>(stream)));
 }
 
 tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,

@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     for (int b = lane; b < p.B; b += 32) {
       int32_t T = p.seq_len[b];
       if (T < 0 || (int64_t)T > p.seg_start[b + 1] - p.seg_start[b]) T = 0;  // flagged by the fold
-      if (p.skip_short && T <= p.budget) T = 0;
+      if (p.skip_short && T < p.prune_from) T = 0;
       live[b] = T;
     }
     __syncwarp();

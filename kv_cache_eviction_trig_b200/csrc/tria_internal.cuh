@@ -85,8 +85,9 @@ struct alignas(64) ScoreParams {
   int32_t max_slots;
   int32_t *err;
   int64_t cap;
-  int32_t L, Hkv, Hq, B, budget;
-  int32_t skip_short;       // 1: sequences with seq_len <= budget are not scored
+  int32_t L, Hkv, Hq, B;
+  int32_t prune_from;       // with skip_short: the shortest seq_len that is pruned
+  int32_t skip_short;       // 1: sequences with seq_len < prune_from are not scored
   int32_t chunks_per_row;   // chunk_prefix[B]
   int32_t chunks_per_cta;
   int32_t total_chunks;     // < 2^31 (checked on the host)
@@ -111,8 +112,9 @@ struct UnitParams {
   int32_t *err;
   int64_t cap;
   int32_t L, Hkv, Hq, B, G, D, budget;
+  int32_t prune_from;       // prune: the shortest seq_len that is pruned (> budget)
   int32_t mode;
-  int32_t write_short_sel;  // prune: also write identity lists for sequences not pruned
+  int32_t write_short_sel;  // prune: also write identity lists for seq_len <= budget
   int32_t smem_bytes;       // dynamic shared memory of the launch
   int32_t cluster;          // CTAs per unit (1 or kUnitCluster)
   int64_t seg_start[TRIA_MAX_BATCH + 1];
@@ -131,6 +133,22 @@ cudaError_t launch_unit(const UnitParams &p, int units, cudaStream_t s, bool pdl
 // CTAs per unit: 8 (one cluster) for few units, 1 for many units whose segments fit.
 int unit_cluster_size(int64_t units, int64_t max_segment);
 int unit_smem_bytes();
+// Decode-loop append: the new token's K, V rows and position into each segment's
+// next free slot, then seq_len and cur_pos advance (two launches).
+struct AppendParams {
+  const uint8_t *k_new;     // bf16 [L][Hkv][B][D]
+  const uint8_t *v_new;
+  uint8_t *k;               // bf16 [L][Hkv][cap][D]
+  uint8_t *v;
+  int32_t *pos;             // [L][Hkv][cap]
+  int32_t *seq_len;         // [B]
+  int32_t *cur_pos;         // [B]
+  int32_t *err;
+  int64_t cap;
+  int32_t L, Hkv, B, D;
+  int64_t seg_start[TRIA_MAX_BATCH + 1];
+};
+cudaError_t launch_append(const AppendParams &p, cudaStream_t s);
 cudaError_t launch_calibrate(const void *q, int q_dtype, int64_t L, int64_t N, int64_t Hq,
                              int64_t D, int layout, float *centre, float *mean_norm, float *mrl,
                              cudaStream_t s);

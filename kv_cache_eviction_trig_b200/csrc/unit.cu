@@ -359,6 +359,8 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       }
       return;
     }
+    // held back by the prune window: the sequence is left as it is
+    if (p.mode == kModePrune && T < p.prune_from) return;
     if (T == 0) return;
     const int64_t lo = (int64_t)T * r / CL, hi = (int64_t)T * (r + 1) / CL;
     const int n = (int)(hi - lo);

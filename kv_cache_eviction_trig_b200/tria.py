@@ -40,11 +40,12 @@ DEVERR_SEQ_LEN = 1
 DEVERR_SELECTION = 2
 DEVERR_TIMEOUT = 4
 DEVERR_SEGMENT_BIG = 8
+DEVERR_SEGMENT_FULL = 16
 
 EXPORTS = ["tria_workspace_size", "tria_workspace_init", "tria_calibrate", "tria_score",
            "tria_select", "tria_compact", "tria_prune", "tria_prune_profiled",
            "tria_prune_stage_name", "tria_get_device_error", "tria_status_string", "tria_version",
-           "tria_prune_noalloc"]
+           "tria_prune_noalloc", "tria_append"]
 
 
 class TriaError(RuntimeError):
@@ -59,7 +60,7 @@ class tria_config(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("rope_theta", ctypes.c_double),
                 ("rope_layout", ctypes.c_int32), ("budget", ctypes.c_int32),
                 ("offsets", ctypes.POINTER(ctypes.c_int32)), ("n_offsets", ctypes.c_int32),
-                ("flags", ctypes.c_uint32)]
+                ("flags", ctypes.c_uint32), ("prune_window", ctypes.c_int32)]
 
 
 class tria_cache(ctypes.Structure):
@@ -100,6 +101,7 @@ def lib():
                                           ctypes.c_size_t, vp, P(vp), P(ctypes.c_int32)]
         L.tria_prune_noalloc.argtypes = [P(tria_config), P(tria_stats), P(tria_cache), vp, vp,
                                          vp]
+        L.tria_append.argtypes = [P(tria_config), P(tria_cache), vp, vp, vp, ctypes.c_size_t, vp]
         L.tria_prune_stage_name.argtypes = [ctypes.c_int32]
         L.tria_prune_stage_name.restype = ctypes.c_char_p
         L.tria_get_device_error.argtypes = [vp, P(ctypes.c_int32), vp]
@@ -142,18 +144,19 @@ class Config:
 
     def __init__(self, *, num_layers: int, batch: int, n_q_heads: int, n_kv_heads: int,
                  head_dim: int, rope_theta: float, budget: int, offsets: Sequence[int],
-                 rope_layout: int = ROPE_HALF_SPLIT, flags: int = 0):
+                 rope_layout: int = ROPE_HALF_SPLIT, flags: int = 0, prune_window: int = 0):
         self._offsets = (ctypes.c_int32 * max(1, len(offsets)))(*offsets)
         self.c = tria_config(num_layers, batch, n_q_heads, n_kv_heads, head_dim,
                              float(rope_theta), rope_layout, budget,
                              ctypes.cast(self._offsets, ctypes.POINTER(ctypes.c_int32)),
-                             len(offsets), flags)
+                             len(offsets), flags, prune_window)
 
     @classmethod
-    def from_workload(cls, wl, flags: int = 0) -> "Config":
+    def from_workload(cls, wl, flags: int = 0, prune_window: int = 0) -> "Config":
         return cls(num_layers=wl.num_layers, batch=wl.batch, n_q_heads=wl.n_q_heads,
                    n_kv_heads=wl.n_kv_heads, head_dim=wl.head_dim, rope_theta=wl.rope_theta,
-                   budget=wl.budget, offsets=wl.offsets, rope_layout=wl.rope_layout, flags=flags)
+                   budget=wl.budget, offsets=wl.offsets, rope_layout=wl.rope_layout, flags=flags,
+                   prune_window=prune_window)
 
 
 class Cache:
@@ -242,6 +245,13 @@ def tria_prune(cfg: Config, stats: Stats, cache: Cache, ws: torch.Tensor,
                sel_out: Optional[torch.Tensor] = None, stream=None):
     _check(lib().tria_prune(ctypes.byref(cfg.c), ctypes.byref(stats.c), ctypes.byref(cache.c),
                             _ptr(sel_out), _ptr(ws), ws.numel(), _stream(stream)), "tria_prune")
+
+
+def tria_append(cfg: Config, cache: Cache, k_new: torch.Tensor, v_new: torch.Tensor,
+                ws: torch.Tensor, stream=None):
+    """k_new, v_new: bf16 [L][Hkv][B][D] device tensors, one new token per sequence."""
+    _check(lib().tria_append(ctypes.byref(cfg.c), ctypes.byref(cache.c), _ptr(k_new),
+                             _ptr(v_new), _ptr(ws), ws.numel(), _stream(stream)), "tria_append")
 
 
 def tria_prune_profiled(cfg: Config, stats: Stats, cache: Cache, ws: torch.Tensor, events,

@@ -163,5 +163,58 @@ def prune(p: Problem, v: np.ndarray):
             "seq_len": sl}
 
 
+def prune_window(p: Problem, v: np.ndarray, window: int):
+    """Window-based pruning (dimensionstp.github.io review, section 3-2 (5); the
+    romaanj.github.io review, "Method", prunes back to the budget every 128
+    decoded tokens): a sequence is pruned only once its live length reaches
+    budget + max(window, 1); every other sequence keeps its cache as it is.
+    Sequences are independent, so a pruned sequence's result is `prune`'s.
+    -> `prune`'s dict; the sel rows of the sequences held back are -2 (not
+    selected this call)."""
+    out = prune(p, v)
+    thr = p.budget + max(int(window), 1)
+    v0 = np.ascontiguousarray(v, dtype=np.uint16)
+    for b in range(p.B):
+        T = int(p.seq_len[b])
+        if T >= thr or T <= p.budget:
+            continue
+        s0, e0 = int(p.seq_start[b]), int(p.seq_start[b + 1])
+        out["k"][:, :, s0:e0] = p.k[:, :, s0:e0]
+        out["v"][:, :, s0:e0] = v0[:, :, s0:e0]
+        out["pos"][:, :, s0:e0] = p.pos[:, :, s0:e0]
+        out["seq_len"][b] = T
+        out["sel"][:, :, b] = -2
+    return out
+
+
+def append(k: np.ndarray, v: np.ndarray, pos: np.ndarray, seq_start: Sequence[int],
+           seq_len: Sequence[int], cur_pos: Sequence[int], k_new: np.ndarray,
+           v_new: np.ndarray):
+    """One decoded token per sequence joins the cache (romaanj.github.io review,
+    "Background"): in every (layer, KV head) row, slot seq_len[b] of segment b
+    takes the new key and value and the position cur_pos[b] + 1; then seq_len[b]
+    and cur_pos[b] grow by one.  A segment with no free slot, or a length out of
+    range, is left as it is.  k, v: uint16 [L][Hkv][cap][D]; k_new, v_new: uint16
+    [L][Hkv][B][D].  -> copies (k, v, pos, seq_len, cur_pos) and the list of
+    sequences that were skipped."""
+    k, v, pos = k.copy(), v.copy(), pos.copy()
+    seq_len = np.array(seq_len, dtype=np.int32)
+    cur_pos = np.array(cur_pos, dtype=np.int32)
+    skipped = []
+    for b in range(len(seq_len)):
+        T = int(seq_len[b])
+        room = int(seq_start[b + 1]) - int(seq_start[b])
+        if T < 0 or T >= room:
+            skipped.append(b)
+            continue
+        slot = int(seq_start[b]) + T
+        k[:, :, slot] = k_new[:, :, b]
+        v[:, :, slot] = v_new[:, :, b]
+        pos[:, :, slot] = cur_pos[b] + 1
+        seq_len[b] = T + 1
+        cur_pos[b] += 1
+    return k, v, pos, seq_len, cur_pos, skipped
+
+
 def num_threads() -> int:
     return int(lib().orc_num_threads())

@@ -112,6 +112,7 @@ def test_workspace_size(L):
     (dict(rope_layout=2), tria.ERR_INVALID_ARG),
     (dict(flags=4), tria.ERR_INVALID_ARG),
     (dict(batch=300), tria.ERR_UNSUPPORTED),
+    (dict(prune_window=-1), tria.ERR_INVALID_ARG),
 ])
 def test_bad_config_rejected_before_launch(L, mutate, status):
     cfg = _cfg(**mutate)
@@ -148,6 +149,32 @@ def test_select_and_compact_reject_bad_args(L):
     assert L.tria_calibrate(ctypes.byref(cfg.c), ctypes.c_void_p(FAKE), 7, 10,
                             ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE),
                             None) == tria.ERR_INVALID_ARG
+
+
+def test_append_rejects_bad_args(L):
+    cfg, cache = _cfg(), _cache()
+    ws = ctypes.c_void_p(FAKE + 0x1000000)
+    kn, vn = ctypes.c_void_p(FAKE + 0x700000), ctypes.c_void_p(FAKE + 0x800000)
+
+    def app(cfg=cfg, cache=cache, kn=kn, vn=vn, ws=ws, ws_bytes=1 << 40):
+        return L.tria_append(ctypes.byref(cfg.c), ctypes.byref(cache.c), kn, vn, ws, ws_bytes,
+                             None)
+
+    assert app(kn=None) == tria.ERR_INVALID_ARG
+    assert app(vn=ctypes.c_void_p(FAKE + 0x800008)) == tria.ERR_INVALID_ARG  # misaligned
+    assert app(cache=_cache(cur=0)) == tria.ERR_INVALID_ARG                  # no cur_pos
+    assert app(cache=_cache(v=0)) == tria.ERR_INVALID_ARG
+    assert app(cfg=_cfg(prune_window=-5)) == tria.ERR_INVALID_ARG
+    assert app(cfg=_cfg(head_dim=100)) == tria.ERR_UNSUPPORTED               # not a multiple of 8
+    assert app(ws_bytes=1000) == tria.ERR_WORKSPACE
+
+
+def test_config_struct_matches_header():
+    """The binding's tria_config has the header's fields in the header's order."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    body = re.search(r"typedef struct \{(.*?)\} tria_config;", text, flags=re.S).group(1)
+    names = re.findall(r"([a-z_]+)\s*;", body)
+    assert names == [f[0] for f in tria.tria_config._fields_]
 
 
 def test_binding_refuses_host_tensors():

@@ -2,6 +2,7 @@
 (compiled on the CPU into a temporary library) and check that each one makes
 at least one pin fail.  The real oracle is untouched."""
 import ctypes
+import inspect
 import os
 import subprocess
 
@@ -74,4 +75,39 @@ def test_planted_mistake_is_caught(name, tmp_path):
                 caught.append(test.__name__)
     finally:
         oracle._lib = real
+    assert caught, f"no pin caught the planted mistake {name!r}"
+
+
+# Mistakes in the decode-loop steps of the oracle (Python functions of the package).
+PY_MUTANTS = {
+    "window threshold off by one": ("prune_window", "if T >= thr or T <= p.budget:",
+                                    "if T > thr or T <= p.budget:"),
+    "window ignored": ("prune_window", "thr = p.budget + max(int(window), 1)",
+                       "thr = p.budget + 1"),
+    "appended position not advanced": ("append", "pos[:, :, slot] = cur_pos[b] + 1",
+                                       "pos[:, :, slot] = cur_pos[b]"),
+    "append over the newest token": ("append", "slot = int(seq_start[b]) + T",
+                                     "slot = int(seq_start[b]) + max(T - 1, 0)"),
+    "full segment overwritten": ("append", "if T < 0 or T >= room:", "if T < 0 or T > room:"),
+}
+
+PY_PIN_TESTS = [pins.test_prune_window_threshold,
+                pins.test_append_writes_the_next_slot_and_advances,
+                pins.test_decode_loop_lengths_follow_the_window_sawtooth]
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_planted_decode_loop_mistake_is_caught(name, monkeypatch):
+    fn, old, new = PY_MUTANTS[name]
+    src = inspect.getsource(getattr(oracle, fn))
+    assert src.count(old) == 1, f"mutation site for {name!r} not found exactly once"
+    ns = dict(vars(oracle))
+    exec(src.replace(old, new), ns)
+    monkeypatch.setattr(oracle, fn, ns[fn])
+    caught = []
+    for test in PY_PIN_TESTS:
+        try:
+            test()
+        except Exception:  # a failed assertion, or the mutant indexing out of its arrays
+            caught.append(test.__name__)
     assert caught, f"no pin caught the planted mistake {name!r}"

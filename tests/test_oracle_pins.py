@@ -389,3 +389,113 @@ def test_empty_segment_is_a_no_op():
     assert np.all(out["sel"][:, :, 1] == -1)
     s0 = data["seq_start"][1]
     np.testing.assert_array_equal(out["k"][:, :, s0:], p.k[:, :, s0:])
+
+
+# ------------------------------------------------------- decode loop: append + windowed prune
+
+def _decode_problem(seed, seq_lens, slack, budget, B=None):
+    wl = workloads.custom("pin-decode", L=1, B=len(seq_lens), Hq=4, Hkv=2, D=16, theta=1.0e4,
+                          budget=budget, offsets=list(range(1, 9)), seq_lens=seq_lens, seed=seed,
+                          nu=0.5, n_calib=64, slack=slack)
+    data = workloads.generate(wl)
+    stats = common.stats_fp32(data["q_calib"], wl.rope_layout)
+    return wl, data, stats
+
+
+def test_prune_window_of_zero_or_one_is_the_plain_prune():
+    """Window-based pruning (3-2 (5)) with a window of 0 or 1 prunes every
+    sequence longer than the budget: it is the plain prune."""
+    wl, data, stats = _decode_problem(21, [40, 11, 10], 0, 10)
+    p = common.problem(wl, data, stats)
+    v = common.bf16_bits(data["v"])
+    a = oracle.prune(p, v)
+    for w in (0, 1):
+        b = oracle.prune_window(p, v, w)
+        for key in ("k", "v", "pos", "seq_len", "sel"):
+            np.testing.assert_array_equal(a[key], b[key])
+
+
+def test_prune_window_threshold():
+    """A sequence is pruned exactly when its length reaches budget + window: one
+    key short it keeps everything, at the threshold it is pruned as by the plain
+    prune, and a sequence within the budget is untouched either way (3-2 (5))."""
+    budget, W = 10, 6
+    lens = [budget + W - 1, budget + W, budget - 3]
+    wl, data, stats = _decode_problem(22, lens, 0, budget)
+    p = common.problem(wl, data, stats)
+    v = common.bf16_bits(data["v"])
+    full = oracle.prune(p, v)
+    win = oracle.prune_window(p, v, W)
+    assert win["seq_len"].tolist() == [budget + W - 1, budget, budget - 3]
+    st = data["seq_start"]
+    s0, e0 = st[0], st[1]
+    np.testing.assert_array_equal(win["k"][:, :, s0:e0], p.k[:, :, s0:e0])
+    np.testing.assert_array_equal(win["v"][:, :, s0:e0], v[:, :, s0:e0])
+    np.testing.assert_array_equal(win["pos"][:, :, s0:e0], p.pos[:, :, s0:e0])
+    assert np.all(win["sel"][:, :, 0] == -2)
+    for b in (1, 2):
+        s0, e0 = st[b], st[b + 1]
+        for key in ("k", "v", "pos"):
+            np.testing.assert_array_equal(win[key][:, :, s0:e0], full[key][:, :, s0:e0])
+        np.testing.assert_array_equal(win["sel"][:, :, b], full["sel"][:, :, b])
+
+
+def test_append_writes_the_next_slot_and_advances():
+    """A decoded token joins the cache (Background): its rows land in slot
+    seq_len[b] of every segment with position cur_pos[b] + 1, the length and the
+    position advance by one, nothing else changes; a full segment is skipped."""
+    rng = np.random.default_rng(5)
+    L, Hkv, D = 2, 2, 8
+    starts, lens, cur = [0, 5, 9, 12], [2, 3, 3], [100, 7, 50]  # segment 2 is full
+    k = rng.integers(0, 1 << 16, size=(L, Hkv, 12, D), dtype=np.uint16)
+    v = rng.integers(0, 1 << 16, size=(L, Hkv, 12, D), dtype=np.uint16)
+    pos = rng.integers(0, 1000, size=(L, Hkv, 12), dtype=np.int32)
+    kn = rng.integers(0, 1 << 16, size=(L, Hkv, 3, D), dtype=np.uint16)
+    vn = rng.integers(0, 1 << 16, size=(L, Hkv, 3, D), dtype=np.uint16)
+    k2, v2, pos2, sl, cp, skipped = oracle.append(k, v, pos, starts, lens, cur, kn, vn)
+    assert skipped == [2]
+    assert sl.tolist() == [3, 4, 3] and cp.tolist() == [101, 8, 50]
+    changed = np.zeros(12, dtype=bool)
+    for b in (0, 1):
+        slot = starts[b] + lens[b]
+        changed[slot] = True
+        np.testing.assert_array_equal(k2[:, :, slot], kn[:, :, b])
+        np.testing.assert_array_equal(v2[:, :, slot], vn[:, :, b])
+        assert np.all(pos2[:, :, slot] == cur[b] + 1)
+    np.testing.assert_array_equal(k2[:, :, ~changed], k[:, :, ~changed])
+    np.testing.assert_array_equal(v2[:, :, ~changed], v[:, :, ~changed])
+    np.testing.assert_array_equal(pos2[:, :, ~changed], pos[:, :, ~changed])
+
+
+def test_decode_loop_lengths_follow_the_window_sawtooth():
+    """One token appended per step and a windowed prune after each: a sequence
+    grows by one per step until it reaches budget + W, and from then on returns
+    to the budget every W steps (Method: the cache is pruned back to the budget
+    every 128 decoded tokens).  Closed form of the length after step t for a
+    start length s: s + t before the first prune, budget + (s + t - budget) mod W
+    after it."""
+    budget, W, steps = 8, 4, 17
+    starts_len = [5, 11, 3]
+    wl, data, stats = _decode_problem(23, starts_len, budget + W - min(starts_len), budget)
+    rng = np.random.default_rng(9)
+    k, v = common.bf16_bits(data["k"]), common.bf16_bits(data["v"])
+    pos, cur = data["pos"].numpy(), data["cur_pos"].numpy()
+    lens = np.array(starts_len, dtype=np.int32)
+    st = data["seq_start"]
+    for t in range(1, steps + 1):
+        kn = common.bf16_bits(torch.randn(1, 2, 3, 16, dtype=torch.float32).to(torch.bfloat16))
+        vn = rng.integers(0, 1 << 16, size=(1, 2, 3, 16), dtype=np.uint16)
+        k, v, pos, lens, cur, skipped = oracle.append(k, v, pos, st, lens, cur, kn, vn)
+        assert skipped == []
+        c, m, r = stats
+        p = oracle.Problem(k=k, pos=pos, seq_start=st, seq_len=lens, cur_pos=cur,
+                           centre=c.astype(np.float64), mean_norm=m.astype(np.float64),
+                           mrl=r.astype(np.float64), theta=wl.rope_theta, budget=budget,
+                           offsets=wl.offsets, n_q_heads=wl.n_q_heads)
+        out = oracle.prune_window(p, v, W)
+        k, v, pos, lens = out["k"], out["v"], out["pos"], out["seq_len"]
+        for b, s in enumerate(starts_len):
+            want = s + t if s + t < budget + W else budget + (s + t - budget) % W
+            assert lens[b] == want, (t, b, lens[b], want)
+            seg = pos[0, 0, st[b]:st[b] + lens[b]]
+            assert np.all(np.diff(seg) > 0)  # kept positions stay in order

@@ -177,8 +177,8 @@ tria_status tria_prune(const tria_config *cfg, const tria_stats *stats, const tr
                        int32_t *sel_out, void *ws, size_t ws_bytes, void *stream);
 
 /* The decode-loop step before the prune (romaanj.github.io review, "Background":
- * every decoded token is appended to the cache; dimensionstp.github.io review,
- * section 3-2 (5), window-based pruning).  k_new and v_new are DEVICE bf16
+ * the cache grows by one key and value per decoded token; dimensionstp.github.io
+ * review, section 3-2 (5), window-based pruning).  k_new and v_new are DEVICE bf16
  * [L][Hkv][B][D], 16-byte aligned: the new token of every sequence.  For every
  * (layer, KV head, sequence) the token's K and V rows go to slot
  * seq_start[b] + seq_len[b] and its position cur_pos[b] + 1 to pos; then
@@ -191,6 +191,23 @@ tria_status tria_prune(const tria_config *cfg, const tria_stats *stats, const tr
  * used). */
 tria_status tria_append(const tria_config *cfg, const tria_cache *cache, const void *k_new,
                         const void *v_new, void *ws, size_t ws_bytes, void *stream);
+
+/* Decode attention over the pruned cache: the step after the prune in a decode
+ * loop (romaanj.github.io review, "Results": decoding reads the budgeted cache,
+ * which is where the throughput gain comes from; dimensionstp.github.io review,
+ * section 6, Limitations: in serving the pruned cache meets the attention kernel).
+ * The cache stores post-RoPE keys, so positions are not needed.  For layer
+ * `layer`, every sequence b and query head h (KV head h / G):
+ *   out[b][h] = sum_{t < seq_len[b]} softmax_t(scale * q[b][h] . k_t) v_t
+ * over the live slots t of segment b.  q is DEVICE bf16 [B][Hq][D], 16-byte
+ * aligned; out is DEVICE float32 [B][Hq][D]; a sequence with seq_len 0 gets
+ * zeros.  Accumulates in float32 with a running maximum (no overflow for any
+ * finite logits).  A seq_len out of range sets TRIA_DEVERR_SEQ_LEN and that
+ * sequence's rows are not written.  ws as for the other calls (only its error
+ * word is used). */
+tria_status tria_decode_attention(const tria_config *cfg, const tria_cache *cache, int32_t layer,
+                                  const void *q, float scale, float *out, void *ws,
+                                  size_t ws_bytes, void *stream);
 
 /* tria_prune with a cudaEvent_t (as void*) recorded on `stream` before each
  * of its kernels and after the last: events[0..n_stages].  Returns the number

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstring>
 
+#include "attention.cuh"
 #include "tria_internal.cuh"
 
 namespace tria {
@@ -391,6 +392,39 @@ tria_status tria_append(const tria_config *cfg, const tria_cache *cache, const v
   ap.D = cfg->head_dim;
   for (int b = 0; b <= cfg->batch; ++b) ap.seg_start[b] = cache->seq_start[b];
   return cuda_status(launch_append(ap, static_cast<cudaStream_t>(stream)));
+}
+
+tria_status tria_decode_attention(const tria_config *cfg, const tria_cache *cache, int32_t layer,
+                                  const void *q, float scale, float *out, void *ws,
+                                  size_t ws_bytes, void *stream) {
+  tria_status s;
+  if ((s = check_config(cfg, false)) != TRIA_OK) return s;
+  if ((s = check_cache(cfg, cache, true)) != TRIA_OK) return s;
+  if (layer < 0 || layer >= cfg->num_layers) return TRIA_ERR_INVALID_ARG;
+  if (!q || !out || !aligned(q, 16) || !aligned(out, 4)) return TRIA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return TRIA_ERR_INVALID_ARG;
+  if (!attention_supported(cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads))
+    return TRIA_ERR_UNSUPPORTED;
+  if ((s = check_ws(cfg, cache, ws, ws_bytes)) != TRIA_OK) return s;
+  const Ws w{ws_layout(*cfg, cache->seq_start, cache->cap_total), static_cast<uint8_t *>(ws)};
+  AttnParams ap;
+  std::memset(&ap, 0, sizeof ap);
+  ap.q = static_cast<const uint16_t *>(q);
+  ap.k = static_cast<const uint16_t *>(cache->k);
+  ap.v = static_cast<const uint16_t *>(cache->v);
+  ap.seq_len = cache->seq_len;
+  ap.out = out;
+  ap.err = w.err();
+  ap.cap = cache->cap_total;
+  ap.layer = layer;
+  ap.B = cfg->batch;
+  ap.Hkv = cfg->n_kv_heads;
+  ap.Hq = cfg->n_q_heads;
+  ap.G = cfg->n_q_heads / cfg->n_kv_heads;
+  ap.D = cfg->head_dim;
+  ap.scale = scale;
+  for (int b = 0; b <= cfg->batch; ++b) ap.seg_start[b] = cache->seq_start[b];
+  return cuda_status(launch_attention(ap, static_cast<cudaStream_t>(stream)));
 }
 
 tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,

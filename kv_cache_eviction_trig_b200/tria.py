@@ -45,7 +45,7 @@ DEVERR_SEGMENT_FULL = 16
 EXPORTS = ["tria_workspace_size", "tria_workspace_init", "tria_calibrate", "tria_score",
            "tria_select", "tria_compact", "tria_prune", "tria_prune_profiled",
            "tria_prune_stage_name", "tria_get_device_error", "tria_status_string", "tria_version",
-           "tria_prune_noalloc", "tria_append"]
+           "tria_prune_noalloc", "tria_append", "tria_decode_attention"]
 
 
 class TriaError(RuntimeError):
@@ -102,6 +102,8 @@ def lib():
         L.tria_prune_noalloc.argtypes = [P(tria_config), P(tria_stats), P(tria_cache), vp, vp,
                                          vp]
         L.tria_append.argtypes = [P(tria_config), P(tria_cache), vp, vp, vp, ctypes.c_size_t, vp]
+        L.tria_decode_attention.argtypes = [P(tria_config), P(tria_cache), ctypes.c_int32, vp,
+                                            ctypes.c_float, vp, vp, ctypes.c_size_t, vp]
         L.tria_prune_stage_name.argtypes = [ctypes.c_int32]
         L.tria_prune_stage_name.restype = ctypes.c_char_p
         L.tria_get_device_error.argtypes = [vp, P(ctypes.c_int32), vp]
@@ -252,6 +254,18 @@ def tria_append(cfg: Config, cache: Cache, k_new: torch.Tensor, v_new: torch.Ten
     """k_new, v_new: bf16 [L][Hkv][B][D] device tensors, one new token per sequence."""
     _check(lib().tria_append(ctypes.byref(cfg.c), ctypes.byref(cache.c), _ptr(k_new),
                              _ptr(v_new), _ptr(ws), ws.numel(), _stream(stream)), "tria_append")
+
+
+def tria_decode_attention(cfg: Config, cache: Cache, layer: int, q: torch.Tensor,
+                          out: torch.Tensor, ws: torch.Tensor, scale: Optional[float] = None,
+                          stream=None):
+    """q: bf16 [B][Hq][D], out: float32 [B][Hq][D] device tensors; scale defaults
+    to 1/sqrt(D)."""
+    if scale is None:
+        scale = cfg.c.head_dim ** -0.5
+    _check(lib().tria_decode_attention(ctypes.byref(cfg.c), ctypes.byref(cache.c), layer,
+                                       _ptr(q), ctypes.c_float(scale), _ptr(out), _ptr(ws),
+                                       ws.numel(), _stream(stream)), "tria_decode_attention")
 
 
 def tria_prune_profiled(cfg: Config, stats: Stats, cache: Cache, ws: torch.Tensor, events,

@@ -164,10 +164,11 @@ def prune(p: Problem, v: np.ndarray):
 
 
 def prune_window(p: Problem, v: np.ndarray, window: int):
-    """Window-based pruning (dimensionstp.github.io review, section 3-2 (5); the
-    romaanj.github.io review, "Method", prunes back to the budget every 128
-    decoded tokens): a sequence is pruned only once its live length reaches
-    budget + max(window, 1); every other sequence keeps its cache as it is.
+    """Window-based pruning (dimensionstp.github.io review, section 3-2 (5); in the
+    romaanj.github.io review, "Method", a prune round runs once per 128 decoded
+    tokens and cuts the cache to the budget): a sequence is pruned only once its
+    live length reaches budget + max(window, 1); every other sequence keeps its
+    cache as it is.
     Sequences are independent, so a pruned sequence's result is `prune`'s.
     -> `prune`'s dict; the sel rows of the sequences held back are -2 (not
     selected this call)."""
@@ -214,6 +215,39 @@ def append(k: np.ndarray, v: np.ndarray, pos: np.ndarray, seq_start: Sequence[in
         seq_len[b] = T + 1
         cur_pos[b] += 1
     return k, v, pos, seq_len, cur_pos, skipped
+
+
+def decode_attention(k: np.ndarray, v: np.ndarray, seq_start: Sequence[int],
+                     seq_len: Sequence[int], layer: int, q: np.ndarray, scale: float):
+    """Decode attention over the (pruned) cache, the step after the prune
+    (romaanj.github.io review, "Results": decoding reads the budgeted cache).
+    Plain definition in float64: for sequence b and query head h, whose KV head
+    is h // G,
+        out[b, h] = sum_t softmax_t(scale * q[b, h] . k_t) v_t
+    over the live slots t < seq_len[b] of segment b (post-RoPE keys, so positions
+    do not enter).  The softmax subtracts the largest logit first, which leaves
+    its value unchanged.  k, v: uint16 bf16 bits [L][Hkv][cap][D]; q: uint16
+    [B][Hq][D].  -> float64 [B][Hq][D]; zeros for an empty sequence."""
+    def f64(bits):
+        return (np.asarray(bits, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+    B, Hq, D = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    qf = f64(q)
+    out = np.zeros((B, Hq, D))
+    for b in range(B):
+        T = int(seq_len[b])
+        if T == 0:
+            continue
+        s0 = int(seq_start[b])
+        for h in range(Hq):
+            g = h // G
+            K = f64(k[layer, g, s0:s0 + T])
+            V = f64(v[layer, g, s0:s0 + T])
+            logits = scale * (K @ qf[b, h])
+            w = np.exp(logits - logits.max())
+            out[b, h] = (w / w.sum()) @ V
+    return out
 
 
 def num_threads() -> int:

@@ -169,6 +169,25 @@ def test_append_rejects_bad_args(L):
     assert app(ws_bytes=1000) == tria.ERR_WORKSPACE
 
 
+def test_decode_attention_rejects_bad_args(L):
+    cfg, cache = _cfg(), _cache()
+    ws = ctypes.c_void_p(FAKE + 0x1000000)
+    q, out = ctypes.c_void_p(FAKE + 0x700000), ctypes.c_void_p(FAKE + 0x800000)
+
+    def att(cfg=cfg, cache=cache, layer=0, q=q, scale=0.1, out=out, ws_bytes=1 << 40):
+        return L.tria_decode_attention(ctypes.byref(cfg.c), ctypes.byref(cache.c), layer, q,
+                                       ctypes.c_float(scale), out, ws, ws_bytes, None)
+
+    assert att(layer=1) == tria.ERR_INVALID_ARG                    # one layer only
+    assert att(layer=-1) == tria.ERR_INVALID_ARG
+    assert att(q=ctypes.c_void_p(FAKE + 0x700002)) == tria.ERR_INVALID_ARG  # misaligned
+    assert att(out=None) == tria.ERR_INVALID_ARG
+    assert att(scale=float("inf")) == tria.ERR_INVALID_ARG
+    assert att(cache=_cache(v=0)) == tria.ERR_INVALID_ARG
+    assert att(cfg=_cfg(head_dim=96)) == tria.ERR_UNSUPPORTED      # no kernel for D = 96
+    assert att(ws_bytes=1000) == tria.ERR_WORKSPACE
+
+
 def test_config_struct_matches_header():
     """The binding's tria_config has the header's fields in the header's order."""
     text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)

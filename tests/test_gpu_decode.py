@@ -195,3 +195,84 @@ def test_decode_loop_matches_oracle_and_its_cuda_graph():
     for n in ("k", "v", "pos", "seq_len", "cur_pos"):
         assert torch.equal(a.dev[n], b.dev[n]), n
     del graph
+
+
+# --------------------------------------------------- decode attention over the pruned cache
+
+ATT_RTOL = ATT_ATOL = 1e-4  # float32 dot products and weights against float64
+
+
+def _queries(case, layer, gen):
+    """One post-RoPE query per (sequence, query head), drawn like the calibration
+    queries (the head's centre plus noise) and rotated to position cur_pos + 1:
+    bf16 [B][Hq][D] on the device."""
+    wl = case.wl
+    B, Hq, D = wl.batch, wl.n_q_heads, wl.head_dim
+    qc = case.host["q_centre"][layer].double()                       # [Hq, D]
+    noise = torch.randn(B, Hq, D, generator=gen, dtype=torch.float64)
+    pre = qc.unsqueeze(0) + 0.3 * qc.norm(dim=-1).view(1, Hq, 1) / math.sqrt(D) * noise
+    p = (case.host["cur_pos"].to(torch.int64) + 1).view(B, 1).expand(B, Hq)
+    q = workloads._rope_rotate(pre, p, wl.rope_theta, wl.rope_layout).to(torch.bfloat16)
+    return q.contiguous().cuda()
+
+
+def _check_attention(case, layer, q, out, scale):
+    st = _state(case)
+    ref = oracle.decode_attention(st["k"], st["v"], case.host["seq_start"], st["seq_len"], layer,
+                                  common.bf16_bits(q), scale)
+    got = out.double().cpu().numpy()
+    assert np.allclose(got, ref, rtol=ATT_RTOL, atol=ATT_ATOL), float(np.abs(got - ref).max())
+    return ref
+
+
+ATT_CASES = {
+    "d128_g4_ragged": lambda: small("att1", L=2, B=3, seq_lens=[2100, 1, 300]),
+    "d64_g8": lambda: small("att2", D=64, Hq=8, Hkv=1, seq_lens=[515], theta=1e4),
+    "d256_g1": lambda: small("att3", D=256, Hq=4, Hkv=4, seq_lens=[300]),
+    "d128_g16_with_empty": lambda: small("att4", Hq=16, Hkv=1, B=2, seq_lens=[130, 0]),
+    "d64_interleaved_g2": lambda: small("att5", D=64, Hq=4, Hkv=2, seq_lens=[700], theta=1e4,
+                                        rope_layout=workloads.INTERLEAVED),
+}
+
+
+@pytest.mark.parametrize("name", sorted(ATT_CASES))
+def test_decode_attention_matches_oracle(name):
+    case = Case(ATT_CASES[name]())
+    wl = case.wl
+    layer = wl.num_layers - 1
+    q = _queries(case, layer, torch.Generator().manual_seed(5))
+    out = torch.full((wl.batch, wl.n_q_heads, wl.head_dim), float("nan"), device="cuda")
+    tria.tria_decode_attention(case.cfg, case.cache, layer, q, out, case.ws)
+    torch.cuda.synchronize()
+    assert tria.tria_get_device_error(case.ws) == 0
+    ref = _check_attention(case, layer, q, out, wl.head_dim ** -0.5)
+    for b, T in enumerate(case.lens):
+        if T == 0:
+            assert torch.all(out[b] == 0)
+        assert np.abs(ref[b]).max() > 0 or T == 0
+
+
+def test_decode_attention_reads_the_pruned_cache():
+    """Attention after a prune (the pruned cache is what decoding reads), with a
+    scale other than 1/sqrt(D)."""
+    case = Case(small("att-pruned", L=2, B=2, seq_lens=[1000, 333], budget=100, slack=5))
+    tria.tria_prune(case.cfg, case.stats, case.cache, case.ws)
+    q = _queries(case, 1, torch.Generator().manual_seed(6))
+    out = torch.empty((2, case.wl.n_q_heads, case.wl.head_dim), device="cuda")
+    tria.tria_decode_attention(case.cfg, case.cache, 1, q, out, case.ws, scale=0.05)
+    torch.cuda.synchronize()
+    assert tria.tria_get_device_error(case.ws) == 0
+    assert case.dev["seq_len"].cpu().tolist() == [100, 100]
+    _check_attention(case, 1, q, out, 0.05)
+
+
+def test_decode_attention_flags_a_bad_length_and_skips_that_sequence():
+    case = Case(small("att-bad", B=2, seq_lens=[300, 300], budget=50), seq_len=[300, 303])
+    case.cache = tria.Cache.from_data(case.dev)
+    q = _queries(case, 0, torch.Generator().manual_seed(7))
+    out = torch.full((2, case.wl.n_q_heads, case.wl.head_dim), 7.0, device="cuda")
+    tria.tria_decode_attention(case.cfg, case.cache, 0, q, out, case.ws)
+    torch.cuda.synchronize()
+    assert tria.tria_get_device_error(case.ws) & tria.DEVERR_SEQ_LEN
+    assert torch.all(out[1] == 7.0)        # the bad sequence's rows are not written
+    assert not torch.any(out[0] == 7.0)    # the good one's are

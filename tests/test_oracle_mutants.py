@@ -89,11 +89,26 @@ PY_MUTANTS = {
     "append over the newest token": ("append", "slot = int(seq_start[b]) + T",
                                      "slot = int(seq_start[b]) + max(T - 1, 0)"),
     "full segment overwritten": ("append", "if T < 0 or T >= room:", "if T < 0 or T > room:"),
+    "softmax without the max shift": ("decode_attention", "w = np.exp(logits - logits.max())",
+                                      "w = np.exp(logits)"),
+    "KV head by modulo": ("decode_attention", "g = h // G", "g = h % Hkv"),
+    "logit scale ignored": ("decode_attention", "logits = scale * (K @ qf[b, h])",
+                            "logits = K @ qf[b, h]"),
+    "weights not normalised": ("decode_attention", "out[b, h] = (w / w.sum()) @ V",
+                               "out[b, h] = w @ V"),
+    "one key short": ("decode_attention", "K = f64(k[layer, g, s0:s0 + T])",
+                      "K = f64(k[layer, g, s0:s0 + T - 1])"),
 }
 
 PY_PIN_TESTS = [pins.test_prune_window_threshold,
                 pins.test_append_writes_the_next_slot_and_advances,
-                pins.test_decode_loop_lengths_follow_the_window_sawtooth]
+                pins.test_decode_loop_lengths_follow_the_window_sawtooth,
+                pins.test_attention_single_key_returns_its_value,
+                pins.test_attention_two_keys_closed_form,
+                pins.test_attention_equal_keys_average_the_values,
+                pins.test_attention_query_heads_read_their_own_kv_head,
+                pins.test_attention_ignores_slot_order_and_empty_sequences,
+                pins.test_attention_large_logits_pick_the_best_key]
 
 
 @pytest.mark.parametrize("name", sorted(PY_MUTANTS))

@@ -470,8 +470,8 @@ def test_append_writes_the_next_slot_and_advances():
 def test_decode_loop_lengths_follow_the_window_sawtooth():
     """One token appended per step and a windowed prune after each: a sequence
     grows by one per step until it reaches budget + W, and from then on returns
-    to the budget every W steps (Method: the cache is pruned back to the budget
-    every 128 decoded tokens).  Closed form of the length after step t for a
+    to the budget every W steps (Method: one prune round per 128 decoded tokens,
+    with W = 128).  Closed form of the length after step t for a
     start length s: s + t before the first prune, budget + (s + t - budget) mod W
     after it."""
     budget, W, steps = 8, 4, 17
@@ -499,3 +499,89 @@ def test_decode_loop_lengths_follow_the_window_sawtooth():
             assert lens[b] == want, (t, b, lens[b], want)
             seg = pos[0, 0, st[b]:st[b] + lens[b]]
             assert np.all(np.diff(seg) > 0)  # kept positions stay in order
+
+
+# ------------------------------------------------- decode attention over the pruned cache
+
+def _bits(x):
+    """bf16-exact float values -> their bf16 bit patterns"""
+    return (np.asarray(x, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _attn_arrays(rng, L, Hkv, G, D, lens, slack=2):
+    starts = [0]
+    for t in lens:
+        starts.append(starts[-1] + t + slack)
+    cap = starts[-1]
+    k = _bits(rng.integers(-8, 9, size=(L, Hkv, cap, D)) / 4.0)  # exact in bf16
+    v = _bits(rng.integers(-8, 9, size=(L, Hkv, cap, D)) / 4.0)
+    q = _bits(rng.integers(-8, 9, size=(len(lens), Hkv * G, D)) / 8.0)
+    return k, v, q, starts
+
+
+def test_attention_single_key_returns_its_value():
+    """With one live key the softmax weight is 1: the output is that key's value."""
+    rng = np.random.default_rng(31)
+    k, v, q, st = _attn_arrays(rng, 2, 2, 2, 8, [1, 1])
+    out = oracle.decode_attention(k, v, st, [1, 1], 1, q, 0.3)
+    for b in range(2):
+        for h in range(4):
+            np.testing.assert_array_equal(out[b, h], common.bits_to_float(v[1, h // 2, st[b]]))
+
+
+def test_attention_two_keys_closed_form():
+    """Two keys with logits a, b weigh their values by 1/(1+e^(b-a)) and 1/(1+e^(a-b))."""
+    k = _bits(np.array([[[[2, 0, 0, 0], [-1, 0, 0, 0]]]], dtype=np.float32))
+    v = _bits(np.array([[[[1, 0, 0, 0], [0, 1, 0, 0]]]], dtype=np.float32))
+    q = _bits(np.array([[[1, 0, 0, 0]]], dtype=np.float32))
+    out = oracle.decode_attention(k, v, [0, 2], [2], 0, q, 0.5)  # logits 1 and -0.5
+    w0 = 1.0 / (1.0 + math.exp(-1.5))
+    np.testing.assert_allclose(out[0, 0], [w0, 1.0 - w0, 0.0, 0.0], rtol=0, atol=1e-15)
+
+
+def test_attention_equal_keys_average_the_values():
+    """Equal keys get equal weights: the output is the mean of the values."""
+    rng = np.random.default_rng(32)
+    k, v, q, st = _attn_arrays(rng, 1, 1, 2, 8, [7])
+    k[0, 0, :] = k[0, 0, 0]
+    out = oracle.decode_attention(k, v, st, [7], 0, q, 0.7)
+    want = common.bits_to_float(v[0, 0, 0:7]).mean(axis=0)
+    for h in range(2):
+        np.testing.assert_allclose(out[0, h], want, rtol=0, atol=1e-14)
+
+
+def test_attention_query_heads_read_their_own_kv_head():
+    """Query head h attends with KV head h // G: zero values in KV head 1 give zero
+    outputs for its query heads and only for them (GQA grouping)."""
+    rng = np.random.default_rng(33)
+    k, v, q, st = _attn_arrays(rng, 1, 2, 2, 8, [9])
+    v[0, 1] = 0
+    v[0, 0] = _bits(rng.integers(1, 9, size=v[0, 0].shape) / 4.0)  # positive values
+    out = oracle.decode_attention(k, v, st, [9], 0, q, 0.4)
+    assert np.all(out[0, 2:4] == 0) and np.all(out[0, 0:2] > 0)
+
+
+def test_attention_ignores_slot_order_and_empty_sequences():
+    """Permuting the live (key, value) slots leaves the output unchanged; an empty
+    sequence gives zeros."""
+    rng = np.random.default_rng(34)
+    k, v, q, st = _attn_arrays(rng, 1, 2, 2, 8, [11, 0])
+    out = oracle.decode_attention(k, v, st, [11, 0], 0, q, 0.6)
+    perm = rng.permutation(11)
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, 0:11] = k[:, :, perm]
+    v2[:, :, 0:11] = v[:, :, perm]
+    out2 = oracle.decode_attention(k2, v2, st, [11, 0], 0, q, 0.6)
+    np.testing.assert_allclose(out2, out, rtol=0, atol=1e-13)
+    assert np.all(out[1] == 0)
+
+
+def test_attention_large_logits_pick_the_best_key():
+    """With very large logits the softmax is the arg-max: the output is the value of
+    the key most aligned with the query, and stays finite."""
+    k = _bits(np.array([[[[1, 0], [3, 0], [-2, 0]]]], dtype=np.float32))
+    v = _bits(np.array([[[[5, 6], [7, 8], [9, 10]]]], dtype=np.float32))
+    q = _bits(np.array([[[4, 0]]], dtype=np.float32))
+    out = oracle.decode_attention(k, v, [0, 3], [3], 0, q, 1.0e4)
+    assert np.all(np.isfinite(out))
+    np.testing.assert_array_equal(out[0, 0], [7.0, 8.0])

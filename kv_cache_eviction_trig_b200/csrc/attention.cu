@@ -80,7 +80,7 @@ __global__ void __cluster_dims__(kAttnCluster, 1, 1) __launch_bounds__(kAttnThre
       float s[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) s[h] = 0.0f;
-#pragma unroll 4
+#pragma unroll 8
       for (int i = 0; i < D / 8; ++i) {
         const uint4 w = __ldg(kr + i);
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -126,8 +126,19 @@ __global__ void __cluster_dims__(kAttnCluster, 1, 1) __launch_bounds__(kAttnThre
     }
 #pragma unroll
     for (int h = 0; h < G; ++h) acc[h] *= alpha[h];
-    for (int j = kg; j < n; j += KG) {
-      const float vv = bf16_to_f(vb[(size_t)(tile + j) * D + d]);
+    // eight value loads in flight per thread, then their products in key order
+    int j = kg;
+    for (; j + 7 * KG < n; j += 8 * KG) {
+      float vv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) vv[u] = bf16_to_f(__ldg(vb + (size_t)(tile + j + u * KG) * D + d));
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc[h] = fmaf(sc[h][j + u * KG], vv[u], acc[h]);
+    }
+    for (; j < n; j += KG) {
+      const float vv = bf16_to_f(__ldg(vb + (size_t)(tile + j) * D + d));
 #pragma unroll
       for (int h = 0; h < G; ++h) acc[h] = fmaf(sc[h][j], vv, acc[h]);
     }

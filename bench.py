@@ -178,11 +178,101 @@ class OracleSample:
         return time.perf_counter() - t0
 
 
-def _cpu_baseline(wl, seconds_target=12.0):
-    s = OracleSample(wl, seconds_target)
-    dt = s.run()
-    return {"value": s.keys / dt, "unit": UNIT, "cores": s.threads, "kind": "oracle",
-            "sample": f"{s.desc}; {dt:.1f} s wall"}
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _host_problem(wl, host, stats, seq_index, n_keys):
+    """The oracle's problem over layer 0 and sequences [0, seq_index) of the pristine
+    cache held in host memory, keeping the first n_keys keys of each sequence (all of
+    them when n_keys is None); the budget scales with the kept fraction."""
+    import numpy as np
+    from tests import common
+
+    import oracle
+    starts = wl.seq_start
+    lens = [wl.seq_lens[b] if n_keys is None else min(n_keys, wl.seq_lens[b])
+            for b in range(seq_index)]
+    k, v, pos = [], [], []
+    new_starts = [0]
+    for b in range(seq_index):
+        s0 = starts[b]
+        k.append(host["k"][0:1, :, s0:s0 + lens[b]])
+        v.append(host["v"][0:1, :, s0:s0 + lens[b]])
+        pos.append(host["pos"][0:1, :, s0:s0 + lens[b]])
+        new_starts.append(new_starts[-1] + lens[b])
+    import torch
+    kk, vv, pp = (torch.cat(x, dim=2) for x in (k, v, pos))
+    full = n_keys is None or all(wl.seq_lens[b] <= n_keys for b in range(seq_index))
+    budget = wl.budget if full else max(1, wl.budget * lens[0] // wl.seq_lens[0])
+    c, m, r = (x[0:1].double().numpy() for x in stats)
+    prob = oracle.Problem(k=common.bf16_bits(kk), pos=pp.numpy(), seq_start=new_starts,
+                          seq_len=lens, cur_pos=host["cur_pos"][:seq_index].numpy(),
+                          centre=c, mean_norm=m, mrl=r, theta=wl.rope_theta, budget=budget,
+                          offsets=wl.offsets, n_q_heads=wl.n_q_heads, layout=wl.rope_layout)
+    keys = wl.n_kv_heads * sum(t for t in lens if t > budget)
+    return prob, common.bf16_bits(vv), keys, budget, np.sum(lens)
+
+
+def _cpu_baseline(wl, host, stats, seconds_target=12.0):
+    """The oracle as it stands on this host's cores.  All cores: the term-by-term
+    prune over the whole workload when that fits about `seconds_target` (else a
+    labelled, extrapolated sample: layer 0, leading sequences, leading keys); one
+    core: a smaller sample of the same kind, extrapolated; and the oracle's folded
+    scoring path (one weight per head and pair, no per-key trigonometry) on the
+    same sample as the all-cores figure."""
+    import oracle
+    threads = oracle.num_threads()
+    out = {"unit": UNIT, "cores": threads, "kind": "oracle", "cpu_model": _cpu_model()}
+    # cost per key (cosine terms) sets the sample: measured once on a small sample
+    probe, probe_v, probe_keys, _, _ = _host_problem(wl, host, stats, 1, 256)
+    t0 = time.perf_counter()
+    oracle.prune(probe, probe_v)
+    rate = probe_keys / max(time.perf_counter() - t0, 1e-6)
+    want = rate * seconds_target
+    if wl.keys_scored <= want:   # layer 0, every sequence, every key
+        prob, v, keys, _, _ = _host_problem(wl, host, stats, wl.batch, None)
+    else:
+        seqs = max(1, min(wl.batch, int(want // (wl.n_kv_heads * max(wl.seq_lens)))))
+        n = int(max(256, min(max(wl.seq_lens), want // (wl.n_kv_heads * seqs))))
+        prob, v, keys, _, _ = _host_problem(wl, host, stats, seqs, n)
+    full = keys == wl.keys_scored  # the whole workload (one layer, nothing cut)
+    t0 = time.perf_counter()
+    oracle.prune(prob, v)
+    dt = time.perf_counter() - t0
+    out["value"] = keys / dt
+    out["extrapolated"] = not full
+    out["sample"] = ("full workload" if full else
+                     f"extrapolated from layer 0, {prob.B} sequence(s) x {prob.Hkv} KV heads, "
+                     f"first {int(max(prob.seq_len))} keys each, budget {prob.budget}") + \
+        f"; term by term; {dt:.1f} s wall"
+    t0 = time.perf_counter()
+    oracle.prune_folded(prob, v)
+    dtf = time.perf_counter() - t0
+    out["value_folded"] = keys / dtf
+    out["sample_folded"] = "same sample, folded scoring path" + ("" if full else " (extrapolated)")
+    # one core: a smaller sample, about a third of the target time
+    n1 = int(max(128, min(max(wl.seq_lens), rate / threads * seconds_target / 3 / wl.n_kv_heads)))
+    p1, v1, k1, _, _ = _host_problem(wl, host, stats, 1, n1)
+    oracle.set_num_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle.prune(p1, v1)
+        dt1 = time.perf_counter() - t0
+    finally:
+        oracle.set_num_threads(threads)
+    k1 = p1.Hkv * sum(int(t) for t in p1.seq_len if t > p1.budget)
+    out["value_1core"] = k1 / dt1
+    out["sample_1core"] = (f"extrapolated from layer 0, sequence 0 x {p1.Hkv} KV heads, first "
+                           f"{int(p1.seq_len[0])} keys, budget {p1.budget}; {dt1:.1f} s wall")
+    return out
 
 
 def run_reference(args):
@@ -354,7 +444,7 @@ def run_ours(args):
         "gpu_launches": n_stages * args.steps,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = _cpu_baseline(wl)
+        out["cpu_baseline"] = _cpu_baseline(wl, host, [t.cpu() for t in stats.tensors])
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:

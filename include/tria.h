@@ -124,11 +124,18 @@ typedef struct {
 } tria_stats;
 
 /* Bytes of workspace the calls below need for this problem (the largest over
- * all calls).  Only the shapes and cache->seq_start/cap_total are read. */
+ * all calls).  The workspace holds the intermediate results of the steps the
+ * problem statement lists (dimensionstp.github.io review, section 2-1, steps
+ * 1-6: score every cached key, normalise per head, keep the top budget, evict
+ * the rest): folded weights, per-head scores, their sums, selection lists and
+ * the error word.  Only the shapes and cache->seq_start/cap_total are read. */
 tria_status tria_workspace_size(const tria_config *cfg, const tria_cache *cache, size_t *bytes);
 
-/* Clears the workspace's device error word (async on stream).  Call once after
- * allocating a workspace; the word is otherwise sticky across calls. */
+/* Prepares a workspace for the steps of the problem statement (dimensionstp.github.io
+ * review, section 2-1, steps 1-6): clears its device error word and its
+ * synchronisation words (async on stream).  Call once after allocating a
+ * workspace, and again after TRIA_DEVERR_TIMEOUT; the error word is otherwise
+ * sticky across calls. */
 tria_status tria_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
 /* Offline calibration (romaanj.github.io review, "Method"; dimensionstp.github.io
@@ -157,7 +164,10 @@ tria_status tria_score(const tria_config *cfg, const tria_stats *stats, const tr
 tria_status tria_select(const tria_config *cfg, const tria_cache *cache, const float *score,
                         int32_t *sel, void *ws, size_t ws_bytes, void *stream);
 
-/* In-place compaction (eviction).  sel is DEVICE int32 [L][Hkv][B][budget] as
+/* In-place compaction: the eviction that follows the selection
+ * (dimensionstp.github.io review, section 3-2 (5), window pruning drops every
+ * key outside the kept set; romaanj.github.io review, "Method", the cache is cut
+ * back to the budget).  sel is DEVICE int32 [L][Hkv][B][budget] as
  * written by tria_select: strictly ascending slots then -1.  Moves K, V and pos
  * rows sel[j] -> j of each segment and sets seq_len[b] to the number of kept
  * slots (every (layer, KV head) list of a sequence must keep the same count).
@@ -166,7 +176,9 @@ tria_status tria_select(const tria_config *cfg, const tria_cache *cache, const f
 tria_status tria_compact(const tria_config *cfg, const tria_cache *cache, const int32_t *sel,
                          void *ws, size_t ws_bytes, void *stream);
 
-/* The whole prune step in one call: score, z-score + group max, select and
+/* The whole prune step in one call (romaanj.github.io review, "Method";
+ * dimensionstp.github.io review, section 2-1, steps 1-6, and section 3-2
+ * (2)-(6)): score, z-score + group max, select and
  * compact every (layer, KV head, sequence) with seq_len > budget (and
  * seq_len >= budget + cfg->prune_window); other sequences are left untouched.
  * seq_len is read once at the start and rewritten at the end.  If sel_out is
@@ -199,7 +211,8 @@ tria_status tria_append(const tria_config *cfg, const tria_cache *cache, const v
  * The cache stores post-RoPE keys, so positions are not needed.  For layer
  * `layer`, every sequence b and query head h (KV head h / G):
  *   out[b][h] = sum_{t < seq_len[b]} softmax_t(scale * q[b][h] . k_t) v_t
- * over the live slots t of segment b.  q is DEVICE bf16 [B][Hq][D], 16-byte
+ * over the live slots t of segment b; scale <= 0 selects the usual 1/sqrt(D)
+ * (any positive finite scale is used as given).  q is DEVICE bf16 [B][Hq][D], 16-byte
  * aligned; out is DEVICE float32 [B][Hq][D]; a sequence with seq_len 0 gets
  * zeros.  Accumulates in float32 with a running maximum (no overflow for any
  * finite logits).  A seq_len out of range sets TRIA_DEVERR_SEQ_LEN and that
@@ -209,7 +222,9 @@ tria_status tria_decode_attention(const tria_config *cfg, const tria_cache *cach
                                   const void *q, float scale, float *out, void *ws,
                                   size_t ws_bytes, void *stream);
 
-/* tria_prune with a cudaEvent_t (as void*) recorded on `stream` before each
+/* tria_prune (same passages: romaanj.github.io review, "Method";
+ * dimensionstp.github.io review, sections 2-1 and 3-2) with a cudaEvent_t
+ * (as void*) recorded on `stream` before each
  * of its kernels and after the last: events[0..n_stages].  Returns the number
  * of stages in *n_stages (events must hold TRIA_PRUNE_MAX_STAGES + 1).  For
  * per-kernel timing only. */
@@ -219,11 +234,15 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
                                 size_t ws_bytes, void *stream, void *const *events,
                                 int32_t *n_stages);
 
-/* Names of the kernels tria_prune launches, in order, for stage i. */
+/* Names of the kernels tria_prune launches (the steps of the dimensionstp.github.io
+ * review, section 2-1, as this library groups them), in order, for stage i. */
 const char *tria_prune_stage_name(int32_t i);
 
 /* Reads the workspace's device error word into *code (synchronous: waits for
- * `stream`).  Returns TRIA_ERR_DEVICE_FLAG if any bit is set, TRIA_OK otherwise. */
+ * `stream`): the inconsistencies that only the device sees while it runs the
+ * steps of the problem statement (dimensionstp.github.io review, section 2-1,
+ * steps 1-6), such as a sequence length beyond its segment.  Returns
+ * TRIA_ERR_DEVICE_FLAG if any bit is set, TRIA_OK otherwise. */
 tria_status tria_get_device_error(const void *ws, int32_t *code, void *stream);
 
 /* tria_prune for callers that cannot allocate device memory.  This entry point
@@ -232,14 +251,17 @@ tria_status tria_get_device_error(const void *ws, int32_t *code, void *stream);
  * its decode loop (cudaMalloc may fail once its pool owns the memory, and
  * cudaFree waits for the whole device).  Same inputs, outputs and results as
  * tria_prune, but the workspace is a fixed array of TRIA_NOALLOC_SCRATCH_BYTES
- * inside the library's device image, held by every device that loads the
- * library until the process exits; the call allocates nothing.
+ * inside the library's device image; the call allocates nothing.
  *   - Problems whose tria_workspace_size exceeds TRIA_NOALLOC_SCRATCH_BYTES
  *     return TRIA_ERR_UNSUPPORTED before anything is launched (16 MiB holds,
  *     for example, one layer of 32 query heads over 32768 cached slots).
- *   - The first call on a device looks up the array's device address with
- *     cudaGetSymbolAddress (with that device current); make that first call
- *     before any stream capture.
+ *   - CUDA loads the part of the library that holds the array lazily: the
+ *     first call on a device (with that device current) looks up the array's
+ *     address with cudaGetSymbolAddress, which loads it and so reserves its
+ *     TRIA_NOALLOC_SCRATCH_BYTES on that device until the process exits.
+ *     Make that first call at start-up, before reserving the device's memory
+ *     for a pool and before any stream capture; later calls reserve nothing.
+ *     A first call that fails (TRIA_ERR_CUDA) is retried by the next call.
  *   - Every call on a device shares the array.  Each call clears the array's
  *     error word, the only part that must start at zero; calls whose kernels
  *     may overlap on one device (different streams, no ordering) race.
@@ -252,10 +274,12 @@ tria_status tria_prune_noalloc(const tria_config *cfg, const tria_stats *stats,
                                const tria_cache *cache, int32_t *sel_out, int32_t *device_error,
                                void *stream);
 
-/* Human-readable name of a status. */
+/* Human-readable name of a status returned by the calls above (which follow the
+ * dimensionstp.github.io review, section 2-1). */
 const char *tria_status_string(tria_status s);
 
-/* Library version string. */
+/* Version string of this implementation of the prune step (romaanj.github.io
+ * review, "Method"). */
 const char *tria_version(void);
 
 #ifdef __cplusplus

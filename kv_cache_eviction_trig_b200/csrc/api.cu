@@ -422,7 +422,7 @@ tria_status tria_decode_attention(const tria_config *cfg, const tria_cache *cach
   ap.Hq = cfg->n_q_heads;
   ap.G = cfg->n_q_heads / cfg->n_kv_heads;
   ap.D = cfg->head_dim;
-  ap.scale = scale;
+  ap.scale = scale > 0.0f ? scale : 1.0f / std::sqrt((float)cfg->head_dim);
   for (int b = 0; b <= cfg->batch; ++b) ap.seg_start[b] = cache->seq_start[b];
   return cuda_status(launch_attention(ap, static_cast<cudaStream_t>(stream)));
 }

@@ -10,14 +10,21 @@
 // outputs; the intermediate buffers (folded phasors, per-head raw scores,
 // per-tile partial sums, selection lists, error word) live in the array below.
 //
-// The array is a file-scope device variable, so every device that loads the
-// library holds TRIA_NOALLOC_SCRATCH_BYTES of it until the process exits.  In
-// host code its name only identifies the variable; the device address comes
-// from cudaGetSymbolAddress, called once per device (with that device current)
-// by the first call made on it.  Every call on a device shares the array and
-// finds the previous call's contents there: the call clears the error word,
-// the only part that must start at zero; everything else is written before it
-// is read.  Two calls whose kernels overlap on a device race on the array.
+// The array is a file-scope device variable.  The library is compiled one
+// translation unit per device module, and CUDA loads a module lazily, on first
+// use: the array's device memory is therefore reserved by the first call on
+// each device (the cudaGetSymbolAddress below loads the module), and every
+// device that has made a call holds TRIA_NOALLOC_SCRATCH_BYTES of it until the
+// process exits.  A caller that reserves all of a device's memory up front must
+// make one call on that device before doing so (and before any stream capture);
+// after that first call nothing is ever allocated again.  In host code the
+// array's name only identifies the variable; its device address comes from
+// cudaGetSymbolAddress, called with the device current.  Only a successful
+// lookup is kept: a failed one (for example under memory pressure) is retried
+// by the next call.  Every call on a device shares the array and finds the
+// previous call's contents there: the call clears the error word, the only
+// part that must start at zero; everything else is written before it is read.  Two calls whose kernels overlap on a
+// device race on the array.
 #include <cstdint>
 #include <mutex>
 
@@ -31,25 +38,24 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[TRIA_NOALLOC_SCRATCH_
 
 constexpr int kMaxDevices = 64;
 
-struct ScratchSlot {
-  std::once_flag once;
-  void *ptr = nullptr;
-  cudaError_t status = cudaSuccess;
-};
+std::mutex g_lock;
+void *g_ptr[kMaxDevices] = {};
 
-ScratchSlot g_slots[kMaxDevices];
-
-// Device address of the scratch array on the current device (nullptr on failure).
+// Device address of the scratch array on the current device (nullptr on failure;
+// the next call tries again).
 void *scratch_on_current_device() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  ScratchSlot &slot = g_slots[dev];
-  std::call_once(slot.once, [&slot]() {
+  std::lock_guard<std::mutex> hold(g_lock);
+  if (!g_ptr[dev]) {
     void *p = nullptr;
-    slot.status = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    slot.ptr = slot.status == cudaSuccess ? p : nullptr;
-  });
-  return slot.ptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess) {
+      g_ptr[dev] = p;
+    } else {
+      (void)cudaGetLastError();  // leave no sticky error for the caller's next CUDA call
+    }
+  }
+  return g_ptr[dev];
 }
 
 }  // namespace

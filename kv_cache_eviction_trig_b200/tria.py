@@ -13,9 +13,7 @@ from typing import Optional, Sequence
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-# TRIA_LIB may name another build of the same library (for example one built with
-# different tuning constants); by default the in-tree build is loaded.
-LIB_PATH = os.environ.get("TRIA_LIB") or os.path.join(_HERE, "libtria.so")
+LIB_PATH = os.path.join(_HERE, "libtria.so")
 
 OK = 0
 ERR_INVALID_ARG = 1
@@ -259,10 +257,10 @@ def tria_append(cfg: Config, cache: Cache, k_new: torch.Tensor, v_new: torch.Ten
 def tria_decode_attention(cfg: Config, cache: Cache, layer: int, q: torch.Tensor,
                           out: torch.Tensor, ws: torch.Tensor, scale: Optional[float] = None,
                           stream=None):
-    """q: bf16 [B][Hq][D], out: float32 [B][Hq][D] device tensors; scale defaults
-    to 1/sqrt(D)."""
+    """q: bf16 [B][Hq][D], out: float32 [B][Hq][D] device tensors; scale None (or
+    <= 0) lets the library use 1/sqrt(D)."""
     if scale is None:
-        scale = cfg.c.head_dim ** -0.5
+        scale = 0.0
     _check(lib().tria_decode_attention(ctypes.byref(cfg.c), ctypes.byref(cache.c), layer,
                                        _ptr(q), ctypes.c_float(scale), _ptr(out), _ptr(ws),
                                        ws.numel(), _stream(stream)), "tria_decode_attention")

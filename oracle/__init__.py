@@ -36,6 +36,8 @@ def lib():
                                        ctypes.c_int32, ctypes.c_int64]
         _lib.orc_key_score.restype = ctypes.c_double
         _lib.orc_raw_scores.argtypes = [ctypes.c_void_p, P(ctypes.c_double)]
+        _lib.orc_raw_scores_folded.argtypes = [ctypes.c_void_p, P(ctypes.c_double)]
+        _lib.orc_set_num_threads.argtypes = [ctypes.c_int32]
         _lib.orc_zmax.argtypes = [ctypes.c_void_p, P(ctypes.c_double), P(ctypes.c_double),
                                   P(ctypes.c_double)]
         _lib.orc_select.argtypes = [ctypes.c_void_p, P(ctypes.c_double), P(ctypes.c_int32)]
@@ -121,6 +123,28 @@ def raw_scores(p: Problem) -> np.ndarray:
     raw = np.full((p.L, p.Hq, p.cap), np.nan)
     lib().orc_raw_scores(p.ref, _ptr(raw, ctypes.c_double))
     return raw
+
+
+def raw_scores_folded(p: Problem) -> np.ndarray:
+    """raw_scores through the angle-addition fold (one weight per head and pair,
+    then one pass per key); pinned to raw_scores, timed as a CPU baseline."""
+    raw = np.full((p.L, p.Hq, p.cap), np.nan)
+    lib().orc_raw_scores_folded(p.ref, _ptr(raw, ctypes.c_double))
+    return raw
+
+
+def prune_folded(p: Problem, v: np.ndarray):
+    """prune with the folded raw scores."""
+    raw = raw_scores_folded(p)
+    z, score = zmax(p, raw)
+    sel = select(p, score)
+    k2, v2, pos2, sl = compact(p, sel, v)
+    return {"raw": raw, "z": z, "score": score, "sel": sel, "k": k2, "v": v2, "pos": pos2,
+            "seq_len": sl}
+
+
+def set_num_threads(n: int):
+    lib().orc_set_num_threads(int(n))
 
 
 def zmax(p: Problem, raw: np.ndarray):

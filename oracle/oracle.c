@@ -163,17 +163,94 @@ double orc_key_score(const orc_problem *p, int32_t l, int32_t h, int32_t b, int6
 }
 
 /* Raw scores of every key of every segment: raw is [L][Hq][cap]; slots outside
- * the live part of a segment are left untouched. */
+ * the live part of a segment are left untouched.  Each key is scored on its
+ * own; the work is shared out over (layer, head, sequence, block of 256 keys). */
 void orc_raw_scores(const orc_problem *p, double *raw) {
+  const int64_t blk = 256;
+  int64_t most = 0;
+  for (int32_t b = 0; b < p->B; ++b)
+    if (p->seq_len[b] > most) most = p->seq_len[b];
+  const int64_t nblk = (most + blk - 1) / blk;
+  const int64_t units = (int64_t)p->L * p->Hq * p->B;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t w = 0; w < units * nblk; ++w) {
+    const int64_t u = w / nblk, kb = w % nblk;
+    const int32_t b = (int32_t)(u % p->B);
+    const int32_t h = (int32_t)((u / p->B) % p->Hq);
+    const int32_t l = (int32_t)(u / ((int64_t)p->B * p->Hq));
+    double *out = raw + ((int64_t)l * p->Hq + h) * p->cap + p->seq_start[b];
+    const int64_t t1 = (kb + 1) * blk < p->seq_len[b] ? (kb + 1) * blk : p->seq_len[b];
+    for (int64_t t = kb * blk; t < t1; ++t) out[t] = orc_key_score(p, l, h, b, t);
+  }
+}
+
+/*
+ * The same raw scores through the angle-addition fold [R1 Method; R2 2-2]: the
+ * key's position cancels between un-rotating the key and the query-key distance,
+ * so with ktilde_f the stored (post-RoPE) pair,
+ *   S_trig = Re sum_f conj(ktilde_f) * W_f,
+ *   W_f    = c_f * (1/|O|) sum_{delta in O} e^{i w_f (cur + delta)},
+ * and |k_f| = |ktilde_f| in the norm term.  One weight per (head, pair) per
+ * sequence, then one pass over each key.  This is not a second reference for the
+ * scores: tests pin it to orc_key_score, and the benchmark times it as the CPU
+ * baseline that does the same arithmetic per key as the GPU path.
+ */
+void orc_raw_scores_folded(const orc_problem *p, double *raw) {
+  const int32_t D = p->D, F = D / 2, G = p->Hq / p->Hkv;
   const int64_t units = (int64_t)p->L * p->Hq * p->B;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t u = 0; u < units; ++u) {
     const int32_t b = (int32_t)(u % p->B);
     const int32_t h = (int32_t)((u / p->B) % p->Hq);
     const int32_t l = (int32_t)(u / ((int64_t)p->B * p->Hq));
+    const int32_t g = h / G;
+    double *wx = (double *)malloc(sizeof(double) * (size_t)F * 3);
+    double *wy = wx + F, *wn = wx + 2 * F;
+    for (int32_t f = 0; f < F; ++f) {
+      const double w = rope_freq(p->theta, D, f);
+      double er = 0.0, ei = 0.0;
+      if (!(p->flags & ORC_NO_TRIG)) {
+        for (int32_t j = 0; j < p->n_offsets; ++j) {
+          const double a = w * ((double)p->cur_pos[b] + (double)p->offsets[j]);
+          er += cos(a);
+          ei += sin(a);
+        }
+        er /= (double)p->n_offsets;
+        ei /= (double)p->n_offsets;
+      }
+      const int64_t o = ((int64_t)l * p->Hq + h) * F + f;
+      const double *cf = p->centre + 2 * o; /* (re, im) of c_f */
+      wx[f] = cf[0] * er - cf[1] * ei;      /* W_f = c_f * e */
+      wy[f] = cf[0] * ei + cf[1] * er;
+      /* norm weight: E|q_f| less the part that the trig term carries, R_f E|q_f| */
+      wn[f] = (p->flags & ORC_NO_CONC_WEIGHT) ? p->mean_norm[o]
+                                              : p->mean_norm[o] - p->mrl[o] * p->mean_norm[o];
+    }
+    const int64_t row = ((int64_t)l * p->Hkv + g) * p->cap + p->seq_start[b];
     double *out = raw + ((int64_t)l * p->Hq + h) * p->cap + p->seq_start[b];
-    for (int64_t t = 0; t < p->seq_len[b]; ++t) out[t] = orc_key_score(p, l, h, b, t);
+    for (int64_t t = 0; t < p->seq_len[b]; ++t) {
+      const uint16_t *k = p->k + (row + t) * D;
+      double s = 0.0;
+      for (int32_t f = 0; f < F; ++f) {
+        int32_t xi, yi;
+        pair_index(D, p->layout, f, &xi, &yi);
+        const double x = bf16_to_double(k[xi]), y = bf16_to_double(k[yi]);
+        /* Re(conj(x + iy) * (wx + i wy)) = x wx + y wy */
+        s += x * wx[f] + y * wy[f] + wn[f] * hypot(x, y);
+      }
+      out[t] = s;
+    }
+    free(wx);
   }
+}
+
+/* Sets the number of threads the oracle's parallel loops use (>= 1). */
+void orc_set_num_threads(int32_t n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
 }
 
 /*

@@ -211,3 +211,30 @@ def test_product_path_has_no_oracle_or_fallback():
         if fn.endswith(".py"):
             src = open(os.path.join(pkg, fn)).read()
             assert "import oracle" not in src and "from oracle" not in src, fn
+
+
+def test_every_declaration_cites_its_passage():
+    """Each entry point in tria.h is preceded by a comment that cites the passage
+    of the pages it follows (a review's page and section), or says that the
+    paper has no counterpart."""
+    text = open(HEADER).read()
+    cite = re.compile(r"(romaanj|dimensionstp)\.github\.io[\s*]+review|no[\s*]+counterpart[\s*]+in[\s*]+the[\s*]+paper")
+    for name in declared_functions():
+        m = re.search(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*" + name + r"\s*\(", text, flags=re.M)
+        assert m, name
+        before = text[:m.start()]
+        # the last comment block before the declaration (#define lines may sit between)
+        end = before.rfind("*/")
+        start = before.rfind("/*", 0, end)
+        between = before[end + 2:]
+        assert all(line.strip() == "" or line.strip().startswith("#define")
+                   for line in between.splitlines()), name
+        assert cite.search(before[start:end]), f"{name}: no passage cited"
+
+
+def test_attention_scale_default_lives_in_the_library():
+    """tria.py passes scale 0 when none is given; the C call picks 1/sqrt(D)."""
+    import inspect
+    src = inspect.getsource(tria.tria_decode_attention).split('"""')[-1]  # code, not docstring
+    assert "sqrt" not in src and "** -0.5" not in src and "head_dim" not in src
+    assert "TRIA_LIB" not in open(tria.__file__).read()

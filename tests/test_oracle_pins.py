@@ -585,3 +585,24 @@ def test_attention_large_logits_pick_the_best_key():
     out = oracle.decode_attention(k, v, [0, 3], [3], 0, q, 1.0e4)
     assert np.all(np.isfinite(out))
     np.testing.assert_array_equal(out[0, 0], [7.0, 8.0])
+
+
+@pytest.mark.parametrize("layout,offsets,flags", [
+    (0, range(1, 33), 0), (1, [2 ** i for i in range(17)], 0), (0, [3, 1, 200, 7], 0),
+    (0, range(1, 9), oracle.NO_TRIG), (1, range(1, 9), oracle.NO_CONC_WEIGHT)])
+def test_folded_scores_equal_term_by_term(layout, offsets, flags):
+    """The folded CPU path (one weight per head and pair, no per-key trigonometry)
+    equals the term-by-term scores: the key position cancels (2-1; 2-2), the offset
+    mean factors out of the sum (Method).  Checked on ragged sequences with
+    positions far from 0, both layouts, the pages' geometric offsets and both
+    ablation flags."""
+    wl, data, stats = _small(seed=21, D=16, B=2, seq_lens=[40, 23], offsets=offsets,
+                             layout=layout, theta=1.0e6)
+    data["pos"] = data["pos"] + 50000
+    data["cur_pos"] = data["cur_pos"] + 50000
+    p = common.problem(wl, data, stats, flags=flags)
+    a, b = oracle.raw_scores(p), oracle.raw_scores_folded(p)
+    live = ~np.isnan(a)
+    assert np.array_equal(live, ~np.isnan(b))
+    scale = np.abs(a[live]).max()
+    np.testing.assert_allclose(b[live], a[live], rtol=0, atol=1e-10 * scale)

@@ -146,3 +146,26 @@ def test_prune_noalloc_rejects_problems_beyond_its_scratch():
     bad_cfg = tria.Config(num_layers=0, batch=2, n_q_heads=8, n_kv_heads=2, head_dim=128,
                           rope_theta=1e6, budget=64, offsets=[1])
     assert call(bad_cfg, small, 2000) == tria.ERR_INVALID_ARG
+
+
+@pytest.mark.gpu
+def test_prune_noalloc_second_call_reserves_no_device_memory():
+    """The scratch array is loaded by the first call on a device; after that a call
+    takes no device memory: free memory is the same before and after it."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from kv_cache_eviction_trig_b200 import build
+    build.build()
+    pair = Pair(_small("noalloc-memory"))
+    sel = pair.sel()
+    err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    tria.tria_prune_noalloc(pair.cfg, pair.stats, pair.caches[1], sel_out=sel, device_error=err)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        tria.tria_prune_noalloc(pair.cfg, pair.stats, pair.caches[1], sel_out=sel,
+                                device_error=err)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert int(err.item()) == 0
+    assert free1 == free0

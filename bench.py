@@ -51,28 +51,6 @@ def _peaks():
         return 6650.0, "fallback"
 
 
-def _score_source_hash():
-    h = hashlib.sha256()
-    for name in ("score.cu", "tria_internal.cuh"):
-        with open(os.path.join(ROOT, "kv_cache_eviction_trig_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
-    return h.hexdigest()[:16]
-
-
-def _traffic_per_launch(workload_index):
-    """DRAM bytes per score-kernel launch from the committed ncu summary, or None
-    if there is none for this workload or the kernel source changed since."""
-    try:
-        with open(TRAFFIC) as f:
-            t = json.load(f)
-        e = t.get(str(workload_index))
-        if e and e.get("source_hash") == _score_source_hash():
-            return float(e["dram_bytes_per_launch"])
-    except Exception:
-        pass
-    return None
-
-
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -301,6 +279,144 @@ def run_reference(args):
     }), flush=True)
 
 
+# Flops per key of the scoring arithmetic: per RoPE pair and query head two FMAs of
+# the trigonometric term and one of the norm term (2 flops each), per pair |k|^2
+# (3 flops) and its square root (1): F * (6 G + 4) = 3 G D + 2 D.
+def flops_per_key(wl):
+    return (wl.head_dim // 2) * (6 * wl.group + 4)
+
+
+def fp32_peak_tflops(sm_mhz):
+    """FP32 peak of a B200 at the given SM clock: 148 SMs x 128 FP32 lanes x 2 flops
+    (one FMA) per lane per clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def _kernel_hash(names):
+    h = hashlib.sha256()
+    for name in names:
+        with open(os.path.join(ROOT, "kv_cache_eviction_trig_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {"prune_kernel": ("prune.cu", "score_math.cuh", "tria_internal.cuh"),
+                  "score_kernel": ("score.cu", "tria_internal.cuh")}
+
+
+def _traffic(kernel, key):
+    """DRAM bytes per launch of `kernel` on workload `key` from the committed ncu
+    summary, or None if there is none or the kernel source changed since."""
+    try:
+        with open(TRAFFIC) as f:
+            t = json.load(f)
+        e = t.get(f"{kernel}:{key}")
+        if e and e.get("source_hash") == _kernel_hash(KERNEL_SOURCES[kernel]):
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class Bench:
+    """One workload resident on the device, ready to be pruned again and again:
+    before every step the rows a prune overwrites are restored from a pristine
+    copy and L2 is flushed (512 MiB written); neither is timed."""
+
+    def __init__(self, wl, dev):
+        self.wl, self.dev = wl, dev
+        data = workloads.generate(wl, device=dev)
+        self.cfg = tria.Config.from_workload(wl)
+        self.stats = tria.calibrate(self.cfg, data["q_calib"])
+        del data["q_calib"]
+        self.data = data
+        self.cache = tria.Cache.from_data(data)
+        self.ws = tria.workspace(self.cfg, self.cache)
+        starts, budget = data["seq_start"], wl.budget
+        # rows a prune overwrites: [seg, seg + budget) of each sequence longer than budget
+        self.restore = [(starts[b], budget) for b in range(wl.batch) if wl.seq_lens[b] > budget]
+        self.backup = {n: [data[n][:, :, s:s + c].clone() for s, c in self.restore]
+                       for n in ("k", "v", "pos")}
+        self.seq_len0 = data["seq_len"].clone()
+        self.flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        self.stream = torch.cuda.current_stream()
+
+    def reset(self):
+        for n in ("k", "v", "pos"):
+            for (s, c), t in zip(self.restore, self.backup[n]):
+                self.data[n][:, :, s:s + c].copy_(t)
+        self.data["seq_len"].copy_(self.seq_len0)
+        self.flush.fill_(1)
+
+    def prune(self):
+        tria.tria_prune(self.cfg, self.stats, self.cache, self.ws, stream=self.stream)
+
+    def warm(self, n):
+        for _ in range(n):
+            self.reset()
+            self.prune()
+        torch.cuda.synchronize()
+        if tria.tria_get_device_error(self.ws) != 0:
+            raise RuntimeError(f"device error flag set on {self.wl.name}")
+        want = [min(t, self.wl.budget) for t in self.wl.seq_lens]
+        if self.data["seq_len"].tolist() != want:
+            raise RuntimeError(f"pruned lengths differ on {self.wl.name}")
+
+    def timed(self, steps):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for i in range(steps):
+            self.reset()
+            ev[i][0].record(self.stream)
+            self.prune()
+            ev[i][1].record(self.stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    def kernels(self, steps):
+        """Per-kernel event times (a separate pass: events between the prune's kernels)."""
+        nst = tria.PRUNE_MAX_STAGES + 1
+        kev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(steps)]
+        names = []
+        for i in range(steps):
+            self.reset()
+            names = tria.tria_prune_profiled(self.cfg, self.stats, self.cache, self.ws, kev[i],
+                                             stream=self.stream)
+        torch.cuda.synchronize()
+        per = [[kev[i][s].elapsed_time(kev[i][s + 1]) for s in range(len(names))]
+               for i in range(steps)]
+        return names, [statistics.mean(k[s] for k in per) for s in range(len(names))]
+
+    def summary(self, step_ms, names, kern_ms, peak, sm_mhz):
+        """Throughput and roofline figures of one workload (device-timed)."""
+        wl = self.wl
+        step = statistics.mean(step_ms)
+        keys = wl.keys_scored
+        algo = wl.algorithmic_bytes()
+        out = {"workload": wl.name, "value": keys / (step / 1e3), "unit": UNIT,
+               "ms_per_step": step, "us_per_layer": step * 1e3 / wl.num_layers,
+               "hbm_gbs_path": algo / (step / 1e3) / 1e9,
+               "frac_path": algo / (step / 1e3) / 1e9 / peak,
+               "kernel_ms": dict(zip(names, kern_ms))}
+        if "prune_kernel" in names:
+            kt = kern_ms[names.index("prune_kernel")]
+            out["prune_kernel_frac"] = algo / (kt / 1e3) / 1e9 / peak
+            busy_ms = kt
+        else:
+            kt = kern_ms[names.index("score_kernel")]
+            out["score_kernel_frac"] = keys * 2 * wl.head_dim / (kt / 1e3) / 1e9 / peak
+            busy_ms = kt
+        tflops = keys * flops_per_key(wl) / (busy_ms / 1e3) / 1e12
+        out["fp32_tflops"] = tflops
+        if sm_mhz:
+            out["frac_fp32"] = tflops / fp32_peak_tflops(sm_mhz)
+        return out
+
+    def free(self):
+        del self.data, self.cache, self.ws, self.backup, self.flush, self.stats
+        torch.cuda.empty_cache()
+
+
 def run_ours(args):
     rank, world, local = _rank_env()
     torch.cuda.set_device(local)
@@ -309,99 +425,48 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
     wl = rank_workload(args.workload, rank)
-
-    data = workloads.generate(wl, device=dev)
-    cfg = tria.Config.from_workload(wl)
-    stats = tria.calibrate(cfg, data["q_calib"])
-    del data["q_calib"]
-    cache = tria.Cache.from_data(data)
-    ws = tria.workspace(cfg, cache)
-    B, budget = wl.batch, wl.budget
-    starts = data["seq_start"]
-    # rows a prune overwrites: [seg, seg + budget) of each sequence longer than budget
-    restore = [(starts[b], budget) for b in range(B) if wl.seq_lens[b] > budget]
-    backup = {n: [data[n][:, :, s:s + c].clone() for s, c in restore] for n in ("k", "v", "pos")}
-    seq_len0 = data["seq_len"].clone()
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-
-    def reset():
-        for n in ("k", "v", "pos"):
-            for (s, c), t in zip(restore, backup[n]):
-                data[n][:, :, s:s + c].copy_(t)
-        data["seq_len"].copy_(seq_len0)
-        flush.fill_(1)
-
-    stream = torch.cuda.current_stream()
-    sel = torch.empty(wl.num_layers, wl.n_kv_heads, B, budget, dtype=torch.int32, device=dev)
-
-    # ---- warm-up and a correctness guard (the pruned lengths)
-    for _ in range(args.warmup):
-        reset()
-        tria.tria_prune(cfg, stats, cache, ws, stream=stream)
-    torch.cuda.synchronize()
-    if tria.tria_get_device_error(ws) != 0:
-        raise RuntimeError("device error flag set during warm-up")
-    assert data["seq_len"].tolist() == [min(t, budget) for t in wl.seq_lens]
+    peak, peak_kind = _peaks()
+    bench = Bench(wl, dev)
+    bench.warm(args.warmup)
 
     # ---- timed region: K steps, each bracketed by events on the launching stream
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        for i in range(args.steps):
-            reset()
-            ev[i][0].record(stream)
-            tria.tria_prune(cfg, stats, cache, ws, stream=stream)
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
+        step_ms = bench.timed(args.steps)
     if world > 1:
         dist.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
     clocks = clk.summary()
-
-    # ---- per-kernel times (separate pass: events between the prune's kernels)
-    nst = tria.PRUNE_MAX_STAGES + 1
-    kern_ms = None
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
-    n_stages = 0
-    for i in range(args.steps):
-        reset()
-        n_stages = tria.tria_prune_profiled(cfg, stats, cache, ws, kev[i], stream=stream)
-    torch.cuda.synchronize()
-    kern_ms = [[kev[i][s].elapsed_time(kev[i][s + 1]) for s in range(n_stages)]
-               for i in range(args.steps)]
-    avg_kern = [statistics.mean(k[s] for k in kern_ms) for s in range(n_stages)]
-    names = [tria.tria_prune_stage_name(s) for s in range(n_stages)]
+    sm_mhz = clocks["sm_mhz"] if clocks else None
+    names, kern_ms = bench.kernels(args.steps)
 
     # ---- end to end through the C ABI with host buffers (pinned), copies timed
+    data, restore, backup = bench.data, bench.restore, bench.backup
     host = {n: data[n].cpu().pin_memory() for n in ("k", "v", "pos", "seq_len", "cur_pos")}
-    for (s, c), t in zip(restore, backup["k"]):
-        host["k"][:, :, s:s + c].copy_(t.cpu())
-    for (s, c), t in zip(restore, backup["v"]):
-        host["v"][:, :, s:s + c].copy_(t.cpu())
-    for (s, c), t in zip(restore, backup["pos"]):
-        host["pos"][:, :, s:s + c].copy_(t.cpu())
-    host["seq_len"].copy_(seq_len0.cpu())
+    for n in ("k", "v", "pos"):
+        for (s, c), t in zip(restore, backup[n]):
+            host[n][:, :, s:s + c].copy_(t.cpu())
+    host["seq_len"].copy_(bench.seq_len0.cpu())
+    budget = wl.budget
     out_k = torch.empty(wl.num_layers, wl.n_kv_heads, len(restore), budget, wl.head_dim,
                         dtype=torch.bfloat16).pin_memory()
     out_v = torch.empty_like(out_k).pin_memory()
     out_p = torch.empty(wl.num_layers, wl.n_kv_heads, len(restore), budget,
                         dtype=torch.int32).pin_memory()
-    out_len = torch.empty(B, dtype=torch.int32).pin_memory()
+    out_len = torch.empty(wl.batch, dtype=torch.int32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in (out_k, out_v, out_p, out_len))
     e2e_steps = max(3, min(args.steps, 20))
     eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(e2e_steps)]
+    stream = bench.stream
     for i in range(e2e_steps):
-        flush.fill_(1)
+        bench.flush.fill_(1)
         eev[i][0].record(stream)
         for n in ("k", "v", "pos", "seq_len", "cur_pos"):
             data[n].copy_(host[n], non_blocking=True)
-        tria.tria_prune(cfg, stats, cache, ws, stream=stream)
+        bench.prune()
         for j, (s, c) in enumerate(restore):
             out_k[:, :, j].copy_(data["k"][:, :, s:s + c], non_blocking=True)
             out_v[:, :, j].copy_(data["v"][:, :, s:s + c], non_blocking=True)
@@ -410,41 +475,87 @@ def run_ours(args):
         eev[i][1].record(stream)
     torch.cuda.synchronize()
     e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in eev)
+    if tria.tria_get_device_error(bench.ws) != 0:
+        raise RuntimeError("device error flag set during the timed runs")
 
-    red = max_over_ranks([total_ms, e2e_ms] + avg_kern, device=dev)
-    total_ms, e2e_ms, avg_kern = red[0], red[1], red[2:]
-
-    keys = wl.keys_scored
-    value = keys * world / (total_ms / 1e3 / args.steps)
+    total_ms = sum(step_ms)
+    red = max_over_ranks([total_ms, e2e_ms] + kern_ms, device=dev)
+    total_ms, e2e_ms, kern_ms = red[0], red[1], red[2:]
     step = total_ms / args.steps
-    peak, peak_kind = _peaks()
-    score_i = names.index("score_kernel")
-    score_bytes = keys * 2 * wl.head_dim        # K read once (positions are not needed)
-    achieved = score_bytes / (avg_kern[score_i] / 1e3) / 1e9
-    traffic = _traffic_per_launch(args.workload)
-    dom = max(range(n_stages), key=lambda s: avg_kern[s])
+    head = bench.summary([step], names, kern_ms, peak, sm_mhz)
+    keys = wl.keys_scored
+    dom = max(range(len(names)), key=lambda s: kern_ms[s])
+    kern = names[dom]
+    if kern == "prune_kernel":
+        algo_launch = wl.algorithmic_bytes()  # the whole step: keys read, kept rows moved
+    else:
+        algo_launch = keys * 2 * wl.head_dim  # the score kernel reads every key once
+    achieved = algo_launch / (kern_ms[dom] / 1e3) / 1e9
     out = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "metric": METRIC, "value": keys * world / (step / 1e3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded; pages' shapes and value distributions)",
         "config": dict(wl.describe(), l2="flushed: 512 MiB write before every step",
                        parallelism=f"dp{world} (independent caches per GPU)"),
-        "hbm_gbs_path": wl.algorithmic_bytes() / (step / 1e3) / 1e9,
-        "frac_path": wl.algorithmic_bytes() / (step / 1e3) / 1e9 / peak,
-        "roofline": {"bound": "hbm", "kernel": names[score_i], "achieved": achieved,
+        "hbm_gbs_path": head["hbm_gbs_path"],
+        "frac_path": head["frac_path"],
+        "us_per_layer": head["us_per_layer"],
+        "roofline": {"bound": "hbm", "kernel": kern, "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_source": peak_kind, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": score_bytes,
-                     "dominant_kernel": names[dom]},
-        "kernel_ms": dict(zip(names, avg_kern)),
+                     "peak_source": peak_kind, "traffic": _traffic(kern, args.workload),
+                     "algorithmic_bytes_per_launch": algo_launch,
+                     "dominant_kernel": kern},
+        "kernel_ms": dict(zip(names, kern_ms)),
+        "fp32_tflops": head["fp32_tflops"], "frac_fp32": head.get("frac_fp32"),
         "clocks": clocks,
         "e2e": {"value": keys * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": n_stages * args.steps,
+        "gpu_launches": len(names) * args.steps,
     }
+    host_stats = [t.cpu() for t in bench.stats.tensors]
+    bench.free()
+    del data
+
+    # ---- the other workloads and the pages' geometric offsets, same protocol, fewer steps
+    if not args.no_extras:
+        extras = {}
+        geo = [2 ** i for i in range(17)]
+        specs = [("workload2", workloads.workload(2)), ("workload3", workloads.workload(3)),
+                 ("workload4", workloads.workload(4)),
+                 ("workload1_geometric", workloads.workload(1, offsets=geo,
+                                                            name=workloads.workload(1).name + " geometric offsets 1..65536")),
+                 ("workload2_geometric", workloads.workload(2, offsets=geo,
+                                                            name=workloads.workload(2).name + " geometric offsets 1..65536"))]
+        for key, xwl in specs:
+            if rank:
+                xwl = workloads.workload(int(key[8]), seed=xwl.seed + 1000 * rank,
+                                         offsets=xwl.offsets, name=xwl.name)
+            try:
+                xb = Bench(xwl, dev)
+                xb.warm(3)
+                with ClockSampler(local) as xclk:
+                    xms = xb.timed(args.extra_steps)
+                xnames, xkern = xb.kernels(args.extra_steps)
+                xsum = max_over_ranks([sum(xms)] + xkern, device=dev)
+                xc = xclk.summary()
+                entry = xb.summary([xsum[0] / args.extra_steps], xnames, xsum[1:], peak,
+                                   xc["sm_mhz"] if xc else None)
+                entry["value"] *= world
+                entry["steps"] = args.extra_steps
+                entry["clocks"] = xc
+                if tria.tria_get_device_error(xb.ws) != 0:
+                    entry["error"] = "device error flag set"
+                xb.free()
+                del xb
+            except Exception as e:  # a workload that does not fit is reported, not fatal
+                entry = {"workload": xwl.name, "error": f"{type(e).__name__}: {e}"}
+                torch.cuda.empty_cache()
+            extras[key] = entry
+        out["extra_workloads"] = extras
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = _cpu_baseline(wl, host, [t.cpu() for t in stats.tensors])
+        out["cpu_baseline"] = _cpu_baseline(wl, host, host_stats)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -460,6 +571,9 @@ def main():
     ap.add_argument("--workload", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="time only the headline workload (not workloads 2-4 and the geometric offsets)")
+    ap.add_argument("--extra-steps", type=int, default=10)
     ap.add_argument("--ref-seconds", type=float, default=8.0)
     args = ap.parse_args()
     if args.warmup < 3:

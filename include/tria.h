@@ -37,7 +37,9 @@
  * - Cache layout: K and V are bf16 [L][Hkv][cap_total][D] (post-RoPE keys),
  *   pos is int32 [L][Hkv][cap_total].  Sequence b owns slots
  *   [seq_start[b], seq_start[b+1]) of every (layer, KV head) row; its live
- *   keys are the first seq_len[b] of them, with ascending positions.
+ *   keys are the first seq_len[b] of them (or the first unit_len of each
+ *   (layer, KV head, sequence) unit, when the cache has per-unit lengths),
+ *   with ascending positions.
  * - Slot indices in selection lists are relative to the segment start.
  * - Query head h uses KV head h / G, G = n_q_heads / n_kv_heads.
  * - Supported shapes: head_dim in {64, 128, 256}; G in {1, 2, 4, 8, 16};
@@ -82,6 +84,7 @@ typedef enum {
 #define TRIA_DEVERR_TIMEOUT 4      /* a bounded wait on an mbarrier ran out: results invalid */
 #define TRIA_DEVERR_SEGMENT_BIG 8  /* a live sequence exceeded the kernel's per-unit capacity */
 #define TRIA_DEVERR_SEGMENT_FULL 16 /* tria_append: no free slot in a segment: that sequence skipped */
+#define TRIA_DEVERR_BUDGET 32      /* a head budget outside [1, budget]: that KV head's units skipped */
 
 /* Host-side description of the prune problem, copied by value. */
 typedef struct {
@@ -102,6 +105,16 @@ typedef struct {
                            sequence back to budget every prune_window decoded tokens);
                            0 or 1: every sequence with seq_len > budget.  Other calls
                            ignore it. */
+  const int32_t *head_budgets; /* DEVICE int32 [L][Hkv], or NULL.  Head-specific budgets
+                           (romaanj.github.io review, "Future work": compression refined
+                           with budgets per head; the pages give no rule for choosing
+                           them, so they are an input): the units of KV head g of layer
+                           l keep head_budgets[l*Hkv + g] keys, each in [1, budget]
+                           (budget stays the length of every selection list, and an
+                           entry outside that range sets TRIA_DEVERR_BUDGET and leaves
+                           that head's units as they are).  Needs cache->unit_len: the
+                           units of one sequence then hold different numbers of keys.
+                           The prune window applies per unit: head budget + window. */
 } tria_config;
 
 /* The cache.  Device pointers except seq_start. */
@@ -114,6 +127,11 @@ typedef struct {
                               (read by the scoring calls, advanced by tria_append) */
   const int64_t *seq_start;/* HOST int64 [B+1], nondecreasing, seq_start[B] <= cap_total */
   int64_t cap_total;       /* slots per (layer, KV head) row */
+  int32_t *unit_len;       /* DEVICE int32 [L][Hkv][B] (in/out), or NULL.  When set, the
+                              live keys of unit (l, g, b) are the first unit_len[(l*Hkv +
+                              g)*B + b] slots of its segment (units of one sequence may
+                              differ, as after a prune with head budgets); seq_len is then
+                              neither read nor written and may be NULL. */
 } tria_cache;
 
 /* Calibration statistics, DEVICE float32, 16-byte aligned. */
@@ -224,18 +242,22 @@ tria_status tria_decode_attention(const tria_config *cfg, const tria_cache *cach
 
 /* tria_prune (same passages: romaanj.github.io review, "Method";
  * dimensionstp.github.io review, sections 2-1 and 3-2) with a cudaEvent_t
- * (as void*) recorded on `stream` before each
- * of its kernels and after the last: events[0..n_stages].  Returns the number
- * of stages in *n_stages (events must hold TRIA_PRUNE_MAX_STAGES + 1).  For
- * per-kernel timing only. */
+ * (as void*) recorded on `stream` before each of its kernels and after the
+ * last: events[0..n_stages].  Returns the number of stages in *n_stages
+ * (events must hold TRIA_PRUNE_MAX_STAGES + 1) and, if stage_ids is not NULL
+ * (HOST, TRIA_PRUNE_MAX_STAGES entries), the kernel of each stage as an index
+ * for tria_prune_stage_name.  tria_prune runs one fused kernel for the shapes
+ * it fits (every supported shape except head_dim 256 with G = 16) and three
+ * kernels otherwise.  For per-kernel timing only. */
 #define TRIA_PRUNE_MAX_STAGES 8
 tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
                                 const tria_cache *cache, int32_t *sel_out, void *ws,
                                 size_t ws_bytes, void *stream, void *const *events,
-                                int32_t *n_stages);
+                                int32_t *n_stages, int32_t *stage_ids);
 
-/* Names of the kernels tria_prune launches (the steps of the dimensionstp.github.io
- * review, section 2-1, as this library groups them), in order, for stage i. */
+/* Name of the kernel with index i (0 fold, 1 score, 2 unit, 3 the fused prune
+ * kernel; the steps of the dimensionstp.github.io review, section 2-1, as this
+ * library groups them), "" for any other i. */
 const char *tria_prune_stage_name(int32_t i);
 
 /* Reads the workspace's device error word into *code (synchronous: waits for
@@ -263,8 +285,9 @@ tria_status tria_get_device_error(const void *ws, int32_t *code, void *stream);
  *     for a pool and before any stream capture; later calls reserve nothing.
  *     A first call that fails (TRIA_ERR_CUDA) is retried by the next call.
  *   - Every call on a device shares the array.  Each call clears the array's
- *     error word, the only part that must start at zero; calls whose kernels
- *     may overlap on one device (different streams, no ordering) race.
+ *     error word; the other parts that must start at zero start zero and every
+ *     call leaves them zero.  Calls whose kernels may overlap on one device
+ *     (different streams, no ordering) race.
  *   - device_error, if not NULL, is a DEVICE int32 that receives the call's
  *     device error word (TRIA_DEVERR_* bits, 0 if none) at the end of the call,
  *     in stream order; the scratch cannot be passed to tria_get_device_error.

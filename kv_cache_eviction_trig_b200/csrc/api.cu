@@ -4,6 +4,7 @@
 // beyond per-device launch-configuration caches.
 #include <cmath>
 #include <cstring>
+#include <vector>
 
 #include "attention.cuh"
 #include "tria_internal.cuh"
@@ -35,20 +36,40 @@ ScoreGrid score_grid(const tria_config &cfg, const int64_t *seq_start) {
 }
 
 WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap) {
+  static_assert(kPruneMaxGroupUnits == 32 && kPruneHistBins == 4096, "prefix layout");
+  static_assert(kWsBcount + 2 * kPruneMaxGroupUnits * 4 <= kWsHist, "prefix layout");
   WsLayout w{};
   const size_t F = (size_t)cfg.head_dim / 2;
   const size_t units = (size_t)cfg.num_layers * cfg.n_kv_heads * cfg.batch;
   const size_t G = cfg.n_kv_heads > 0 ? (size_t)(cfg.n_q_heads / cfg.n_kv_heads) : 1;
   w.max_slots = score_grid(cfg, seq_start).max_slots;
-  size_t o = 0;
-  w.err = o;      o += 256;
+  w.err = kWsErr;
+  size_t o = kWsPrefix;
   w.seqlen = o;   o = align_up(o + 4ull * cfg.batch, 256);
   w.w = o;        o = align_up(o + 4ull * units * (F / 2) * G * 6, 256);
   w.raw = o;      o = align_up(o + 4ull * cfg.num_layers * cfg.n_q_heads * (size_t)cap, 256);
   w.sel = o;      o = align_up(o + 4ull * units * cfg.budget, 256);
   w.partials = o;
   o = align_up(o + 16ull * units * (size_t)w.max_slots * kScoreConsumerWarps * G, 256);
-  w.total = o;
+  size_t end = o;
+  const PrunePlan pl = prune_plan(cfg, seq_start);
+  w.fused = pl.ok;
+  if (pl.ok) {
+    const size_t nc = (size_t)pl.ncta, ug = (size_t)pl.ug, rowb = 2ull * cfg.head_dim;
+    o = kWsPrefix;
+    w.f_raw = o;       o = align_up(o + 2ull * nc * pl.range_keys * G * 4, 256);
+    w.f_partial = o;   o = align_up(o + 2ull * nc * pl.range_units * G * 16, 256);
+    w.f_zk = o;        o = align_up(o + 2ull * (size_t)pl.zk_stride * 4, 256);
+    w.f_bucket = o;    o = align_up(o + 2ull * ug * kPruneBucketMax * 8, 256);
+    w.f_above = o;     o = align_up(o + 2ull * ug * nc * 4, 256);
+    w.f_thr = o;       o = align_up(o + 2ull * ug * 8, 256);
+    w.f_kcount = o;    o = align_up(o + 2ull * ug * nc * 4, 256);
+    w.f_stage_k = o;   o = align_up(o + ug * (size_t)cfg.budget * rowb, 256);
+    w.f_stage_v = o;   o = align_up(o + ug * (size_t)cfg.budget * rowb, 256);
+    w.f_stage_pos = o; o = align_up(o + ug * (size_t)cfg.budget * 4, 256);
+    if (o > end) end = o;
+  }
+  w.total = end;
   return w;
 }
 
@@ -256,7 +277,110 @@ struct Ws {
   int32_t *sel() const { return reinterpret_cast<int32_t *>(base + lay.sel); }
 };
 
-const char *kStageNames[] = {"fold_kernel", "score_kernel", "unit_kernel"};
+const char *kStageNames[] = {"fold_kernel", "score_kernel", "unit_kernel", "prune_kernel"};
+enum StageId : int32_t { kStageFold = 0, kStageScore = 1, kStageUnit = 2, kStagePrune = 3 };
+
+// Mean over the offsets of e^{i w_f delta} for every RoPE pair (the part of the
+// trigonometric weight that depends on neither the keys nor the current position),
+// in float64 on the host.  The last problem's table is kept per host thread: a
+// decode loop calls with the same offsets every time.
+struct OffsetMean {
+  double theta = 0.0;
+  int32_t D = 0;
+  std::vector<int32_t> offsets;
+  std::vector<double> re, im;
+};
+
+const OffsetMean &offset_mean(const tria_config *cfg) {
+  static thread_local OffsetMean m;
+  const bool same = m.theta == cfg->rope_theta && m.D == cfg->head_dim &&
+                    (int)m.offsets.size() == cfg->n_offsets &&
+                    std::memcmp(m.offsets.data(), cfg->offsets, sizeof(int32_t) * cfg->n_offsets) == 0;
+  if (!same) {
+    const int F = cfg->head_dim / 2;
+    m.theta = cfg->rope_theta;
+    m.D = cfg->head_dim;
+    m.offsets.assign(cfg->offsets, cfg->offsets + cfg->n_offsets);
+    m.re.assign(F, 0.0);
+    m.im.assign(F, 0.0);
+    for (int f = 0; f < F; ++f) {
+      const double w = std::pow(cfg->rope_theta, -2.0 * (double)f / (double)cfg->head_dim);
+      double re = 0.0, im = 0.0;
+      for (int j = 0; j < cfg->n_offsets; ++j) {
+        re += std::cos(w * (double)cfg->offsets[j]);
+        im += std::sin(w * (double)cfg->offsets[j]);
+      }
+      m.re[f] = re / (double)cfg->n_offsets;
+      m.im[f] = im / (double)cfg->n_offsets;
+    }
+  }
+  return m;
+}
+
+// Parameters of the fused prune kernel.
+cudaError_t fill_prune(PruneParams &pp, const tria_config *cfg, const tria_stats *st,
+                       const tria_cache *c, const WsLayout &lay, uint8_t *ws, int32_t *sel_out) {
+  std::memset(&pp, 0, sizeof pp);
+  const PrunePlan pl = prune_plan(*cfg, c->seq_start);
+  if (!pl.ok) return cudaErrorInvalidValue;
+  const int G = cfg->n_q_heads / cfg->n_kv_heads, F = cfg->head_dim / 2;
+  pp.k = static_cast<uint8_t *>(c->k);
+  pp.v = static_cast<uint8_t *>(c->v);
+  pp.pos = c->pos;
+  pp.seq_len = c->seq_len;
+  pp.cur_pos = c->cur_pos;
+  pp.centre = reinterpret_cast<const float2 *>(st->centre);
+  pp.mean_norm = st->mean_norm;
+  pp.mrl = st->mrl;
+  pp.sel_out = sel_out;
+  pp.err = reinterpret_cast<int32_t *>(ws + kWsErr);
+  pp.sync = reinterpret_cast<int32_t *>(ws + kWsSync);
+  pp.bcount = reinterpret_cast<int32_t *>(ws + kWsBcount);
+  pp.hist = reinterpret_cast<uint32_t *>(ws + kWsHist);
+  pp.raw = reinterpret_cast<float *>(ws + lay.f_raw);
+  pp.partial = reinterpret_cast<double *>(ws + lay.f_partial);
+  pp.zk = reinterpret_cast<uint32_t *>(ws + lay.f_zk);
+  pp.bucket = reinterpret_cast<unsigned long long *>(ws + lay.f_bucket);
+  pp.above = reinterpret_cast<int32_t *>(ws + lay.f_above);
+  pp.thr = reinterpret_cast<unsigned long long *>(ws + lay.f_thr);
+  pp.kcount = reinterpret_cast<int32_t *>(ws + lay.f_kcount);
+  pp.stage_k = ws + lay.f_stage_k;
+  pp.stage_v = ws + lay.f_stage_v;
+  pp.stage_pos = reinterpret_cast<int32_t *>(ws + lay.f_stage_pos);
+  pp.cap = c->cap_total;
+  pp.zk_stride = pl.zk_stride;
+  pp.L = cfg->num_layers;
+  pp.Hkv = cfg->n_kv_heads;
+  pp.Hq = cfg->n_q_heads;
+  pp.B = cfg->batch;
+  pp.budget = cfg->budget;
+  pp.window = cfg->prune_window;
+  pp.write_short_sel = sel_out ? 1 : 0;
+  pp.flags = (int32_t)cfg->flags;
+  pp.units = cfg->num_layers * cfg->n_kv_heads * cfg->batch;
+  pp.ug = pl.ug;
+  pp.ngroups = pl.ngroups;
+  pp.ncta = pl.ncta;
+  pp.cpr = pl.cpr;
+  pp.range_keys = pl.range_keys;
+  pp.range_units = pl.range_units;
+  int32_t acc = 0;
+  for (int b = 0; b <= cfg->batch; ++b) {
+    pp.seg_start[b] = c->seq_start[b];
+    pp.chunk_prefix[b] = acc;
+    if (b < cfg->batch)
+      acc += (int32_t)((c->seq_start[b + 1] - c->seq_start[b] + pl.chunk_keys - 1) / pl.chunk_keys);
+  }
+  const OffsetMean &om = offset_mean(cfg);
+  const bool no_trig = (cfg->flags & TRIA_NO_TRIG) != 0;
+  for (int f = 0; f < F && f < 128; ++f) {
+    pp.omega[f] = std::pow(cfg->rope_theta, -2.0 * (double)f / (double)cfg->head_dim);
+    pp.A[f] = no_trig ? make_double2(0.0, 0.0) : make_double2(om.re[f], om.im[f]);
+  }
+  (void)G;
+  const int64_t rows = (int64_t)cfg->num_layers * cfg->n_kv_heads * c->cap_total;
+  return make_key_tensor_map(&pp.tmap, c->k, cfg->head_dim, rows, pl.chunk_keys);
+}
 
 }  // namespace
 
@@ -274,7 +398,8 @@ tria_status tria_workspace_size(const tria_config *cfg, const tria_cache *cache,
 
 tria_status tria_workspace_init(void *ws, size_t ws_bytes, void *stream) {
   if (!ws || ws_bytes < 256 || !aligned(ws, 256)) return TRIA_ERR_WORKSPACE;
-  return cuda_status(cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)));
+  const size_t n = ws_bytes < kWsPrefix ? ws_bytes : kWsPrefix;
+  return cuda_status(cudaMemsetAsync(ws, 0, n, static_cast<cudaStream_t>(stream)));
 }
 
 tria_status tria_calibrate(const tria_config *cfg, const void *q_pre, int32_t q_dtype,
@@ -430,7 +555,7 @@ tria_status tria_decode_attention(const tria_config *cfg, const tria_cache *cach
 tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
                                 const tria_cache *cache, int32_t *sel_out, void *ws,
                                 size_t ws_bytes, void *stream, void *const *events,
-                                int32_t *n_stages) {
+                                int32_t *n_stages, int32_t *stage_ids) {
   tria_status s;
   if ((s = check_config(cfg, true)) != TRIA_OK) return s;
   if ((s = check_cache(cfg, cache, true)) != TRIA_OK) return s;
@@ -440,14 +565,30 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
   if (sel_out && !aligned(sel_out, 4)) return TRIA_ERR_INVALID_ARG;
   if ((s = check_ws(cfg, cache, ws, ws_bytes)) != TRIA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Ws w{ws_layout(*cfg, cache->seq_start, cache->cap_total), static_cast<uint8_t *>(ws)};
+  const WsLayout lay = ws_layout(*cfg, cache->seq_start, cache->cap_total);
+  const Ws w{lay, static_cast<uint8_t *>(ws)};
   int stage = 0;
-  auto mark = [&]() -> bool {
+  auto mark = [&](int32_t id) -> bool {
     if (events && cudaEventRecord(static_cast<cudaEvent_t>(events[stage]), st) != cudaSuccess)
       return false;
+    if (stage_ids && id >= 0 && stage < TRIA_PRUNE_MAX_STAGES) stage_ids[stage] = id;
     ++stage;
     return true;
   };
+
+  if (lay.fused) {
+    // the whole step in one cooperative launch
+    static thread_local PruneParams pp;
+    if (fill_prune(pp, cfg, stats, cache, lay, static_cast<uint8_t *>(ws), sel_out) != cudaSuccess)
+      return TRIA_ERR_CUDA;
+    if (!mark(kStagePrune)) return TRIA_ERR_CUDA;
+    if (launch_prune(pp, cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads, cfg->rope_layout, st) !=
+        cudaSuccess)
+      return TRIA_ERR_CUDA;
+    if (!mark(-1)) return TRIA_ERR_CUDA;
+    if (n_stages) *n_stages = stage - 1;
+    return TRIA_OK;
+  }
 
   static thread_local FoldParams fp;
   fill_fold(fp, cfg, stats, cache, w.seqlen(), w.w(), w.err());
@@ -456,9 +597,9 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
   if (fill_score(sp, cfg, cache, w.w(), w.raw(), w.partials(), w.err(), 1, &grid) != cudaSuccess)
     return TRIA_ERR_CUDA;
   const bool pdl = events == nullptr;  // stage events between kernels would defeat the overlap
-  if (!mark()) return TRIA_ERR_CUDA;
+  if (!mark(kStageFold)) return TRIA_ERR_CUDA;
   if (launch_fold(fp, st) != cudaSuccess) return TRIA_ERR_CUDA;
-  if (!mark()) return TRIA_ERR_CUDA;
+  if (!mark(kStageScore)) return TRIA_ERR_CUDA;
   if (grid > 0 && launch_score(sp, cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads,
                                cfg->rope_layout, grid, st, pdl) != cudaSuccess)
     return TRIA_ERR_CUDA;
@@ -471,17 +612,18 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
   up.seqlen = w.seqlen();
   up.seq_len_out = cache->seq_len;
   up.err = w.err();
-  if (!mark()) return TRIA_ERR_CUDA;
+  if (!mark(kStageUnit)) return TRIA_ERR_CUDA;
   if (launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch, st, pdl) != cudaSuccess)
     return TRIA_ERR_CUDA;
-  if (!mark()) return TRIA_ERR_CUDA;
+  if (!mark(-1)) return TRIA_ERR_CUDA;
   if (n_stages) *n_stages = stage - 1;
   return TRIA_OK;
 }
 
 tria_status tria_prune(const tria_config *cfg, const tria_stats *stats, const tria_cache *cache,
                        int32_t *sel_out, void *ws, size_t ws_bytes, void *stream) {
-  return tria_prune_profiled(cfg, stats, cache, sel_out, ws, ws_bytes, stream, nullptr, nullptr);
+  return tria_prune_profiled(cfg, stats, cache, sel_out, ws, ws_bytes, stream, nullptr, nullptr,
+                             nullptr);
 }
 
 const char *tria_prune_stage_name(int32_t i) {

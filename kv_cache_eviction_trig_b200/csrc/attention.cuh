@@ -10,6 +10,7 @@ struct AttnParams {
   const uint16_t *k;        // bf16 [L][Hkv][cap][D]
   const uint16_t *v;
   const int32_t *seq_len;   // [B]
+  const int32_t *unit_len;  // [L][Hkv][B] per-unit lengths (instead of seq_len), or null
   float *out;               // [B][Hq][D]
   int32_t *err;
   int64_t cap;

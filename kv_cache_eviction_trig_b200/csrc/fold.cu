@@ -15,8 +15,9 @@
 // sequence, then writes, for a share y of
 // the (unit, head) pairs, the float32 weights
 //   w[unit][fp][h] = (Re W_2fp, Re W_2fp+1, Im W_2fp, Im W_2fp+1, Nw_2fp, Nw_2fp+1).
-// Block (0, 0) also snapshots and checks seq_len, so that every later kernel of
-// the call sees the lengths as they were at its start.
+// Block (0, 0) also snapshots and checks seq_len (blocks (0, y) the per-unit
+// lengths, when the cache has them), so that every later kernel of the call sees
+// the lengths as they were at its start.
 #include "tria_internal.cuh"
 
 namespace tria {
@@ -49,7 +50,7 @@ __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldP
     }
   }
   const int32_t cur = threadIdx.x < p.B ? p.cur_pos[threadIdx.x] : 0;
-  const bool snap = blockIdx.x == 0 && blockIdx.y == 0 && (int)threadIdx.x < p.B;
+  const bool snap = !p.unit_len && blockIdx.x == 0 && blockIdx.y == 0 && (int)threadIdx.x < p.B;
   const int32_t t_in = snap ? p.seq_len[threadIdx.x] : 0;
   // w_f = theta^(-2f/D), evaluated on the host in double precision
   const double w[2] = {p.omega[2 * fp], p.omega[2 * fp + 1]};
@@ -122,6 +123,17 @@ __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldP
       T = 0;
     }
     p.seqlen_snap[threadIdx.x] = T;
+  }
+  if (p.unit_len && blockIdx.x == 0) {  // per-unit lengths: blocks (0, y) share the units
+    for (int64_t u = (int64_t)blockIdx.y * blockDim.x + threadIdx.x; u < p.units;
+         u += (int64_t)gridDim.y * blockDim.x) {
+      int32_t T = p.unit_len[u];
+      if (T < 0 || (int64_t)T > p.seg_cap[u % p.B]) {
+        dev::set_error(p.err, TRIA_DEVERR_SEQ_LEN);
+        T = 0;
+      }
+      p.seqlen_snap[u] = T;
+    }
   }
 }
 

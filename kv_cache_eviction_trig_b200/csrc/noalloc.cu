@@ -22,8 +22,10 @@
 // cudaGetSymbolAddress, called with the device current.  Only a successful
 // lookup is kept: a failed one (for example under memory pressure) is retried
 // by the next call.  Every call on a device shares the array and finds the
-// previous call's contents there: the call clears the error word, the only
-// part that must start at zero; everything else is written before it is read.  Two calls whose kernels overlap on a
+// previous call's contents there: the call clears the error word; the other
+// parts that must start at zero (the fused prune kernel's synchronisation words
+// and histograms) start zero with the array and every prune leaves them zero;
+// everything else is written before it is read.  Two calls whose kernels overlap on a
 // device race on the array.
 #include <cstdint>
 #include <mutex>
@@ -72,7 +74,10 @@ extern "C" tria_status tria_prune_noalloc(const tria_config *cfg, const tria_sta
   void *scratch = scratch_on_current_device();
   if (!scratch) return TRIA_ERR_CUDA;
   const size_t bytes = TRIA_NOALLOC_SCRATCH_BYTES;
-  if ((s = tria_workspace_init(scratch, bytes, stream)) != TRIA_OK) return s;
+  // only the error word needs clearing: the rest of the array's zero-at-rest prefix
+  // (synchronisation words, histograms) starts zero and every prune leaves it zero
+  if (cudaMemsetAsync(scratch, 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return TRIA_ERR_CUDA;
   if ((s = tria_prune(cfg, stats, cache, sel_out, scratch, bytes, stream)) != TRIA_OK) return s;
   if (device_error &&
       cudaMemcpyAsync(device_error, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice,

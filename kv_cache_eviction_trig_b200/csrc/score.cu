@@ -169,13 +169,26 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   if (threadIdx.x == 0) dev::pdl_launch_dependents();
   const int c0 = blockIdx.x * p.chunks_per_cta;
   const int c1 = min(c0 + p.chunks_per_cta, p.total_chunks);
+  // Keys to score of unit (row, b): the live length, 0 if out of range or (with
+  // skip_short) too short to prune; per sequence from `live`, or per unit.
+  auto live_of = [&](int row, int b) -> int {
+    if (!p.unit_len) return live[b];
+    int32_t T = p.unit_len[(int64_t)row * p.B + b];
+    if (T < 0 || (int64_t)T > p.seg_start[b + 1] - p.seg_start[b]) return 0;  // flagged by the fold
+    if (p.skip_short) {
+      const int bud = p.head_budget ? p.head_budget[row] : p.budget;
+      if (bud < 1 || bud > p.budget) return 0;
+      if ((int64_t)T < (int64_t)bud + (p.window > 1 ? p.window : 1)) return 0;
+    }
+    return T;
+  };
   // The first unit with live chunks: its weights are copied by the consumers
   // themselves straight from L2 (not queued behind the key stream) into slot 0.
   auto find_first_unit = [&]() {
     for (int c = c0; c < c1; ++c) {
       int row, b, jc;
       chunk_coords(p, c, row, b, jc);
-      if (live[b] > jc * CH) return row * p.B + b;
+      if (live_of(row, b) > jc * CH) return row * p.B + b;
       c += max(0, (p.chunk_prefix[b + 1] - p.chunk_prefix[b]) - jc - 1);  // skip the dead rest
     }
     return -1;
@@ -186,7 +199,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
   if (warp == NW) {
     // ---------------------------------------------------------------- producer
-    for (int b = lane; b < p.B; b += 32) {
+    for (int b = lane; b < p.B && !p.unit_len; b += 32) {
       int32_t T = p.seq_len[b];
       if (T < 0 || (int64_t)T > p.seg_start[b + 1] - p.seg_start[b]) T = 0;  // flagged by the fold
       if (p.skip_short && T < p.prune_from) T = 0;
@@ -236,7 +249,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           int jc;
           chunk_coords(p, c, row, lo, jc);
           key0 = jc * CH;
-          n = min(max(live[lo] - key0, 0), CH);
+          n = min(max(live_of(row, lo) - key0, 0), CH);
         }
         tab[lane] = make_int4(row, lo, key0, n);
         taby[lane] = (int32_t)((int64_t)row * p.cap + p.seg_start[lo] + key0);

@@ -11,6 +11,18 @@
 namespace tria {
 
 // ------------------------------------------------------------------ workspace layout
+// The workspace starts with a fixed prefix that holds state which must be zero
+// when a call starts (tria_workspace_init clears it; the fused prune kernel leaves
+// it zero): the error word, the fused kernel's synchronisation words, bucket
+// counters and histograms.  After it come the per-call regions of either path
+// (fold/score/unit kernels, or the fused kernel); a call uses one path, so the
+// two share the same bytes.
+constexpr size_t kWsErr = 0;
+constexpr size_t kWsSync = 256;
+constexpr size_t kWsBcount = 512;
+constexpr size_t kWsHist = 1024;
+constexpr size_t kWsPrefix = kWsHist + 2ull * 32 * 4096 * 4;  // 2 slots x 32 units x 4096 bins
+
 struct WsLayout {
   size_t err;       // int32 device error word (+ padding)
   size_t seqlen;    // int32 [B]   snapshot of seq_len taken at the start of a call
@@ -19,6 +31,10 @@ struct WsLayout {
   size_t sel;       // int32 [L][Hkv][B][budget] selection scratch
   size_t partials;  // double [L*Hkv*B][max_slots][score warps][G][2] sums of s and s^2
   int32_t max_slots;
+  // fused prune kernel (same bytes as the regions above)
+  int fused;        // the fused kernel runs this problem's prune
+  size_t f_raw, f_partial, f_zk, f_bucket, f_above, f_thr, f_kcount, f_stage_k, f_stage_v,
+      f_stage_pos;
   size_t total;
 };
 WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap_total);
@@ -62,7 +78,9 @@ constexpr int kUnitSmemLarge = 200 * 1024;  // one CTA per SM
 struct FoldParams {
   const int32_t *cur_pos;   // [B]
   const int32_t *seq_len;   // [B] caller's live lengths
-  int32_t *seqlen_snap;     // [B] out
+  const int32_t *unit_len;  // [U] per-unit live lengths (instead of seq_len), or null
+  int32_t *seqlen_snap;     // [B], or [U] with per-unit lengths, out
+  int64_t units;
   int32_t *err;
   const float2 *centre;     // [L][Hq][F]
   const float *mean_norm;   // [L][Hq][F]
@@ -80,6 +98,9 @@ struct alignas(64) ScoreParams {
   CUtensorMap tmap;         // K as a 2-D bf16 tensor [L*Hkv*cap][D], 128-byte swizzled boxes
   const float *w;           // folded weights (written by the fold kernel)
   const int32_t *seq_len;   // [B] caller's live lengths (not modified during the call)
+  const int32_t *unit_len;  // [U] per-unit live lengths instead, or null
+  const int32_t *head_budget;  // [L*Hkv] per-head budgets (with skip_short), or null
+  int32_t budget, window;   // with skip_short: units shorter than budget + max(window, 1) are skipped
   float *raw;               // [L][Hq][cap]
   double *partials;         // per (unit, slot, warp): float64 sums of s and s^2 per head
   int32_t max_slots;
@@ -107,8 +128,11 @@ struct UnitParams {
   int32_t chunk_prefix[TRIA_MAX_BATCH + 1];
   float *score;             // [L][Hkv][cap]     (zmax writes, select reads)
   int32_t *sel;             // [L][Hkv][B][budget]
-  const int32_t *seqlen;    // [B] snapshot (zmax, select, prune)
-  int32_t *seq_len_out;     // [B] (compact, prune)
+  const int32_t *seqlen;    // [B] snapshot (zmax, select, prune), or [U] with unit_mode
+  int32_t *seq_len_out;     // [B] (compact, prune), or [U] with unit_mode
+  int32_t unit_mode;        // lengths per (layer, KV head, sequence) unit
+  const int32_t *head_budget;  // [L*Hkv] per-head budgets, or null
+  int32_t window;           // prune: a unit is pruned once T >= its budget + max(window, 1)
   int32_t *err;
   int64_t cap;
   int32_t L, Hkv, Hq, B, G, D, budget;
@@ -119,6 +143,68 @@ struct UnitParams {
   int32_t cluster;          // CTAs per unit (1 or kUnitCluster)
   int64_t seg_start[TRIA_MAX_BATCH + 1];
 };
+
+// ------------------------------------------------------------------ fused prune kernel
+// One cooperative, persistent launch (one CTA per SM) scores, z-scores, selects and
+// compacts every unit.  Units are taken in groups of consecutive units; every CTA
+// scores an equal share of each group's key chunks, and select warps finish a group
+// (through four grid-wide rounds on counters in the workspace) while the consumer
+// warps already score the next one.
+constexpr int kPruneConsumerWarps = 8;
+constexpr int kPruneSelectWarps = 4;
+constexpr int kPruneThreads = (kPruneConsumerWarps + 1 + kPruneSelectWarps) * 32;
+constexpr int kPruneRangeKeys = 2048;  // keys of one CTA's share of a group, at most
+constexpr int kPruneHistBins = 4096;   // bins of a unit's z histogram (1/256 over [-8, 8))
+constexpr int kPruneBucketMax = 4096;  // threshold-bin keys gathered by every CTA
+constexpr int kPruneMaxGroupUnits = 32;
+// sync words (int32) at the start of the persistent prefix of the workspace
+enum PruneSync : int { kSyncA = 0, kSyncB = 2, kSyncC = 4, kSyncD = 6, kSyncExit = 8,
+                       kSyncAbort = 9, kSyncWords = 16 };
+
+struct alignas(64) PruneParams {
+  CUtensorMap tmap;           // K as [L*Hkv*cap][D] bf16, 128-byte swizzled boxes
+  uint8_t *k, *v;             // bf16 rows
+  int32_t *pos;
+  int32_t *seq_len;           // [B] in/out (null with per-unit lengths)
+  int32_t *unit_len;          // [U] in/out per-unit lengths, or null
+  const int32_t *head_budget; // [L*Hkv] per-head budgets, or null
+  const int32_t *cur_pos;     // [B]
+  const float2 *centre;       // [L][Hq][F]
+  const float *mean_norm;     // [L][Hq][F]
+  const float *mrl;           // [L][Hq][F]
+  int32_t *sel_out;           // [U][budget] or null
+  int32_t *err;
+  int32_t *sync;              // kSyncWords
+  int32_t *bcount;            // [2][kPruneMaxGroupUnits] bucket fill counters (zero at rest)
+  uint32_t *hist;             // [2][kPruneMaxGroupUnits][kPruneHistBins] (zero at rest)
+  float *raw;                 // [2][ncta][range_keys][G]
+  double *partial;            // [2][ncta][range_units][G][2]
+  uint32_t *zk;               // [2][zk_stride] z keys of a group, by chunk position
+  unsigned long long *bucket; // [2][ug][kPruneBucketMax] (key << 18 | ~slot) of threshold bins
+  int32_t *above;             // [2][ug][ncta] per covering CTA: keys above the threshold bin
+  unsigned long long *thr;    // [2][ug] threshold key of an exactly selected unit
+  int32_t *kcount;            // [2][ug][ncta] per covering CTA: kept keys (exact path)
+  uint8_t *stage_k, *stage_v; // [ug][budget] rows
+  int32_t *stage_pos;         // [ug][budget]
+  int64_t cap;
+  int64_t zk_stride;
+  int32_t L, Hkv, Hq, B, budget, window, write_short_sel, flags;
+  int32_t units, ug, ngroups, ncta, cpr, range_keys, range_units;
+  int64_t seg_start[TRIA_MAX_BATCH + 1];
+  int32_t chunk_prefix[TRIA_MAX_BATCH + 1];
+  double omega[128];          // w_f = theta^(-2f/D)
+  double2 A[128];             // mean over the offsets of e^{i w_f delta} (0 without the trig term)
+};
+
+struct PrunePlan {
+  int ok;                     // 0: the fused kernel cannot run this problem
+  int chunk_keys, ncta, ug, ngroups, cpr, range_keys, range_units;
+  int64_t zk_stride;
+};
+PrunePlan prune_plan(const tria_config &cfg, const int64_t *seq_start);
+bool prune_supported(int D, int G, int layout);
+size_t prune_smem_bytes(int D, int G);
+cudaError_t launch_prune(const PruneParams &p, int D, int G, int layout, cudaStream_t s);
 
 // ------------------------------------------------------------------ launchers (host)
 cudaError_t launch_fold(const FoldParams &p, cudaStream_t s);
@@ -136,6 +222,7 @@ int unit_smem_bytes();
 // Decode-loop append: the new token's K, V rows and position into each segment's
 // next free slot, then seq_len and cur_pos advance (two launches).
 struct AppendParams {
+  int32_t *unit_len;        // [L][Hkv][B] per-unit lengths (instead of seq_len), or null
   const uint8_t *k_new;     // bf16 [L][Hkv][B][D]
   const uint8_t *v_new;
   uint8_t *k;               // bf16 [L][Hkv][cap][D]

@@ -39,6 +39,7 @@ DEVERR_SELECTION = 2
 DEVERR_TIMEOUT = 4
 DEVERR_SEGMENT_BIG = 8
 DEVERR_SEGMENT_FULL = 16
+DEVERR_BUDGET = 32
 
 EXPORTS = ["tria_workspace_size", "tria_workspace_init", "tria_calibrate", "tria_score",
            "tria_select", "tria_compact", "tria_prune", "tria_prune_profiled",
@@ -58,13 +59,15 @@ class tria_config(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("rope_theta", ctypes.c_double),
                 ("rope_layout", ctypes.c_int32), ("budget", ctypes.c_int32),
                 ("offsets", ctypes.POINTER(ctypes.c_int32)), ("n_offsets", ctypes.c_int32),
-                ("flags", ctypes.c_uint32), ("prune_window", ctypes.c_int32)]
+                ("flags", ctypes.c_uint32), ("prune_window", ctypes.c_int32),
+                ("head_budgets", ctypes.c_void_p)]
 
 
 class tria_cache(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("pos", ctypes.c_void_p),
                 ("seq_len", ctypes.c_void_p), ("cur_pos", ctypes.c_void_p),
-                ("seq_start", ctypes.POINTER(ctypes.c_int64)), ("cap_total", ctypes.c_int64)]
+                ("seq_start", ctypes.POINTER(ctypes.c_int64)), ("cap_total", ctypes.c_int64),
+                ("unit_len", ctypes.c_void_p)]
 
 
 class tria_stats(ctypes.Structure):
@@ -96,7 +99,8 @@ def lib():
         L.tria_prune.argtypes = [P(tria_config), P(tria_stats), P(tria_cache), vp, vp,
                                  ctypes.c_size_t, vp]
         L.tria_prune_profiled.argtypes = [P(tria_config), P(tria_stats), P(tria_cache), vp, vp,
-                                          ctypes.c_size_t, vp, P(vp), P(ctypes.c_int32)]
+                                          ctypes.c_size_t, vp, P(vp), P(ctypes.c_int32),
+                                          P(ctypes.c_int32)]
         L.tria_prune_noalloc.argtypes = [P(tria_config), P(tria_stats), P(tria_cache), vp, vp,
                                          vp]
         L.tria_append.argtypes = [P(tria_config), P(tria_cache), vp, vp, vp, ctypes.c_size_t, vp]
@@ -144,32 +148,39 @@ class Config:
 
     def __init__(self, *, num_layers: int, batch: int, n_q_heads: int, n_kv_heads: int,
                  head_dim: int, rope_theta: float, budget: int, offsets: Sequence[int],
-                 rope_layout: int = ROPE_HALF_SPLIT, flags: int = 0, prune_window: int = 0):
+                 rope_layout: int = ROPE_HALF_SPLIT, flags: int = 0, prune_window: int = 0,
+                 head_budgets: Optional[torch.Tensor] = None):
+        """head_budgets: int32 [L][Hkv] device tensor of per-head budgets (each <= budget),
+        or None for the single budget."""
         self._offsets = (ctypes.c_int32 * max(1, len(offsets)))(*offsets)
+        self.head_budgets = head_budgets
         self.c = tria_config(num_layers, batch, n_q_heads, n_kv_heads, head_dim,
                              float(rope_theta), rope_layout, budget,
                              ctypes.cast(self._offsets, ctypes.POINTER(ctypes.c_int32)),
-                             len(offsets), flags, prune_window)
+                             len(offsets), flags, prune_window, _ptr(head_budgets))
 
     @classmethod
-    def from_workload(cls, wl, flags: int = 0, prune_window: int = 0) -> "Config":
+    def from_workload(cls, wl, flags: int = 0, prune_window: int = 0,
+                      head_budgets: Optional[torch.Tensor] = None) -> "Config":
         return cls(num_layers=wl.num_layers, batch=wl.batch, n_q_heads=wl.n_q_heads,
                    n_kv_heads=wl.n_kv_heads, head_dim=wl.head_dim, rope_theta=wl.rope_theta,
                    budget=wl.budget, offsets=wl.offsets, rope_layout=wl.rope_layout, flags=flags,
-                   prune_window=prune_window)
+                   prune_window=prune_window, head_budgets=head_budgets)
 
 
 class Cache:
     """tria_cache over torch tensors (k, v bf16 [L][Hkv][cap][D]; pos int32 [L][Hkv][cap];
-    seq_len, cur_pos int32 [B] on the device; seq_start a host list of B+1 ints)."""
+    seq_len, cur_pos int32 [B] on the device; seq_start a host list of B+1 ints;
+    optionally unit_len int32 [L][Hkv][B], the per-unit live lengths)."""
 
     def __init__(self, k, v, pos, seq_len, cur_pos, seq_start: Sequence[int],
-                 cap_total: Optional[int] = None):
-        self.tensors = (k, v, pos, seq_len, cur_pos)
+                 cap_total: Optional[int] = None, unit_len=None):
+        self.tensors = (k, v, pos, seq_len, cur_pos, unit_len)
         self._starts = (ctypes.c_int64 * len(seq_start))(*seq_start)
         cap = cap_total if cap_total is not None else (k.shape[2] if k is not None else 0)
         self.c = tria_cache(_ptr(k), _ptr(v), _ptr(pos), _ptr(seq_len), _ptr(cur_pos),
-                            ctypes.cast(self._starts, ctypes.POINTER(ctypes.c_int64)), cap)
+                            ctypes.cast(self._starts, ctypes.POINTER(ctypes.c_int64)), cap,
+                            _ptr(unit_len))
 
     @classmethod
     def from_data(cls, data: dict) -> "Cache":
@@ -267,19 +278,21 @@ def tria_decode_attention(cfg: Config, cache: Cache, layer: int, q: torch.Tensor
 
 
 def tria_prune_profiled(cfg: Config, stats: Stats, cache: Cache, ws: torch.Tensor, events,
-                        sel_out: Optional[torch.Tensor] = None, stream=None) -> int:
-    """events: PRUNE_MAX_STAGES + 1 torch.cuda.Event(enable_timing=True); returns n_stages."""
+                        sel_out: Optional[torch.Tensor] = None, stream=None):
+    """events: PRUNE_MAX_STAGES + 1 torch.cuda.Event(enable_timing=True).
+    Returns the kernel name of each stage (stage i runs between events i and i+1)."""
     for e in events:
         if not e.cuda_event:  # torch creates the CUDA event on its first record
             e.record(stream if stream is not None else torch.cuda.current_stream())
     arr = (ctypes.c_void_p * (PRUNE_MAX_STAGES + 1))(
         *[ctypes.c_void_p(e.cuda_event) for e in events])
     n = ctypes.c_int32(0)
+    ids = (ctypes.c_int32 * PRUNE_MAX_STAGES)()
     _check(lib().tria_prune_profiled(ctypes.byref(cfg.c), ctypes.byref(stats.c),
                                      ctypes.byref(cache.c), _ptr(sel_out), _ptr(ws), ws.numel(),
-                                     _stream(stream), arr, ctypes.byref(n)),
+                                     _stream(stream), arr, ctypes.byref(n), ids),
            "tria_prune_profiled")
-    return int(n.value)
+    return [tria_prune_stage_name(ids[i]) for i in range(n.value)]
 
 
 def tria_prune_noalloc(cfg: Config, stats: Stats, cache: Cache,

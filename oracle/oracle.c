@@ -62,7 +62,23 @@ typedef struct {
   const double *centre;             /* [L][Hq][D/2][2] complex E[q_f] */
   const double *mean_norm;          /* [L][Hq][D/2] E|q_f| */
   const double *mrl;                /* [L][Hq][D/2] R_f */
+  const int32_t *head_budget;       /* [L][Hkv] keys kept per unit of each KV head, or NULL */
+  const int32_t *unit_len;          /* [L][Hkv][B] live keys per unit, or NULL (seq_len) */
 } orc_problem;
+
+/*
+ * Head-specific budgets [R1 Future work: refined compression with budgets per
+ * head]: the pages name the idea without a rule for choosing the budgets, so the
+ * budgets are an input, one per (layer, KV head), each at most `budget` (the row
+ * length of the selection lists).  Once heads keep different numbers of keys,
+ * the units of one sequence have different lengths: unit_len holds them.
+ */
+static int64_t unit_T(const orc_problem *p, int32_t l, int32_t g, int32_t b) {
+  return p->unit_len ? p->unit_len[((int64_t)l * p->Hkv + g) * p->B + b] : p->seq_len[b];
+}
+static int32_t unit_budget(const orc_problem *p, int32_t l, int32_t g) {
+  return p->head_budget ? p->head_budget[(int64_t)l * p->Hkv + g] : p->budget;
+}
 
 /* bfloat16 bits -> double: the bf16 value is the top half of a float32. */
 static double bf16_to_double(uint16_t b) {
@@ -167,9 +183,12 @@ double orc_key_score(const orc_problem *p, int32_t l, int32_t h, int32_t b, int6
  * own; the work is shared out over (layer, head, sequence, block of 256 keys). */
 void orc_raw_scores(const orc_problem *p, double *raw) {
   const int64_t blk = 256;
+  const int32_t G = p->Hq / p->Hkv;
   int64_t most = 0;
-  for (int32_t b = 0; b < p->B; ++b)
-    if (p->seq_len[b] > most) most = p->seq_len[b];
+  for (int32_t l = 0; l < p->L; ++l)
+    for (int32_t g = 0; g < p->Hkv; ++g)
+      for (int32_t b = 0; b < p->B; ++b)
+        if (unit_T(p, l, g, b) > most) most = unit_T(p, l, g, b);
   const int64_t nblk = (most + blk - 1) / blk;
   const int64_t units = (int64_t)p->L * p->Hq * p->B;
 #pragma omp parallel for schedule(dynamic, 1)
@@ -179,7 +198,8 @@ void orc_raw_scores(const orc_problem *p, double *raw) {
     const int32_t h = (int32_t)((u / p->B) % p->Hq);
     const int32_t l = (int32_t)(u / ((int64_t)p->B * p->Hq));
     double *out = raw + ((int64_t)l * p->Hq + h) * p->cap + p->seq_start[b];
-    const int64_t t1 = (kb + 1) * blk < p->seq_len[b] ? (kb + 1) * blk : p->seq_len[b];
+    const int64_t T = unit_T(p, l, h / G, b);
+    const int64_t t1 = (kb + 1) * blk < T ? (kb + 1) * blk : T;
     for (int64_t t = kb * blk; t < t1; ++t) out[t] = orc_key_score(p, l, h, b, t);
   }
 }
@@ -228,7 +248,7 @@ void orc_raw_scores_folded(const orc_problem *p, double *raw) {
     }
     const int64_t row = ((int64_t)l * p->Hkv + g) * p->cap + p->seq_start[b];
     double *out = raw + ((int64_t)l * p->Hq + h) * p->cap + p->seq_start[b];
-    for (int64_t t = 0; t < p->seq_len[b]; ++t) {
+    for (int64_t t = 0; t < unit_T(p, l, g, b); ++t) {
       const uint16_t *k = p->k + (row + t) * D;
       double s = 0.0;
       for (int32_t f = 0; f < F; ++f) {
@@ -269,7 +289,7 @@ void orc_zmax(const orc_problem *p, const double *raw, double *z, double *score)
     const int32_t b = (int32_t)(u % p->B);
     const int32_t g = (int32_t)((u / p->B) % p->Hkv);
     const int32_t l = (int32_t)(u / ((int64_t)p->B * p->Hkv));
-    const int64_t T = p->seq_len[b], s0 = p->seq_start[b];
+    const int64_t T = unit_T(p, l, g, b), s0 = p->seq_start[b];
     double *sc = score + ((int64_t)l * p->Hkv + g) * p->cap + s0;
     for (int64_t t = 0; t < T; ++t) sc[t] = -INFINITY;
     for (int32_t j = 0; j < G; ++j) {
@@ -308,8 +328,9 @@ static int by_value(const void *a, const void *b) {
 /*
  * Top-budget selection [R1 Method; R2 3-2 (5)]: per (layer, KV head,
  * sequence), sort the keys by (score descending, slot ascending), keep the
- * first `budget`, and list them by ascending slot.  A sequence of at most
- * `budget` keys keeps every key.  sel is [L][Hkv][B][budget], padded with -1.
+ * first `budget` (the unit's head budget when budgets are per head), and list
+ * them by ascending slot.  A unit of at most that many keys keeps every key.
+ * sel is [L][Hkv][B][budget], padded with -1.
  */
 void orc_select(const orc_problem *p, const double *score, int32_t *sel) {
   const int64_t units = (int64_t)p->L * p->Hkv * p->B;
@@ -318,10 +339,11 @@ void orc_select(const orc_problem *p, const double *score, int32_t *sel) {
     const int32_t b = (int32_t)(u % p->B);
     const int32_t g = (int32_t)((u / p->B) % p->Hkv);
     const int32_t l = (int32_t)(u / ((int64_t)p->B * p->Hkv));
-    const int64_t T = p->seq_len[b];
+    const int64_t T = unit_T(p, l, g, b);
+    const int32_t keep = unit_budget(p, l, g);
     int32_t *out = sel + (((int64_t)l * p->Hkv + g) * p->B + b) * p->budget;
     for (int32_t j = 0; j < p->budget; ++j) out[j] = -1;
-    if (T <= p->budget) {
+    if (T <= keep) {
       for (int64_t t = 0; t < T; ++t) out[t] = (int32_t)t;
       continue;
     }
@@ -329,8 +351,8 @@ void orc_select(const orc_problem *p, const double *score, int32_t *sel) {
     orc_key *keys = (orc_key *)malloc((size_t)T * sizeof(orc_key));
     for (int64_t t = 0; t < T; ++t) { keys[t].score = sc[t]; keys[t].slot = t; }
     qsort(keys, (size_t)T, sizeof(orc_key), by_score_then_slot);
-    for (int32_t j = 0; j < p->budget; ++j) out[j] = (int32_t)keys[j].slot;
-    qsort(out, (size_t)p->budget, sizeof(int32_t), by_value);
+    for (int32_t j = 0; j < keep; ++j) out[j] = (int32_t)keys[j].slot;
+    qsort(out, (size_t)keep, sizeof(int32_t), by_value);
     free(keys);
   }
 }
@@ -340,20 +362,29 @@ void orc_select(const orc_problem *p, const double *score, int32_t *sel) {
  * pos move to the front of the segment in ascending slot order and the
  * sequence length becomes the number kept.  k, v ([L][Hkv][cap][D] bf16 bits)
  * and pos ([L][Hkv][cap]) are updated in place through a temporary copy;
- * seq_len_out[b] receives the new length.
+ * seq_len_out[b] receives the new length (the one all units of sequence b share
+ * when there is a single budget), unit_len_out[L][Hkv][B] every unit's.
  */
 void orc_compact(const orc_problem *p, const int32_t *sel, uint16_t *k, uint16_t *v,
-                 int32_t *pos, int32_t *seq_len_out) {
+                 int32_t *pos, int32_t *seq_len_out, int32_t *unit_len_out) {
   const int32_t D = p->D;
   for (int32_t b = 0; b < p->B; ++b)
     seq_len_out[b] = p->seq_len[b] < p->budget ? p->seq_len[b] : p->budget;
   const int64_t units = (int64_t)p->L * p->Hkv * p->B;
+  for (int64_t u = 0; u < units; ++u) {
+    const int32_t b = (int32_t)(u % p->B);
+    const int32_t g = (int32_t)((u / p->B) % p->Hkv);
+    const int32_t l = (int32_t)(u / ((int64_t)p->B * p->Hkv));
+    const int64_t T = unit_T(p, l, g, b);
+    const int32_t kept_max = unit_budget(p, l, g);
+    unit_len_out[u] = (int32_t)(T < kept_max ? T : kept_max);
+  }
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t u = 0; u < units; ++u) {
     const int32_t b = (int32_t)(u % p->B);
     const int32_t g = (int32_t)((u / p->B) % p->Hkv);
     const int32_t l = (int32_t)(u / ((int64_t)p->B * p->Hkv));
-    const int64_t n = seq_len_out[b];
+    const int64_t n = unit_len_out[u];
     const int64_t base = ((int64_t)l * p->Hkv + g) * p->cap + p->seq_start[b];
     const int32_t *s = sel + (((int64_t)l * p->Hkv + g) * p->B + b) * p->budget;
     uint16_t *tk = (uint16_t *)malloc((size_t)(n > 0 ? n : 1) * D * sizeof(uint16_t));

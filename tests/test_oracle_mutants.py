@@ -34,6 +34,13 @@ MUTANTS = {
                                   "hypot(centre[2 * o], centre[2 * o + 1]) / (mean_norm[o] * (double)N)"),
     "conjugated centre": ("const double cx = p->centre[2 * o], cy = p->centre[2 * o + 1];",
                           "const double cx = p->centre[2 * o], cy = -p->centre[2 * o + 1];"),
+    "head budget ignored": ("const int32_t keep = unit_budget(p, l, g);",
+                            "const int32_t keep = p->budget;"),
+    "unit length ignored": ("return p->unit_len ? p->unit_len[((int64_t)l * p->Hkv + g) * p->B + b] : p->seq_len[b];",
+                            "return p->seq_len[b];"),
+    "kept count one short of the head budget": (
+        "unit_len_out[u] = (int32_t)(T < kept_max ? T : kept_max);",
+        "unit_len_out[u] = (int32_t)(T < kept_max ? T : kept_max - 1);"),
 }
 
 PIN_TESTS = [
@@ -47,6 +54,8 @@ PIN_TESTS = [
     (pins.test_zscore_invariants_and_max, {}),
     (pins.test_select_equals_brute_force_with_ties, {"T": 64, "budget": 7}),
     (pins.test_compaction_moves_selected_rows_in_order, {}),
+    (pins.test_uniform_head_budgets_are_the_plain_prune, {}),
+    (pins.test_head_budgets_keep_each_heads_top_b, {}),
 ]
 
 
@@ -81,15 +90,15 @@ def test_planted_mistake_is_caught(name, tmp_path):
 
 # Mistakes in the decode-loop steps of the oracle (Python functions of the package).
 PY_MUTANTS = {
-    "window threshold off by one": ("prune_window", "if T >= thr or T <= p.budget:",
-                                    "if T > thr or T <= p.budget:"),
-    "window ignored": ("prune_window", "thr = p.budget + max(int(window), 1)",
-                       "thr = p.budget + 1"),
-    "appended position not advanced": ("append", "pos[:, :, slot] = cur_pos[b] + 1",
-                                       "pos[:, :, slot] = cur_pos[b]"),
+    "window threshold off by one": ("prune_window", "if T >= thr or T <= bud:",
+                                    "if T > thr or T <= bud:"),
+    "window ignored": ("prune_window", "thr = bud + max(int(window), 1)", "thr = bud + 1"),
+    "appended position not advanced": ("append", "pos[l, g, slot] = cur_pos[b] + 1",
+                                       "pos[l, g, slot] = cur_pos[b]"),
     "append over the newest token": ("append", "slot = int(seq_start[b]) + T",
                                      "slot = int(seq_start[b]) + max(T - 1, 0)"),
-    "full segment overwritten": ("append", "if T < 0 or T >= room:", "if T < 0 or T > room:"),
+    "full segment overwritten": ("append", "if (Ts < 0).any() or (Ts >= room).any():",
+                                 "if (Ts < 0).any() or (Ts > room).any():"),
     "softmax without the max shift": ("decode_attention", "w = np.exp(logits - logits.max())",
                                       "w = np.exp(logits)"),
     "KV head by modulo": ("decode_attention", "g = h // G", "g = h % Hkv"),
@@ -102,6 +111,8 @@ PY_MUTANTS = {
 }
 
 PY_PIN_TESTS = [pins.test_prune_window_threshold,
+                pins.test_head_budget_window_decides_per_unit,
+                pins.test_append_and_attention_follow_each_units_length,
                 pins.test_append_writes_the_next_slot_and_advances,
                 pins.test_decode_loop_lengths_follow_the_window_sawtooth,
                 pins.test_attention_single_key_returns_its_value,

@@ -606,3 +606,123 @@ def test_folded_scores_equal_term_by_term(layout, offsets, flags):
     assert np.array_equal(live, ~np.isnan(b))
     scale = np.abs(a[live]).max()
     np.testing.assert_allclose(b[live], a[live], rtol=0, atol=1e-10 * scale)
+
+
+# ------------------------------------------------------- head-specific budgets
+# romaanj.github.io review, "Future work": refined compression with budgets per head.
+# The pages give no rule for choosing them, so they are an input per (layer, KV head);
+# once heads keep different numbers of keys every unit has its own length.
+
+def _budget_problem(seed, budgets, unit_len, seq_lens, budget_max, L=2, Hkv=3):
+    wl = workloads.custom("pin-heads", L=L, B=len(seq_lens), Hq=2 * Hkv, Hkv=Hkv, D=16,
+                          theta=1.0e4, budget=budget_max, offsets=list(range(1, 9)),
+                          seq_lens=seq_lens, seed=seed, nu=0.5, n_calib=64)
+    data = workloads.generate(wl)
+    stats = common.stats_fp32(data["q_calib"], wl.rope_layout)
+    c, m, r = stats
+    p = oracle.Problem(k=common.bf16_bits(data["k"]), pos=data["pos"].numpy(),
+                       seq_start=data["seq_start"], seq_len=data["seq_len"].numpy(),
+                       cur_pos=data["cur_pos"].numpy(), centre=c.astype(np.float64),
+                       mean_norm=m.astype(np.float64), mrl=r.astype(np.float64),
+                       theta=wl.rope_theta, budget=budget_max, offsets=wl.offsets,
+                       n_q_heads=wl.n_q_heads, budgets=budgets, unit_len=unit_len)
+    return wl, data, stats, p
+
+
+def test_uniform_head_budgets_are_the_plain_prune():
+    """Every head at the same budget, every unit at its sequence's length: the
+    per-head prune is the plain prune, byte for byte."""
+    lens = [40, 12, 9]
+    wl, data, stats, p = _budget_problem(31, np.full((2, 3), 10), np.broadcast_to(
+        np.array(lens, np.int32), (2, 3, 3)), lens, 10)
+    plain = oracle.prune(common.problem(wl, data, stats), common.bf16_bits(data["v"]))
+    heads = oracle.prune(p, common.bf16_bits(data["v"]))
+    for key in ("raw", "score", "sel", "k", "v", "pos", "unit_len"):
+        np.testing.assert_array_equal(np.nan_to_num(plain[key], nan=-7.0),
+                                      np.nan_to_num(heads[key], nan=-7.0), err_msg=key)
+
+
+def test_head_budgets_keep_each_heads_top_b():
+    """Ragged budgets and ragged unit lengths: each unit keeps exactly the top
+    min(T_u, b_h) keys of its own scores (brute-force count of better keys, ties to
+    the lower slot), in slot order; a head whose budget is at least the unit's
+    length keeps the unit untouched; the z-score runs over the unit's own live
+    keys (mean 0, population std 1 per query head)."""
+    rng = np.random.default_rng(32)
+    seq_lens = [30, 30]
+    budgets = np.array([[4, 30, 11], [1, 7, 29]], np.int32)
+    unit_len = rng.integers(5, 31, size=(2, 3, 2)).astype(np.int32)
+    unit_len[0, 1, 0] = 30
+    wl, data, stats, p = _budget_problem(33, budgets, unit_len, seq_lens, 30)
+    v = common.bf16_bits(data["v"])
+    out = oracle.prune(p, v)
+    G = wl.group
+    for l in range(2):
+        for g in range(3):
+            for b in range(2):
+                T, bud = int(unit_len[l, g, b]), int(budgets[l, g])
+                s0 = data["seq_start"][b]
+                for h in range(g * G, (g + 1) * G):
+                    z = out["z"][l, h, s0:s0 + T]
+                    assert abs(z.mean()) < 1e-12 and abs(z.std() - 1.0) < 1e-12
+                    assert np.all(np.isnan(out["z"][l, h, s0 + T:data["seq_start"][b + 1]]))
+                sc = out["score"][l, g, s0:s0 + T]
+                want = _brute_select(sc, bud)
+                sel = out["sel"][l, g, b]
+                assert sel[:len(want)].tolist() == want and np.all(sel[len(want):] == -1)
+                n = min(T, bud)
+                assert out["unit_len"][l, g, b] == n
+                np.testing.assert_array_equal(out["k"][l, g, s0:s0 + n], p.k[l, g, s0 + sel[:n]])
+                np.testing.assert_array_equal(out["v"][l, g, s0:s0 + n], v[l, g, s0 + sel[:n]])
+                if T <= bud:  # untouched
+                    np.testing.assert_array_equal(out["k"][l, g, s0:s0 + 30], p.k[l, g, s0:s0 + 30])
+
+
+def test_head_budget_window_decides_per_unit():
+    """With per-head budgets the prune window applies to each unit: a unit is pruned
+    once its length reaches its own budget + window, else left as it is."""
+    budgets = np.array([[5, 9]], np.int32)
+    unit_len = np.array([[[9, 8]], [[12, 13]]], np.int32).reshape(1, 2, 2)
+    wl, data, stats, p = _budget_problem(34, budgets, unit_len, [20, 20], 12, L=1, Hkv=2)
+    v = common.bf16_bits(data["v"])
+    full = oracle.prune(p, v)
+    win = oracle.prune_window(p, v, 4)
+    # head 0 (budget 5): 9 >= 5 + 4 is pruned, 8 is held back; head 1 (budget 9): 12 < 13
+    # is held back, 13 is pruned
+    assert win["unit_len"].tolist() == [[[5, 8], [12, 9]]]
+    assert np.all(win["sel"][0, 0, 1] == -2) and np.all(win["sel"][0, 1, 0] == -2)
+    np.testing.assert_array_equal(win["sel"][0, 0, 0], full["sel"][0, 0, 0])
+    np.testing.assert_array_equal(win["sel"][0, 1, 1], full["sel"][0, 1, 1])
+    s1 = data["seq_start"][1]
+    np.testing.assert_array_equal(win["k"][0, 0, s1:], p.k[0, 0, s1:])
+
+
+def test_append_and_attention_follow_each_units_length():
+    """Per-unit lengths: a decoded token lands at each unit's own next slot, every
+    unit grows by one; a sequence with a full unit is skipped whole; attention reads
+    each unit's live slots only."""
+    rng = np.random.default_rng(35)
+    L, Hkv, D = 1, 2, 8
+    starts, cur = [0, 6, 10], [40, 70]
+    ul = np.array([[[3, 4], [5, 2]]], np.int32)            # [L][Hkv][B]; unit (0,1,1) has room
+    k = rng.integers(0, 1 << 16, size=(L, Hkv, 10, D), dtype=np.uint16) & 0x3FFF
+    v = rng.integers(0, 1 << 16, size=(L, Hkv, 10, D), dtype=np.uint16) & 0x3FFF
+    pos = rng.integers(0, 100, size=(L, Hkv, 10), dtype=np.int32)
+    kn = rng.integers(0, 1 << 16, size=(L, Hkv, 2, D), dtype=np.uint16) & 0x3FFF
+    vn = rng.integers(0, 1 << 16, size=(L, Hkv, 2, D), dtype=np.uint16) & 0x3FFF
+    k2, v2, pos2, ul2, cp, skipped = oracle.append(k, v, pos, starts, None, cur, kn, vn, unit_len=ul)
+    assert skipped == [1] and cp.tolist() == [41, 70]     # segment 1 holds 4 slots; unit (0,0,1) full
+    assert ul2.tolist() == [[[4, 4], [6, 2]]]
+    for g in range(2):
+        slot = ul[0, g, 0]
+        np.testing.assert_array_equal(k2[0, g, slot], kn[0, g, 0])
+        assert pos2[0, g, slot] == 41
+    q = rng.integers(0, 1 << 16, size=(2, 4, D), dtype=np.uint16) & 0x3FFF
+    out = oracle.decode_attention(k2, v2, starts, None, 0, q, 0.3, unit_len=ul2)
+    for b in range(2):
+        for h in range(4):
+            g = h // 2
+            T = ul2[0, g, b]
+            one = oracle.decode_attention(k2[:, g:g + 1], v2[:, g:g + 1], starts, [T if bb == b else 0 for bb in range(2)],
+                                          0, q[:, h:h + 1], 0.3)
+            np.testing.assert_allclose(out[b, h], one[b, 0], rtol=1e-12, atol=0)

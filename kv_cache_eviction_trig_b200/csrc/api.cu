@@ -45,7 +45,7 @@ WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap
   w.max_slots = score_grid(cfg, seq_start).max_slots;
   w.err = kWsErr;
   size_t o = kWsPrefix;
-  w.seqlen = o;   o = align_up(o + 4ull * cfg.batch, 256);
+  w.seqlen = o;   o = align_up(o + 4ull * (units > (size_t)cfg.batch ? units : cfg.batch), 256);
   w.w = o;        o = align_up(o + 4ull * units * (F / 2) * G * 6, 256);
   w.raw = o;      o = align_up(o + 4ull * cfg.num_layers * cfg.n_q_heads * (size_t)cap, 256);
   w.sel = o;      o = align_up(o + 4ull * units * cfg.budget, 256);
@@ -123,7 +123,12 @@ tria_status check_config(const tria_config *cfg, bool scoring) {
 
 tria_status check_cache(const tria_config *cfg, const tria_cache *c, bool need_kv) {
   if (!c) return TRIA_ERR_INVALID_ARG;
-  if (!c->seq_start || !c->seq_len || c->cap_total < 0) return TRIA_ERR_INVALID_ARG;
+  if (!c->seq_start || c->cap_total < 0) return TRIA_ERR_INVALID_ARG;
+  // lengths per sequence, or per unit (then seq_len may be null); head budgets need the latter
+  if (!c->seq_len && !c->unit_len) return TRIA_ERR_INVALID_ARG;
+  if (c->unit_len && !aligned(c->unit_len, 4)) return TRIA_ERR_INVALID_ARG;
+  if (cfg->head_budgets && (!c->unit_len || !aligned(cfg->head_budgets, 4)))
+    return TRIA_ERR_INVALID_ARG;
   if (need_kv) {
     if (!c->k || !c->v || !c->pos) return TRIA_ERR_INVALID_ARG;
     if (!aligned(c->k, 16) || !aligned(c->v, 16) || !aligned(c->pos, 16))
@@ -172,6 +177,8 @@ void fill_fold(FoldParams &fp, const tria_config *cfg, const tria_stats *st,
   std::memset(&fp, 0, sizeof fp);
   fp.cur_pos = c->cur_pos;
   fp.seq_len = c->seq_len;
+  fp.unit_len = c->unit_len;
+  fp.units = (int64_t)cfg->num_layers * cfg->n_kv_heads * cfg->batch;
   fp.seqlen_snap = seqlen_snap;
   fp.err = err;
   fp.centre = reinterpret_cast<const float2 *>(st->centre);
@@ -202,6 +209,10 @@ cudaError_t fill_score(ScoreParams &sp, const tria_config *cfg, const tria_cache
   const int ch = sg.chunk_keys;
   sp.w = w;
   sp.seq_len = c->seq_len;
+  sp.unit_len = c->unit_len;
+  sp.head_budget = cfg->head_budgets;
+  sp.budget = cfg->budget;
+  sp.window = cfg->prune_window;
   sp.raw = raw;
   sp.partials = partials;
   sp.max_slots = sg.max_slots;
@@ -255,6 +266,9 @@ void fill_unit(UnitParams &up, const tria_config *cfg, const tria_cache *c, int 
   up.D = cfg->head_dim;
   up.budget = cfg->budget;
   up.prune_from = prune_from(cfg);
+  up.unit_mode = c->unit_len != nullptr;
+  up.head_budget = cfg->head_budgets;
+  up.window = cfg->prune_window;
   up.mode = mode;
   int64_t most = 0;
   for (int b = 0; b <= cfg->batch; ++b) {
@@ -328,6 +342,8 @@ cudaError_t fill_prune(PruneParams &pp, const tria_config *cfg, const tria_stats
   pp.v = static_cast<uint8_t *>(c->v);
   pp.pos = c->pos;
   pp.seq_len = c->seq_len;
+  pp.unit_len = c->unit_len;
+  pp.head_budget = cfg->head_budgets;
   pp.cur_pos = c->cur_pos;
   pp.centre = reinterpret_cast<const float2 *>(st->centre);
   pp.mean_norm = st->mean_norm;
@@ -467,7 +483,7 @@ tria_status tria_select(const tria_config *cfg, const tria_cache *cache, const f
   fill_unit(up, cfg, cache, kModeSelect);
   up.score = const_cast<float *>(score);
   up.sel = sel;
-  up.seqlen = cache->seq_len;
+  up.seqlen = cache->unit_len ? cache->unit_len : cache->seq_len;
   up.err = w.err();
   return cuda_status(launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch,
                                  static_cast<cudaStream_t>(stream), false));
@@ -484,7 +500,7 @@ tria_status tria_compact(const tria_config *cfg, const tria_cache *cache, const 
   UnitParams up;
   fill_unit(up, cfg, cache, kModeCompact);
   up.sel = const_cast<int32_t *>(sel);
-  up.seq_len_out = cache->seq_len;
+  up.seq_len_out = cache->unit_len ? cache->unit_len : cache->seq_len;
   up.err = w.err();
   return cuda_status(launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch,
                                  static_cast<cudaStream_t>(stream), false));
@@ -508,6 +524,7 @@ tria_status tria_append(const tria_config *cfg, const tria_cache *cache, const v
   ap.v = static_cast<uint8_t *>(cache->v);
   ap.pos = cache->pos;
   ap.seq_len = cache->seq_len;
+  ap.unit_len = cache->unit_len;
   ap.cur_pos = cache->cur_pos;
   ap.err = w.err();
   ap.cap = cache->cap_total;
@@ -538,6 +555,7 @@ tria_status tria_decode_attention(const tria_config *cfg, const tria_cache *cach
   ap.k = static_cast<const uint16_t *>(cache->k);
   ap.v = static_cast<const uint16_t *>(cache->v);
   ap.seq_len = cache->seq_len;
+  ap.unit_len = cache->unit_len;
   ap.out = out;
   ap.err = w.err();
   ap.cap = cache->cap_total;
@@ -610,7 +628,7 @@ tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
   up.sel = sel_out ? sel_out : w.sel();
   up.write_short_sel = sel_out ? 1 : 0;
   up.seqlen = w.seqlen();
-  up.seq_len_out = cache->seq_len;
+  up.seq_len_out = cache->unit_len ? cache->unit_len : cache->seq_len;
   up.err = w.err();
   if (!mark(kStageUnit)) return TRIA_ERR_CUDA;
   if (launch_unit(up, cfg->num_layers * cfg->n_kv_heads * cfg->batch, st, pdl) != cudaSuccess)

@@ -3,7 +3,8 @@
 // dimensionstp.github.io review, section 6, Limitations: in serving the pruned
 // cache meets the attention kernel).  One new query token per sequence; for each
 // query head h of KV head g = h / G
-//   out[b][h] = sum_t softmax_t(scale * q[b][h] . k_t) v_t,  t < seq_len[b].
+//   out[b][h] = sum_t softmax_t(scale * q[b][h] . k_t) v_t,  t < seq_len[b]
+// (or t < the unit's own length, when the cache has per-unit lengths).
 // The cache holds post-RoPE keys, so the (non-contiguous) positions of the
 // surviving keys play no part.
 //
@@ -50,9 +51,9 @@ __global__ void __cluster_dims__(kAttnCluster, 1, 1) __launch_bounds__(kAttnThre
   const int b = unit / p.Hkv, g = unit - b * p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t cap_b = p.seg_start[b + 1] - p.seg_start[b];
-  const int32_t T = p.seq_len[b];
+  const int32_t T = p.unit_len ? p.unit_len[((int64_t)p.layer * p.Hkv + g) * p.B + b] : p.seq_len[b];
   if (T < 0 || (int64_t)T > cap_b) {  // the same decision in every CTA of the cluster
-    if (r == 0 && tid == 0 && g == 0) dev::set_error(p.err, TRIA_DEVERR_SEQ_LEN);
+    if (r == 0 && tid == 0 && (g == 0 || p.unit_len)) dev::set_error(p.err, TRIA_DEVERR_SEQ_LEN);
     return;
   }
   const int t0 = (int)((int64_t)T * r / kAttnCluster), t1 = (int)((int64_t)T * (r + 1) / kAttnCluster);

@@ -270,6 +270,10 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
   const int64_t seg = p.seg_start[b];
   const int64_t seg_cap = p.seg_start[b + 1] - seg;
   const int tid = threadIdx.x, nthr = blockDim.x;
+  // keys this unit keeps (a head budget, or the single budget; p.budget is also the
+  // length of every selection list), and whether the unit's budget is valid
+  const int32_t bud = p.head_budget ? p.head_budget[row] : p.budget;
+  const bool bud_ok = bud >= 1 && bud <= p.budget;
 
   extern __shared__ __align__(128) uint8_t smem[];
   Ctl &c = *reinterpret_cast<Ctl *>(smem);
@@ -321,12 +325,13 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       kept = min(kept, c.peer[q][0]);
       any_bad |= c.peer[q][1];
     }
-    if (any_bad) {
-      if (r == 0 && tid == 0) dev::set_error(p.err, TRIA_DEVERR_SELECTION);
+    if (any_bad || !bud_ok || kept > bud) {
+      if (r == 0 && tid == 0)
+        dev::set_error(p.err, any_bad || bud_ok ? TRIA_DEVERR_SELECTION : TRIA_DEVERR_BUDGET);
       return;
     }
   } else {
-    const int32_t T = p.seqlen[b];  // issued first: the loads below do not need it
+    const int32_t T = p.seqlen[p.unit_mode ? unit : b];  // issued first: the loads below do not need it
     if (zmodes) {
       // The score kernel left, per (CTA slot, warp), float64 sums of s and s^2 of the
       // unit's keys; every CTA of the cluster adds them in the same fixed order
@@ -351,7 +356,11 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       return;  // same decision in every CTA of the cluster
     }
     const bool selects = (p.mode == kModeSelect || p.mode == kModePrune);
-    if (selects && T <= p.budget) {
+    if (selects && !bud_ok) {
+      if (r == 0 && tid == 0) dev::set_error(p.err, TRIA_DEVERR_BUDGET);
+      return;
+    }
+    if (selects && T <= bud) {
       // sequence at or under budget: every slot is kept, nothing moves
       if (p.mode == kModeSelect || p.write_short_sel) {
         const int64_t j0 = (int64_t)p.budget * r / CL, j1 = (int64_t)p.budget * (r + 1) / CL;
@@ -359,8 +368,8 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       }
       return;
     }
-    // held back by the prune window: the sequence is left as it is
-    if (p.mode == kModePrune && T < p.prune_from) return;
+    // held back by the prune window: the unit is left as it is
+    if (p.mode == kModePrune && (int64_t)T < (int64_t)bud + (p.window > 1 ? p.window : 1)) return;
     if (T == 0) return;
     const int64_t lo = (int64_t)T * r / CL, hi = (int64_t)T * (r + 1) / CL;
     const int n = (int)(hi - lo);
@@ -472,7 +481,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     }
     cl.sync();  // every CTA's first-round histogram is complete
     uint32_t prefix = 0, mask = 0, bin0 = 0;
-    int krem = p.budget, bucket = 0;
+    int krem = bud, bucket = 0;
     int top = fine ? 32 : 20;  // bits below `top` are not fixed by prefix/mask
     {
       // coarse bin holding the krem-th largest key, then its fine bin
@@ -655,7 +664,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     // CTA q keeps its keys above the bucket, its bucket keys above thr, and those
     // of its keys equal to thr whose cluster-wide rank in slot order is < k_eq.
     // Destination share of each CTA when the unit is compacted in one batch.
-    const int per = (p.budget + CL - 1) / CL;
+    const int per = (bud + CL - 1) / CL;
     const bool balanced_fit = p.mode == kModePrune &&
                               per <= (int)min((size_t)kOwnRows, data_bytes / (2 * (size_t)ROW + 4));
     if (tid < 32) {
@@ -725,7 +734,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
         const bool keep = in && (key > thr || (is_eq && er + __popc(eqm & below) < k_eq));
         const uint32_t km = __ballot_sync(0xffffffffu, keep);
         const int oi = o + __popc(km & below);
-        if (keep && oi < p.budget) {
+        if (keep && oi < bud) {
           const int32_t slot = (int32_t)(lo + i);
           sel[oi] = slot;
           if (balanced) c.kept_src[oi - c.bc[4]] = slot;  // read by the compacting CTAs
@@ -734,12 +743,16 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
         er += __popc(eqm);
       }
     }
+    // a head budget below the list length leaves the rest of the list empty
+    for (int64_t j = bud + (int64_t)(p.budget - bud) * r / CL + tid;
+         j < bud + (int64_t)(p.budget - bud) * (r + 1) / CL; j += nthr)
+      sel[j] = -1;
     cl.sync();  // selection lists complete and visible; peers' keys are no longer read
     if (p.mode == kModeSelect) return;
     if (balanced) {
       // ------------------------------------- one batch: this CTA's share of destinations
       const int j0 = r * per;
-      const int m = max(0, min(per, p.budget - j0));
+      const int m = max(0, min(per, bud - j0));
       for (int jj = tid; jj < m; jj += nthr) {
         const int j = j0 + jj;
         int q = 0;  // the peer whose kept keys include output index j
@@ -761,10 +774,13 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       }
       for (int jj = tid; jj < m; jj += nthr) pg[j0 + jj] = sp[jj];
       if (tid == 0) bulk_wait_read0();  // shared memory stays valid until the copies read it
-      if (r == 0 && tid == 0 && l == 0 && g == 0) p.seq_len_out[b] = p.budget;
+      if (r == 0 && tid == 0) {
+        if (p.unit_mode) p.seq_len_out[unit] = bud;
+        else if (l == 0 && g == 0) p.seq_len_out[b] = bud;
+      }
       return;
     }
-    kept = p.budget;
+    kept = bud;
   }
 
   // -------------------------------------------------------------- batched compaction
@@ -803,7 +819,10 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     if (tid == 0) bulk_wait_read0();  // the staging buffers may be reused by the next batch
     __syncthreads();
   }
-  if (r == 0 && tid == 0 && l == 0 && g == 0) p.seq_len_out[b] = kept;
+  if (r == 0 && tid == 0) {
+    if (p.unit_mode) p.seq_len_out[unit] = kept;
+    else if (l == 0 && g == 0) p.seq_len_out[b] = kept;
+  }
 }
 
 // Launch configuration: 8-CTA clusters of 1024 threads, one CTA per SM

@@ -275,7 +275,7 @@ tria_status tria_get_device_error(const void *ws, int32_t *code, void *stream);
  * tria_prune, but the workspace is a fixed array of TRIA_NOALLOC_SCRATCH_BYTES
  * inside the library's device image; the call allocates nothing.
  *   - Problems whose tria_workspace_size exceeds TRIA_NOALLOC_SCRATCH_BYTES
- *     return TRIA_ERR_UNSUPPORTED before anything is launched (16 MiB holds,
+ *     return TRIA_ERR_UNSUPPORTED before anything is launched (32 MiB holds,
  *     for example, one layer of 32 query heads over 32768 cached slots).
  *   - CUDA loads the part of the library that holds the array lazily: the
  *     first call on a device (with that device current) looks up the array's
@@ -292,7 +292,7 @@ tria_status tria_get_device_error(const void *ws, int32_t *code, void *stream);
  *     device error word (TRIA_DEVERR_* bits, 0 if none) at the end of the call,
  *     in stream order; the scratch cannot be passed to tria_get_device_error.
  */
-#define TRIA_NOALLOC_SCRATCH_BYTES (16 << 20)
+#define TRIA_NOALLOC_SCRATCH_BYTES (32 << 20)
 tria_status tria_prune_noalloc(const tria_config *cfg, const tria_stats *stats,
                                const tria_cache *cache, int32_t *sel_out, int32_t *device_error,
                                void *stream);

@@ -57,13 +57,18 @@ WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap
   if (pl.ok) {
     const size_t nc = (size_t)pl.ncta, ug = (size_t)pl.ug, rowb = 2ull * cfg.head_dim;
     o = kWsPrefix;
+    w.f_ea = o;        o = align_up(o + 16ull * cfg.batch * F, 256);
+    w.f_w = o;         o = align_up(o + 4ull * units * (F / 2) * G * 6, 256);
     w.f_raw = o;       o = align_up(o + 2ull * nc * pl.range_keys * G * 4, 256);
-    w.f_partial = o;   o = align_up(o + 2ull * nc * pl.range_units * G * 16, 256);
+    w.f_csum = o;      o = align_up(o + 2ull * nc * (pl.range_keys / pl.chunk_keys) * G * 16, 256);
+    w.f_partial = o;   o = align_up(o + 2ull * nc * ug * G * 16, 256);
     w.f_zk = o;        o = align_up(o + 2ull * (size_t)pl.zk_stride * 4, 256);
     w.f_bucket = o;    o = align_up(o + 2ull * ug * kPruneBucketMax * 8, 256);
     w.f_above = o;     o = align_up(o + 2ull * ug * nc * 4, 256);
     w.f_thr = o;       o = align_up(o + 2ull * ug * 8, 256);
     w.f_kcount = o;    o = align_up(o + 2ull * ug * nc * 4, 256);
+    w.f_klist = o;     o = align_up(o + ug * (size_t)cfg.budget * 4, 256);
+    w.f_khaz = o;      o = align_up(o + 2ull * kPruneMaxGroupUnits * 4, 256);
     w.f_stage_k = o;   o = align_up(o + ug * (size_t)cfg.budget * rowb, 256);
     w.f_stage_v = o;   o = align_up(o + ug * (size_t)cfg.budget * rowb, 256);
     w.f_stage_pos = o; o = align_up(o + ug * (size_t)cfg.budget * 4, 256);
@@ -353,13 +358,18 @@ cudaError_t fill_prune(PruneParams &pp, const tria_config *cfg, const tria_stats
   pp.sync = reinterpret_cast<int32_t *>(ws + kWsSync);
   pp.bcount = reinterpret_cast<int32_t *>(ws + kWsBcount);
   pp.hist = reinterpret_cast<uint32_t *>(ws + kWsHist);
+  pp.ea = reinterpret_cast<double2 *>(ws + lay.f_ea);
+  pp.w = reinterpret_cast<float *>(ws + lay.f_w);
   pp.raw = reinterpret_cast<float *>(ws + lay.f_raw);
+  pp.csum = reinterpret_cast<double *>(ws + lay.f_csum);
   pp.partial = reinterpret_cast<double *>(ws + lay.f_partial);
   pp.zk = reinterpret_cast<uint32_t *>(ws + lay.f_zk);
   pp.bucket = reinterpret_cast<unsigned long long *>(ws + lay.f_bucket);
   pp.above = reinterpret_cast<int32_t *>(ws + lay.f_above);
   pp.thr = reinterpret_cast<unsigned long long *>(ws + lay.f_thr);
   pp.kcount = reinterpret_cast<int32_t *>(ws + lay.f_kcount);
+  pp.klist = reinterpret_cast<int32_t *>(ws + lay.f_klist);
+  pp.khaz = reinterpret_cast<int32_t *>(ws + lay.f_khaz);
   pp.stage_k = ws + lay.f_stage_k;
   pp.stage_v = ws + lay.f_stage_v;
   pp.stage_pos = reinterpret_cast<int32_t *>(ws + lay.f_stage_pos);
@@ -380,6 +390,7 @@ cudaError_t fill_prune(PruneParams &pp, const tria_config *cfg, const tria_stats
   pp.cpr = pl.cpr;
   pp.range_keys = pl.range_keys;
   pp.range_units = pl.range_units;
+  pp.range_chunks = pl.range_keys / pl.chunk_keys;
   int32_t acc = 0;
   for (int b = 0; b <= cfg->batch; ++b) {
     pp.seg_start[b] = c->seq_start[b];

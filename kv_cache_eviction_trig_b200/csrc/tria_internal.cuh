@@ -19,8 +19,8 @@ namespace tria {
 // two share the same bytes.
 constexpr size_t kWsErr = 0;
 constexpr size_t kWsSync = 256;
-constexpr size_t kWsBcount = 512;
-constexpr size_t kWsHist = 1024;
+constexpr size_t kWsBcount = 256 + 16 * 128;  // after kSyncWords lines of 128 bytes
+constexpr size_t kWsHist = 4096;
 constexpr size_t kWsPrefix = kWsHist + 2ull * 32 * 4096 * 4;  // 2 slots x 32 units x 4096 bins
 
 struct WsLayout {
@@ -33,8 +33,8 @@ struct WsLayout {
   int32_t max_slots;
   // fused prune kernel (same bytes as the regions above)
   int fused;        // the fused kernel runs this problem's prune
-  size_t f_raw, f_partial, f_zk, f_bucket, f_above, f_thr, f_kcount, f_stage_k, f_stage_v,
-      f_stage_pos;
+  size_t f_ea, f_w, f_raw, f_csum, f_partial, f_zk, f_bucket, f_above, f_thr, f_kcount, f_klist,
+      f_khaz, f_stage_k, f_stage_v, f_stage_pos;
   size_t total;
 };
 WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap_total);
@@ -153,13 +153,15 @@ struct UnitParams {
 constexpr int kPruneConsumerWarps = 8;
 constexpr int kPruneSelectWarps = 4;
 constexpr int kPruneThreads = (kPruneConsumerWarps + 1 + kPruneSelectWarps) * 32;
-constexpr int kPruneRangeKeys = 2048;  // keys of one CTA's share of a group, at most
+constexpr int kPruneRangeKeys = 8192;  // keys of one CTA's share of a group, at most (fewer for G > 4)
 constexpr int kPruneHistBins = 4096;   // bins of a unit's z histogram (1/256 over [-8, 8))
 constexpr int kPruneBucketMax = 4096;  // threshold-bin keys gathered by every CTA
 constexpr int kPruneMaxGroupUnits = 32;
-// sync words (int32) at the start of the persistent prefix of the workspace
+// sync words (int32) at the start of the persistent prefix of the workspace, each on
+// its own 128-byte line (word w at int offset w * kSyncStride): every CTA polls them
 enum PruneSync : int { kSyncA = 0, kSyncB = 2, kSyncC = 4, kSyncD = 6, kSyncExit = 8,
-                       kSyncAbort = 9, kSyncWords = 16 };
+                       kSyncAbort = 9, kSyncP1 = 10, kSyncP2 = 11, kSyncE = 12, kSyncWords = 16 };
+constexpr int kSyncStride = 32;
 
 struct alignas(64) PruneParams {
   CUtensorMap tmap;           // K as [L*Hkv*cap][D] bf16, 128-byte swizzled boxes
@@ -177,19 +179,24 @@ struct alignas(64) PruneParams {
   int32_t *sync;              // kSyncWords
   int32_t *bcount;            // [2][kPruneMaxGroupUnits] bucket fill counters (zero at rest)
   uint32_t *hist;             // [2][kPruneMaxGroupUnits][kPruneHistBins] (zero at rest)
+  double2 *ea;                // [B][F] e^{i w_f cur_b} * mean_delta e^{i w_f delta} (prologue)
+  float *w;                   // [U][F/2][G][6] folded weights of every unit (prologue)
   float *raw;                 // [2][ncta][range_keys][G]
-  double *partial;            // [2][ncta][range_units][G][2]
+  double *csum;               // [2][ncta][range_chunks][G][2] per-chunk sums of s, s^2 (consumers)
+  double *partial;            // [2][ncta][ug][G][2] per CTA and unit of the group
   uint32_t *zk;               // [2][zk_stride] z keys of a group, by chunk position
   unsigned long long *bucket; // [2][ug][kPruneBucketMax] (key << 18 | ~slot) of threshold bins
   int32_t *above;             // [2][ug][ncta] per covering CTA: keys above the threshold bin
   unsigned long long *thr;    // [2][ug] threshold key of an exactly selected unit
   int32_t *kcount;            // [2][ug][ncta] per covering CTA: kept keys (exact path)
+  int32_t *klist;             // [ug][budget] kept slots of every unit of a group, by destination
+  int32_t *khaz;              // [2][kPruneMaxGroupUnits] kept slots below the unit's budget
   uint8_t *stage_k, *stage_v; // [ug][budget] rows
   int32_t *stage_pos;         // [ug][budget]
   int64_t cap;
   int64_t zk_stride;
   int32_t L, Hkv, Hq, B, budget, window, write_short_sel, flags;
-  int32_t units, ug, ngroups, ncta, cpr, range_keys, range_units;
+  int32_t units, ug, ngroups, ncta, cpr, range_keys, range_units, range_chunks;
   int64_t seg_start[TRIA_MAX_BATCH + 1];
   int32_t chunk_prefix[TRIA_MAX_BATCH + 1];
   double omega[128];          // w_f = theta^(-2f/D)
@@ -313,6 +320,24 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *map, int32_t 
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// An L2 policy that evicts the lines it tags first (for data read once, so that it
+// does not push out scratch that is read again).
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// tma_load_2d with an L2 cache policy.
+__device__ __forceinline__ void tma_load_2d_hint(void *dst, const void *map, int32_t x, int32_t y,
+                                                 uint64_t *bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(pol)
       : "memory");
 }
 

@@ -32,7 +32,7 @@ MAX_BATCH = 256
 MAX_OFFSETS = 4096
 MAX_SEGMENT = 1 << 18
 PRUNE_MAX_STAGES = 8
-NOALLOC_SCRATCH_BYTES = 16 << 20
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 DEVERR_SEQ_LEN = 1
 DEVERR_SELECTION = 2

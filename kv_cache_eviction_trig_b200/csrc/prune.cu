@@ -164,8 +164,9 @@ __device__ bool grid_round(const PruneParams &p, SwMisc &ms, int w, int g, int t
   if (t == 0) {
     int32_t *ctr = sync_word(p, w + (g & 1));
     const int32_t target = p.ncta * ((g >> 1) + 1);
-    __threadfence();
-    atomicAdd(ctr, 1);
+    // a release add: the select threads' writes (ordered before it by the barrier
+    // above) are visible to every CTA whose acquiring poll sees the count
+    asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(ctr) : "memory");
     bool ok = false;
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 0;; ++i) {
@@ -179,7 +180,6 @@ __device__ bool grid_round(const PruneParams &p, SwMisc &ms, int w, int g, int t
         }
       }
     }
-    __threadfence();
     ms.ok = ok;
   }
   sw_sync();
@@ -468,7 +468,7 @@ __device__ __forceinline__ int warp_sum_scatter(double (&v)[NV], int lane) {
 
 // ------------------------------------------------------------------ compaction helpers
 constexpr int kCopyPiece = 4096;  // destinations per pass (two int lists in the 32 KB area)
-constexpr int kCopyBatch = 16;    // 16-byte loads per thread in flight
+constexpr int kCopyRows = 8;      // row steps per warp in flight
 
 // Loads kept-list entries [q0, q0 + n) into ksh and lists in mv (any order) the
 // destinations that move: src != j, and with hazards_only also src < lim (a kept row
@@ -499,46 +499,55 @@ __device__ int gather_moves(SwMisc &ms, const int32_t *klg, int q0, int n, int l
 }
 
 // Copies the nm listed rows: destination q0 + j takes row ksh[j] of the unit (or its
-// staged copy), K and V as 16-byte vectors and the position as one int32.
+// staged copy).  A row's K and V are 2 * ROWB / 16 vectors of 16 bytes; a warp moves
+// RPW rows per step (VPL vectors per lane), kCopyRows steps with every load in flight
+// before the first store; the row's first lane moves its position.
 template <int ROWB>
-__device__ __noinline__ void copy_rows(const PruneParams &p, SwMisc &ms, const int32_t *ksh, const int32_t *mv,
-                          int nm, int q0, int64_t base, int bud, int ug_i, bool from_stage,
-                          bool to_stage, int t) {
-  constexpr int VPR = ROWB / 16;        // vectors per K (or V) row
-  constexpr int VR = 2 * VPR + 1;       // + one slot for the position
+__device__ __noinline__ void copy_rows(const PruneParams &p, const int32_t *ksh, const int32_t *mv,
+                                       int nm, int q0, int64_t base, int bud, int ug_i,
+                                       bool from_stage, bool to_stage, int t) {
+  constexpr int VPR = ROWB / 16;                 // vectors per K (or V) row
+  constexpr int VT = 2 * VPR;                    // K and V
+  constexpr int RPW = VT >= 32 ? 1 : 32 / VT;    // rows per warp step
+  constexpr int VPL = VT >= 32 ? VT / 32 : 1;    // vectors per lane per row
+  constexpr int LPR = 32 / RPW;                  // lanes per row
+  const int lane = t & 31, wid = t >> 5;
+  const int rsub = lane / LPR, lr = lane - rsub * LPR;
   const size_t st0 = (size_t)ug_i * p.budget;
-  const int nv = nm * VR;
-  for (int w0 = t; w0 < nv; w0 += SWT * kCopyBatch) {
-    uint4 a[kCopyBatch];
+  for (int r0 = wid * RPW * kCopyRows; r0 < nm; r0 += NSW * RPW * kCopyRows) {
+    uint4 a[kCopyRows][VPL];
+    int32_t ps[kCopyRows];
 #pragma unroll
-    for (int q = 0; q < kCopyBatch; ++q) {
-      const int w = w0 + q * SWT;
-      if (w < nv) {
-        const int r = w / VR, x = w - r * VR;
+    for (int u = 0; u < kCopyRows; ++u) {
+      const int r = r0 + u * RPW + rsub;
+      if (r < nm) {
         const int j = mv[r], src = ksh[j], d = q0 + j;
         const bool stg = from_stage && src < bud;
-        if (x < 2 * VPR) {
-          const uint8_t *rowp = stg ? (x < VPR ? p.stage_k : p.stage_v) + (st0 + d) * ROWB
-                                    : (x < VPR ? p.k : p.v) + (size_t)(base + src) * ROWB;
-          a[q] = __ldcg(reinterpret_cast<const uint4 *>(rowp) + (x < VPR ? x : x - VPR));
-        } else {
-          a[q].x = (uint32_t)__ldcg(stg ? p.stage_pos + st0 + d : p.pos + base + src);
+        const uint8_t *kr = stg ? p.stage_k + (st0 + d) * ROWB : p.k + (size_t)(base + src) * ROWB;
+        const uint8_t *vr = stg ? p.stage_v + (st0 + d) * ROWB : p.v + (size_t)(base + src) * ROWB;
+#pragma unroll
+        for (int e = 0; e < VPL; ++e) {
+          const int x = lr + e * LPR;  // vector of the row's K | V
+          a[u][e] = __ldcg(reinterpret_cast<const uint4 *>(x < VPR ? kr : vr) + (x < VPR ? x : x - VPR));
         }
+        if (lr == 0) ps[u] = __ldcg(stg ? p.stage_pos + st0 + d : p.pos + base + src);
       }
     }
 #pragma unroll
-    for (int q = 0; q < kCopyBatch; ++q) {
-      const int w = w0 + q * SWT;
-      if (w < nv) {
-        const int r = w / VR, x = w - r * VR;
+    for (int u = 0; u < kCopyRows; ++u) {
+      const int r = r0 + u * RPW + rsub;
+      if (r < nm) {
         const int d = q0 + mv[r];
-        if (x < 2 * VPR) {
-          uint8_t *rowp = to_stage ? (x < VPR ? p.stage_k : p.stage_v) + (st0 + d) * ROWB
-                                   : (x < VPR ? p.k : p.v) + (size_t)(base + d) * ROWB;
-          reinterpret_cast<uint4 *>(rowp)[x < VPR ? x : x - VPR] = a[q];
-        } else {
-          if (to_stage) p.stage_pos[st0 + d] = (int32_t)a[q].x;
-          else p.pos[base + d] = (int32_t)a[q].x;
+        uint8_t *kr = to_stage ? p.stage_k + (st0 + d) * ROWB : p.k + (size_t)(base + d) * ROWB;
+        uint8_t *vr = to_stage ? p.stage_v + (st0 + d) * ROWB : p.v + (size_t)(base + d) * ROWB;
+#pragma unroll
+        for (int e = 0; e < VPL; ++e) {
+          const int x = lr + e * LPR;
+          reinterpret_cast<uint4 *>(x < VPR ? kr : vr)[x < VPR ? x : x - VPR] = a[u][e];
+        }
+        if (lr == 0) {
+          if (to_stage) p.stage_pos[st0 + d] = ps[u];
+          else p.pos[base + d] = ps[u];
         }
       }
     }
@@ -1081,8 +1090,7 @@ __device__ __noinline__ void sel_stage(const PruneParams &p, uint8_t *swb, const
     // The kept slots below bud are the first Kh destinations (Kh from the range that
     // holds slot bud - 1), which 5a splits evenly too.
     // Both passes put the share's list in shared memory, gather the rows to move, and
-    // copy them as one flat run of 16-byte vectors (K and V of every row), with
-    // kCopyBatch independent loads per thread in flight before the stores.
+    // copy them with kCopyRows rows per warp in flight before the stores.
     for (int i = 0; i < nu; ++i) {  // 5a
       const UEnt e = utab[i];
       if (e.mode != kPruneU) continue;
@@ -1100,7 +1108,7 @@ __device__ __noinline__ void sel_stage(const PruneParams &p, uint8_t *swb, const
       for (int q0 = d0; q0 < d1; q0 += kCopyPiece) {
         const int n = min(kCopyPiece, d1 - q0);
         int nm = gather_moves(ms, klg, q0, n, e.bud, /*hazards_only=*/true, ksh, mv, t);
-        copy_rows<ROWB>(p, ms, ksh, mv, nm, q0, base, e.bud, ug_i, /*from_stage=*/false,
+        copy_rows<ROWB>(p, ksh, mv, nm, q0, base, e.bud, ug_i, /*from_stage=*/false,
                         /*to_stage=*/true, t);
       }
     }
@@ -1148,7 +1156,7 @@ __device__ __noinline__ void sel_write(const PruneParams &p, uint8_t *swb, const
         for (int q0 = d0; q0 < d1; q0 += kCopyPiece) {
           const int n = min(kCopyPiece, d1 - q0);
           int nm = gather_moves(ms, klg, q0, n, e.T, /*hazards_only=*/false, ksh, mv, t);
-          copy_rows<ROWB>(p, ms, ksh, mv, nm, q0, base, e.bud, ug_i, /*from_stage=*/true,
+          copy_rows<ROWB>(p, ksh, mv, nm, q0, base, e.bud, ug_i, /*from_stage=*/true,
                           /*to_stage=*/false, t);
         }
         if (c == e.clo) {

@@ -323,10 +323,10 @@ class Bench:
     before every step the rows a prune overwrites are restored from a pristine
     copy and L2 is flushed (512 MiB written); neither is timed."""
 
-    def __init__(self, wl, dev):
+    def __init__(self, wl, dev, flags=0):
         self.wl, self.dev = wl, dev
         data = workloads.generate(wl, device=dev)
-        self.cfg = tria.Config.from_workload(wl)
+        self.cfg = tria.Config.from_workload(wl, flags=flags)
         self.stats = tria.calibrate(self.cfg, data["q_calib"])
         del data["q_calib"]
         self.data = data
@@ -403,6 +403,8 @@ class Bench:
             out["prune_kernel_frac"] = algo / (kt / 1e3) / 1e9 / peak
             busy_ms = kt
         else:
+            ut = kern_ms[names.index("unit_kernel")]
+            out["unit_kernel_frac"] = (algo - keys * 2 * wl.head_dim) / (ut / 1e3) / 1e9 / peak
             kt = kern_ms[names.index("score_kernel")]
             out["score_kernel_frac"] = keys * 2 * wl.head_dim / (kt / 1e3) / 1e9 / peak
             busy_ms = kt
@@ -488,6 +490,8 @@ def run_ours(args):
     kern = names[dom]
     if kern == "prune_kernel":
         algo_launch = wl.algorithmic_bytes()  # the whole step: keys read, kept rows moved
+    elif kern == "unit_kernel":
+        algo_launch = wl.algorithmic_bytes() - keys * 2 * wl.head_dim  # kept rows moved
     else:
         algo_launch = keys * 2 * wl.head_dim  # the score kernel reads every key once
     achieved = algo_launch / (kern_ms[dom] / 1e3) / 1e9
@@ -526,13 +530,16 @@ def run_ours(args):
                  ("workload1_geometric", workloads.workload(1, offsets=geo,
                                                             name=workloads.workload(1).name + " geometric offsets 1..65536")),
                  ("workload2_geometric", workloads.workload(2, offsets=geo,
-                                                            name=workloads.workload(2).name + " geometric offsets 1..65536"))]
+                                                            name=workloads.workload(2).name + " geometric offsets 1..65536")),
+                 # the same prune as one persistent launch (TRIA_FUSED_PRUNE)
+                 ("workload1_fused", workloads.workload(1)),
+                 ("workload2_fused", workloads.workload(2))]
         for key, xwl in specs:
             if rank:
                 xwl = workloads.workload(int(key[8]), seed=xwl.seed + 1000 * rank,
                                          offsets=xwl.offsets, name=xwl.name)
             try:
-                xb = Bench(xwl, dev)
+                xb = Bench(xwl, dev, flags=tria.FUSED_PRUNE if key.endswith("_fused") else 0)
                 xb.warm(3)
                 with ClockSampler(local) as xclk:
                     xms = xb.timed(args.extra_steps)

@@ -70,6 +70,12 @@ typedef enum {
 
 #define TRIA_NO_TRIG 1u          /* ablation: score without the trigonometric term */
 #define TRIA_NO_CONC_WEIGHT 2u   /* ablation: norm term weighted by E|q_f| instead of (1-R_f)E|q_f| */
+/* tria_prune / tria_prune_noalloc as one persistent cooperative launch (every CTA scores
+   a share of each group of units, and grid rounds order the selection and compaction
+   steps) instead of the fold, score and unit kernels.  Same results; shapes that launch
+   cannot take run the default kernels.  Set the flag before tria_workspace_size: the
+   launch needs its own workspace regions. */
+#define TRIA_FUSED_PRUNE 4u
 
 #define TRIA_DTYPE_F32 0
 #define TRIA_DTYPE_BF16 1
@@ -98,7 +104,7 @@ typedef struct {
   int32_t budget;       /* keys kept per (layer, KV head, sequence) */
   const int32_t *offsets; /* HOST [n_offsets] future query offsets, each >= 1 */
   int32_t n_offsets;
-  uint32_t flags;       /* 0, or TRIA_NO_TRIG / TRIA_NO_CONC_WEIGHT */
+  uint32_t flags;       /* 0, or TRIA_NO_TRIG / TRIA_NO_CONC_WEIGHT / TRIA_FUSED_PRUNE */
   int32_t prune_window; /* >= 0.  tria_prune / tria_prune_noalloc prune a sequence only
                            once seq_len >= budget + max(prune_window, 1) (a decode loop
                            that calls tria_prune after every tria_append then prunes each
@@ -275,7 +281,7 @@ tria_status tria_get_device_error(const void *ws, int32_t *code, void *stream);
  * tria_prune, but the workspace is a fixed array of TRIA_NOALLOC_SCRATCH_BYTES
  * inside the library's device image; the call allocates nothing.
  *   - Problems whose tria_workspace_size exceeds TRIA_NOALLOC_SCRATCH_BYTES
- *     return TRIA_ERR_UNSUPPORTED before anything is launched (32 MiB holds,
+ *     return TRIA_ERR_UNSUPPORTED before anything is launched (16 MiB holds,
  *     for example, one layer of 32 query heads over 32768 cached slots).
  *   - CUDA loads the part of the library that holds the array lazily: the
  *     first call on a device (with that device current) looks up the array's
@@ -292,7 +298,7 @@ tria_status tria_get_device_error(const void *ws, int32_t *code, void *stream);
  *     device error word (TRIA_DEVERR_* bits, 0 if none) at the end of the call,
  *     in stream order; the scratch cannot be passed to tria_get_device_error.
  */
-#define TRIA_NOALLOC_SCRATCH_BYTES (32 << 20)
+#define TRIA_NOALLOC_SCRATCH_BYTES (16 << 20)
 tria_status tria_prune_noalloc(const tria_config *cfg, const tria_stats *stats,
                                const tria_cache *cache, int32_t *sel_out, int32_t *device_error,
                                void *stream);

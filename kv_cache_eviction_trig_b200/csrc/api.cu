@@ -52,7 +52,7 @@ WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap
   w.partials = o;
   o = align_up(o + 16ull * units * (size_t)w.max_slots * kScoreConsumerWarps * G, 256);
   size_t end = o;
-  const PrunePlan pl = prune_plan(cfg, seq_start);
+  const PrunePlan pl = (cfg.flags & TRIA_FUSED_PRUNE) ? prune_plan(cfg, seq_start) : PrunePlan{};
   w.fused = pl.ok;
   if (pl.ok) {
     const size_t nc = (size_t)pl.ncta, ug = (size_t)pl.ug, rowb = 2ull * cfg.head_dim;
@@ -117,7 +117,8 @@ tria_status check_config(const tria_config *cfg, bool scoring) {
     if (cfg->n_offsets > TRIA_MAX_OFFSETS) return TRIA_ERR_UNSUPPORTED;
     for (int i = 0; i < cfg->n_offsets; ++i)
       if (cfg->offsets[i] < 1) return TRIA_ERR_INVALID_ARG;
-    if (cfg->flags & ~(TRIA_NO_TRIG | TRIA_NO_CONC_WEIGHT)) return TRIA_ERR_INVALID_ARG;
+    if (cfg->flags & ~(TRIA_NO_TRIG | TRIA_NO_CONC_WEIGHT | TRIA_FUSED_PRUNE))
+      return TRIA_ERR_INVALID_ARG;
     if (!score_supported(cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads, cfg->rope_layout))
       return TRIA_ERR_UNSUPPORTED;
   } else {

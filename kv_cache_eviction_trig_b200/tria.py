@@ -26,13 +26,14 @@ ROPE_HALF_SPLIT = 0
 ROPE_INTERLEAVED = 1
 NO_TRIG = 1
 NO_CONC_WEIGHT = 2
+FUSED_PRUNE = 4
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
 MAX_BATCH = 256
 MAX_OFFSETS = 4096
 MAX_SEGMENT = 1 << 18
 PRUNE_MAX_STAGES = 8
-NOALLOC_SCRATCH_BYTES = 32 << 20
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 DEVERR_SEQ_LEN = 1
 DEVERR_SELECTION = 2

@@ -110,7 +110,7 @@ def test_workspace_size(L):
     (dict(offsets=[]), tria.ERR_INVALID_ARG),
     (dict(offsets=list(range(1, 5000))), tria.ERR_UNSUPPORTED),
     (dict(rope_layout=2), tria.ERR_INVALID_ARG),
-    (dict(flags=4), tria.ERR_INVALID_ARG),
+    (dict(flags=8), tria.ERR_INVALID_ARG),      # an unknown flag bit
     (dict(batch=300), tria.ERR_UNSUPPORTED),
     (dict(prune_window=-1), tria.ERR_INVALID_ARG),
 ])

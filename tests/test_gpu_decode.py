@@ -127,11 +127,13 @@ def test_append_matches_oracle():
     assert after["cur_pos"].tolist() == cp.tolist()
 
 
-def test_prune_window_matches_oracle():
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_prune_window_matches_oracle(fused):
     budget, W = 100, 40
     wl = small("window", B=4, seq_lens=[139, 140, 90, 500], budget=budget, slack=5)
     case = Case(wl)
-    cfg = tria.Config.from_workload(wl, prune_window=W)
+    cfg = tria.Config.from_workload(wl, prune_window=W, flags=tria.FUSED_PRUNE if fused else 0)
+    case.ws = tria.workspace(cfg, case.cache)
     before = _state(case)
     ref = oracle.prune_window(case.prob, before["v"], W)
     sel = torch.full((1, 2, 4, budget), -7, dtype=torch.int32, device="cuda")
@@ -142,7 +144,8 @@ def test_prune_window_matches_oracle():
     _check_windowed(case, W, before, _state(case), sel.cpu().numpy(), ref)
 
 
-def test_decode_loop_matches_oracle_and_its_cuda_graph():
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_decode_loop_matches_oracle_and_its_cuda_graph(fused):
     """40 decode steps (append, then the windowed prune) on three ragged
     sequences: every step against the oracle run from the GPU's state before it,
     and the same loop replayed from one captured CUDA graph ends bit-identical."""
@@ -150,7 +153,8 @@ def test_decode_loop_matches_oracle_and_its_cuda_graph():
     wl = small("decode", L=2, B=3, Hq=4, Hkv=2, D=64, theta=1e4, seq_lens=[40, 60, 63],
                budget=budget, slack=26, offsets=range(1, 33))
     a = Case(wl)
-    cfg = tria.Config.from_workload(wl, prune_window=W)
+    cfg = tria.Config.from_workload(wl, prune_window=W, flags=tria.FUSED_PRUNE if fused else 0)
+    a.ws = tria.workspace(cfg, a.cache)
     gen = torch.Generator().manual_seed(11)
     tokens, cur = [], a.host["cur_pos"].clone()
     for _ in range(steps):
@@ -179,6 +183,7 @@ def test_decode_loop_matches_oracle_and_its_cuda_graph():
     assert pruned_steps == 8  # sequences reach budget + W at steps 1, 4, 17, 20, 24, 33, 36, 40
 
     b = Case(wl)
+    b.ws = tria.workspace(cfg, b.cache)
     kbuf = torch.empty_like(tokens[0][0], device="cuda")
     vbuf = torch.empty_like(tokens[0][1], device="cuda")
     sel_b = torch.empty_like(sel_a)

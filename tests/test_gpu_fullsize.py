@@ -35,13 +35,14 @@ def _topk_slots(score, budget):
     return np.sort(order[:budget])
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
 @pytest.mark.parametrize("index,n_units,n_keys", [(1, 8, 48), (4, 4, 12), (2, 6, 24), (3, 6, 16)])
-def test_full_size_workload(index, n_units, n_keys):
+def test_full_size_workload(index, n_units, n_keys, fused):
     wl = workloads.workload(index)
     data = workloads.generate(wl, device="cuda")
     stats_np = common.stats_fp32(data["q_calib"], wl.rope_layout)
     del data["q_calib"]
-    cfg = tria.Config.from_workload(wl)
+    cfg = tria.Config.from_workload(wl, flags=tria.FUSED_PRUNE if fused else 0)
     cache = tria.Cache.from_data(data)
     stats = tria.Stats(*[torch.from_numpy(s).cuda() for s in stats_np])
     ws = tria.workspace(cfg, cache)
@@ -112,7 +113,8 @@ def test_full_size_workload(index, n_units, n_keys):
         assert torch.equal(data["pos"][l, g, s0:s0 + n], pp[idx])
 
 
-def test_whole_unit_of_the_8b_layer_matches_the_oracle_prune():
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_whole_unit_of_the_8b_layer_matches_the_oracle_prune(fused):
     """One whole (layer, KV head, sequence) unit of the 8B-shaped layer at 32K keys,
     pruned by tria_prune in the benchmark's launch configuration (all 8 KV heads in
     one call), against the oracle's prune of that unit: every raw score, the group
@@ -125,7 +127,7 @@ def test_whole_unit_of_the_8b_layer_matches_the_oracle_prune():
     data = workloads.generate(wl, device="cuda")
     stats_np = common.stats_fp32(data["q_calib"], wl.rope_layout)
     del data["q_calib"]
-    cfg = tria.Config.from_workload(wl)
+    cfg = tria.Config.from_workload(wl, flags=tria.FUSED_PRUNE if fused else 0)
     cache = tria.Cache.from_data(data)
     stats = tria.Stats(*[torch.from_numpy(s).cuda() for s in stats_np])
     ws = tria.workspace(cfg, cache)

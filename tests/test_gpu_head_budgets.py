@@ -3,10 +3,11 @@ compression refined with a budget per head) against the oracle.
 
 Every (layer, KV head) has its own budget and every (layer, KV head, sequence)
 unit its own live length (tria_cache.unit_len), as after an earlier prune with
-head budgets.  Checked through the fused prune, the separate select and compact
-calls (one 8-CTA cluster per unit and one CTA per unit), the three-kernel prune
-(head_dim 256 with 16 query heads per KV head), the decode-loop append and the
-decode attention.  Tolerances as in test_gpu_parity: selections by the
+head budgets.  Checked through both prune paths (the fold, score and unit
+kernels, and the single persistent launch), the separate select and compact calls
+(one 8-CTA cluster per unit and one CTA per unit), a shape the single launch does
+not take (head_dim 256 with 16 query heads per KV head), the decode-loop append
+and the decode attention.  Tolerances as in test_gpu_parity: selections by the
 threshold rule, compacted rows, lengths and selection lists of identical scores
 bit-exact."""
 import numpy as np
@@ -35,7 +36,7 @@ class HeadCase:
     """A drawn cache with per-unit lengths and per-head budgets, on the GPU and in
     the oracle's form."""
 
-    def __init__(self, wl, seed, budget_lo=1, len_lo=0.5, window=0, headroom=0):
+    def __init__(self, wl, seed, budget_lo=1, len_lo=0.5, window=0, headroom=0, fused=False):
         rng = np.random.default_rng(seed)
         self.wl = wl
         data = workloads.generate(wl)
@@ -52,7 +53,8 @@ class HeadCase:
         self.dev["budgets"] = torch.from_numpy(self.budgets.copy()).cuda()
         self.pristine = {k: self.dev[k].clone() for k in ("k", "v", "pos", "unit_len")}
         self.cfg = tria.Config.from_workload(wl, head_budgets=self.dev["budgets"],
-                                             prune_window=window)
+                                             prune_window=window,
+                                             flags=tria.FUSED_PRUNE if fused else 0)
         self.cache = tria.Cache(self.dev["k"], self.dev["v"], self.dev["pos"], None,
                                 self.dev["cur_pos"], self.host["seq_start"],
                                 unit_len=self.dev["unit_len"])
@@ -124,7 +126,7 @@ def _small(name, **kw):
     return workloads.custom(name, **d)
 
 
-FUSED = {
+SHAPES = {
     "g4": lambda: _small("hb-g4"),
     "g8_two_layers": lambda: _small("hb-g8", L=2, Hq=16, Hkv=2, seq_lens=[900, 2000, 50], B=3),
     "d64_interleaved": lambda: _small("hb-d64", D=64, theta=1e4, rope_layout=workloads.INTERLEAVED),
@@ -133,9 +135,10 @@ FUSED = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(FUSED))
-def test_prune_with_head_budgets_matches_oracle(name):
-    case = HeadCase(FUSED[name](), seed=len(name))
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+@pytest.mark.parametrize("name", sorted(SHAPES))
+def test_prune_with_head_budgets_matches_oracle(name, fused):
+    case = HeadCase(SHAPES[name](), seed=len(name), fused=fused)
     wl = case.wl
     ref = oracle.prune(case.prob, common.bf16_bits(case.host["v"]))
     sel = torch.full((wl.num_layers, wl.n_kv_heads, wl.batch, wl.budget), -7, dtype=torch.int32,
@@ -152,9 +155,10 @@ def test_prune_with_head_budgets_matches_oracle(name):
 
 def test_three_kernel_prune_with_head_budgets_matches_oracle():
     """head_dim 256 with 16 query heads per KV head runs the fold, score and unit
-    kernels instead of the fused one."""
+    kernels even when the single-launch prune is asked for (that launch does not
+    take this shape)."""
     case = HeadCase(_small("hb-d256g16", D=256, Hq=16, Hkv=1, seq_lens=[600, 300], budget=100),
-                    seed=3)
+                    seed=3, fused=True)
     wl = case.wl
     ref = oracle.prune(case.prob, common.bf16_bits(case.host["v"]))
     sel = torch.full((1, 1, 2, wl.budget), -7, dtype=torch.int32, device="cuda")
@@ -214,7 +218,8 @@ def test_head_budget_out_of_range_sets_flag_and_skips_the_head():
         np.testing.assert_array_equal(got[0, g], np.minimum(case.unit_len[0, g], bad[0, g]))
 
 
-def test_decode_loop_with_head_budgets_matches_oracle():
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_decode_loop_with_head_budgets_matches_oracle(fused):
     """Append a token to every sequence, then prune with a window, 12 times, with
     per-head budgets: lengths, cache and positions follow the oracle step by step
     (the selections are compared with the threshold rule, then the oracle continues
@@ -222,7 +227,7 @@ def test_decode_loop_with_head_budgets_matches_oracle():
     wl = _small("hb-loop", B=2, Hq=8, Hkv=2, seq_lens=[330, 310], budget=300, slack=40,
                 offsets=range(1, 9))
     W = 4
-    case = HeadCase(wl, seed=5, budget_lo=280, len_lo=0.9, window=W, headroom=1)
+    case = HeadCase(wl, seed=5, budget_lo=280, len_lo=0.9, window=W, headroom=1, fused=fused)
     gen = torch.Generator().manual_seed(0)
     L, Hkv, B, D = wl.num_layers, wl.n_kv_heads, wl.batch, wl.head_dim
     for step in range(12):

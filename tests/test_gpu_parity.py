@@ -39,7 +39,8 @@ def _lib():
 class Case:
     """One drawn workload on the GPU plus its oracle problem."""
 
-    def __init__(self, wl, flags=0, seq_len=None, gen_device="cpu", calib_on_gpu=False):
+    def __init__(self, wl, flags=0, seq_len=None, gen_device="cpu", calib_on_gpu=False,
+                 fused=False):
         self.wl = wl
         data = workloads.generate(wl, device=gen_device)
         self.stats_np = common.stats_fp32(data["q_calib"], wl.rope_layout)
@@ -48,7 +49,7 @@ class Case:
             self.host["seq_len"] = torch.tensor(seq_len, dtype=torch.int32)
         self.dev = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in self.host.items()}
         self.pristine = {k: self.dev[k].clone() for k in ("k", "v", "pos", "seq_len")}
-        self.cfg = tria.Config.from_workload(wl, flags=flags)
+        self.cfg = tria.Config.from_workload(wl, flags=flags | (tria.FUSED_PRUNE if fused else 0))
         self.cache = tria.Cache.from_data(self.dev)
         self.stats = tria.Stats(*[torch.from_numpy(s).cuda() for s in self.stats_np])
         self.ws = tria.workspace(self.cfg, self.cache)
@@ -304,9 +305,10 @@ def test_compact_many_units_multi_batch(kind, L, D, budget, T):
     check_compacted(case, sel, [budget])
 
 
-def test_prune_many_units_matches_oracle():
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_prune_many_units_matches_oracle(fused):
     case = Case(small("prune-multi", L=2, Hq=32, Hkv=8, B=1, seq_lens=[4000], budget=3500,
-                      offsets=range(1, 17)))
+                      offsets=range(1, 17)), fused=fused)
     wl = case.wl
     ref = oracle.prune(case.prob, common.bf16_bits(case.host["v"]))
     sel = torch.empty((wl.num_layers, wl.n_kv_heads, wl.batch, wl.budget), dtype=torch.int32,
@@ -335,8 +337,9 @@ def test_compact_rejects_malformed_selection():
 
 @pytest.mark.parametrize("name", ["tiny", "ragged2seq", "d64_interleaved", "g8", "two_layers",
                                   "g16_geometric"])
-def test_prune_matches_oracle(name):
-    case = Case(CASES[name]())
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_prune_matches_oracle(name, fused):
+    case = Case(CASES[name](), fused=fused)
     wl = case.wl
     ref = oracle.prune(case.prob, common.bf16_bits(case.host["v"]))
     sel = torch.full((wl.num_layers, wl.n_kv_heads, wl.batch, wl.budget), -7, dtype=torch.int32,
@@ -351,9 +354,10 @@ def test_prune_matches_oracle(name):
     check_compacted(case, gsel, kept)
 
 
-def test_prune_without_sel_out_equals_with():
-    a = Case(CASES["ragged2seq"]())
-    b = Case(CASES["ragged2seq"]())
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_prune_without_sel_out_equals_with(fused):
+    a = Case(CASES["ragged2seq"](), fused=fused)
+    b = Case(CASES["ragged2seq"](), fused=fused)
     wl = a.wl
     sel = torch.empty((wl.num_layers, wl.n_kv_heads, wl.batch, wl.budget), dtype=torch.int32,
                       device="cuda")
@@ -364,10 +368,11 @@ def test_prune_without_sel_out_equals_with():
         assert torch.equal(a.dev[n], b.dev[n])
 
 
-def test_prune_edge_lengths():
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_prune_edge_lengths(fused):
     """T = 0, T < budget, T = budget, T = budget + 1, and a long one, in one batch."""
     wl = small("edges", B=5, seq_lens=[0, 50, 100, 101, 900], budget=100, slack=3)
-    case = Case(wl)
+    case = Case(wl, fused=fused)
     ref = oracle.prune(case.prob, common.bf16_bits(case.host["v"]))
     sel = torch.empty((1, 2, 5, 100), dtype=torch.int32, device="cuda")
     tria.tria_prune(case.cfg, case.stats, case.cache, case.ws, sel_out=sel)
@@ -379,8 +384,9 @@ def test_prune_edge_lengths():
     check_compacted(case, gsel, [0, 50, 100, 100, 100])
 
 
-def test_prune_budget_one():
-    case = Case(small("b1", seq_lens=[333], budget=1))
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_prune_budget_one(fused):
+    case = Case(small("b1", seq_lens=[333], budget=1), fused=fused)
     ref = oracle.prune(case.prob, common.bf16_bits(case.host["v"]))
     sel = torch.empty((1, 2, 1, 1), dtype=torch.int32, device="cuda")
     tria.tria_prune(case.cfg, case.stats, case.cache, case.ws, sel_out=sel)
@@ -389,9 +395,10 @@ def test_prune_budget_one():
     check_compacted(case, sel.cpu().numpy(), [1])
 
 
-def test_seq_len_beyond_capacity_sets_flag_and_skips_sequence():
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_seq_len_beyond_capacity_sets_flag_and_skips_sequence(fused):
     wl = small("overflow", B=2, seq_lens=[300, 300], budget=50)
-    case = Case(wl, seq_len=[300, 301])      # sequence 1 claims more than its segment
+    case = Case(wl, seq_len=[300, 301], fused=fused)  # sequence 1 claims more than its segment
     case.cache = tria.Cache.from_data(case.dev)
     tria.tria_prune(case.cfg, case.stats, case.cache, case.ws)
     torch.cuda.synchronize()
@@ -402,9 +409,10 @@ def test_seq_len_beyond_capacity_sets_flag_and_skips_sequence():
     assert tria.tria_get_device_error(case.ws) == 0
 
 
-def test_repeated_prune_is_stable():
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_repeated_prune_is_stable(fused):
     """A second prune of an already pruned cache (T = budget) changes nothing."""
-    case = Case(CASES["ragged2seq"]())
+    case = Case(CASES["ragged2seq"](), fused=fused)
     tria.tria_prune(case.cfg, case.stats, case.cache, case.ws)
     torch.cuda.synchronize()
     snap = {n: case.dev[n].clone() for n in ("k", "v", "pos", "seq_len")}
@@ -416,11 +424,12 @@ def test_repeated_prune_is_stable():
 
 # Problems with more than 15 units run one CTA per unit instead of one 8-CTA cluster.
 
-def test_prune_edge_lengths_one_cta_per_unit():
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_prune_edge_lengths_one_cta_per_unit(fused):
     """40 units (L2 x Hkv4 x B5): T = 0, < budget, = budget, budget + 1 and long."""
     wl = small("edges-1cta", L=2, B=5, Hq=8, Hkv=4, seq_lens=[0, 50, 100, 101, 900], budget=100,
                slack=3)
-    case = Case(wl)
+    case = Case(wl, fused=fused)
     ref = oracle.prune(case.prob, common.bf16_bits(case.host["v"]))
     sel = torch.full((2, 4, 5, 100), -7, dtype=torch.int32, device="cuda")
     tria.tria_prune(case.cfg, case.stats, case.cache, case.ws, sel_out=sel)
@@ -507,12 +516,13 @@ def test_select_large_bucket_is_exact(pattern, L):
 
 
 @pytest.mark.parametrize("L", [1, 2])
-def test_prune_degenerate_groups_keep_the_lowest_slots(L):
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_prune_degenerate_groups_keep_the_lowest_slots(L, fused):
     """KV groups whose query heads all have zero centre and zero mean norm score
     every key 0, so sigma = 0 and z = 0 (the z-score reading for sigma = 0): every
     key ties and the prune keeps slots 0..budget-1.  The other groups are ordinary."""
     wl = small("degenerate", L=L, Hq=32, Hkv=8, seq_lens=[8192], budget=2048, offsets=[1, 2, 3])
-    case = Case(wl)
+    case = Case(wl, fused=fused)
     c, m, r = (np.array(x) for x in case.stats_np)
     G = wl.group
     dead = [0, 5]

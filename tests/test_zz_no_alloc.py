@@ -74,7 +74,7 @@ def test_prune_noalloc_matches_prune_on_consecutive_calls():
     build.build()
     problems = [
         _small("noalloc-ragged"),
-        workloads.workload(1),          # one 8B-shaped layer at 32K keys, about 21 MB of scratch
+        workloads.workload(1),          # one 8B-shaped layer at 32K keys, about 4.4 MB of scratch
         _small("noalloc-two-layers", L=2, B=3, seq_lens=[129, 400, 90], budget=128,
                offsets=range(1, 33), seed=5),
     ]

@@ -301,7 +301,8 @@ def _kernel_hash(names):
 
 
 KERNEL_SOURCES = {"prune_kernel": ("prune.cu", "score_math.cuh", "tria_internal.cuh"),
-                  "score_kernel": ("score.cu", "tria_internal.cuh")}
+                  "score_kernel": ("score.cu", "tria_internal.cuh"),
+                  "unit_kernel": ("unit.cu", "tria_internal.cuh")}
 
 
 def _traffic(kernel, key):

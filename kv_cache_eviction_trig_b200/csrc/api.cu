@@ -178,6 +178,43 @@ int32_t prune_from(const tria_config *cfg) {
   return t < INT32_MAX ? (int32_t)t : INT32_MAX;
 }
 
+// Mean over the offsets of e^{i w_f delta} for every RoPE pair (the part of the
+// trigonometric weight that depends on neither the keys nor the current position),
+// in float64 on the host.  The last problem's table is kept per host thread: a
+// decode loop calls with the same offsets every time.
+struct OffsetMean {
+  double theta = 0.0;
+  int32_t D = 0;
+  std::vector<int32_t> offsets;
+  std::vector<double> re, im;
+};
+
+const OffsetMean &offset_mean(const tria_config *cfg) {
+  static thread_local OffsetMean m;
+  const bool same = m.theta == cfg->rope_theta && m.D == cfg->head_dim &&
+                    (int)m.offsets.size() == cfg->n_offsets &&
+                    std::memcmp(m.offsets.data(), cfg->offsets, sizeof(int32_t) * cfg->n_offsets) == 0;
+  if (!same) {
+    const int F = cfg->head_dim / 2;
+    m.theta = cfg->rope_theta;
+    m.D = cfg->head_dim;
+    m.offsets.assign(cfg->offsets, cfg->offsets + cfg->n_offsets);
+    m.re.assign(F, 0.0);
+    m.im.assign(F, 0.0);
+    for (int f = 0; f < F; ++f) {
+      const double w = std::pow(cfg->rope_theta, -2.0 * (double)f / (double)cfg->head_dim);
+      double re = 0.0, im = 0.0;
+      for (int j = 0; j < cfg->n_offsets; ++j) {
+        re += std::cos(w * (double)cfg->offsets[j]);
+        im += std::sin(w * (double)cfg->offsets[j]);
+      }
+      m.re[f] = re / (double)cfg->n_offsets;
+      m.im[f] = im / (double)cfg->n_offsets;
+    }
+  }
+  return m;
+}
+
 void fill_fold(FoldParams &fp, const tria_config *cfg, const tria_stats *st,
                const tria_cache *c, int32_t *seqlen_snap, float *w, int32_t *err) {
   std::memset(&fp, 0, sizeof fp);
@@ -198,12 +235,16 @@ void fill_fold(FoldParams &fp, const tria_config *cfg, const tria_stats *st,
   fp.Hkv = cfg->n_kv_heads;
   fp.Hq = cfg->n_q_heads;
   fp.G = cfg->n_q_heads / cfg->n_kv_heads;
-  fp.n_offsets = cfg->n_offsets;
   fp.flags = cfg->flags;
   for (int b = 0; b < cfg->batch; ++b) fp.seg_cap[b] = c->seq_start[b + 1] - c->seq_start[b];
-  std::memcpy(fp.offsets, cfg->offsets, sizeof(int32_t) * cfg->n_offsets);
-  for (int f = 0; f < cfg->head_dim / 2 && f < 128; ++f)
+  // the offset average does not depend on the call's positions: it is formed on the host
+  // in float64 (once per offset set, then cached) and passed with the frequencies
+  const OffsetMean &om = offset_mean(cfg);
+  const bool no_trig = (cfg->flags & TRIA_NO_TRIG) != 0;
+  for (int f = 0; f < cfg->head_dim / 2 && f < 128; ++f) {
     fp.omega[f] = std::pow(cfg->rope_theta, -2.0 * (double)f / (double)cfg->head_dim);
+    fp.A[f] = no_trig ? make_double2(0.0, 0.0) : make_double2(om.re[f], om.im[f]);
+  }
 }
 
 // Builds the score kernel parameters; *grid receives the grid size (0: nothing to launch).
@@ -300,42 +341,6 @@ struct Ws {
 const char *kStageNames[] = {"fold_kernel", "score_kernel", "unit_kernel", "prune_kernel"};
 enum StageId : int32_t { kStageFold = 0, kStageScore = 1, kStageUnit = 2, kStagePrune = 3 };
 
-// Mean over the offsets of e^{i w_f delta} for every RoPE pair (the part of the
-// trigonometric weight that depends on neither the keys nor the current position),
-// in float64 on the host.  The last problem's table is kept per host thread: a
-// decode loop calls with the same offsets every time.
-struct OffsetMean {
-  double theta = 0.0;
-  int32_t D = 0;
-  std::vector<int32_t> offsets;
-  std::vector<double> re, im;
-};
-
-const OffsetMean &offset_mean(const tria_config *cfg) {
-  static thread_local OffsetMean m;
-  const bool same = m.theta == cfg->rope_theta && m.D == cfg->head_dim &&
-                    (int)m.offsets.size() == cfg->n_offsets &&
-                    std::memcmp(m.offsets.data(), cfg->offsets, sizeof(int32_t) * cfg->n_offsets) == 0;
-  if (!same) {
-    const int F = cfg->head_dim / 2;
-    m.theta = cfg->rope_theta;
-    m.D = cfg->head_dim;
-    m.offsets.assign(cfg->offsets, cfg->offsets + cfg->n_offsets);
-    m.re.assign(F, 0.0);
-    m.im.assign(F, 0.0);
-    for (int f = 0; f < F; ++f) {
-      const double w = std::pow(cfg->rope_theta, -2.0 * (double)f / (double)cfg->head_dim);
-      double re = 0.0, im = 0.0;
-      for (int j = 0; j < cfg->n_offsets; ++j) {
-        re += std::cos(w * (double)cfg->offsets[j]);
-        im += std::sin(w * (double)cfg->offsets[j]);
-      }
-      m.re[f] = re / (double)cfg->n_offsets;
-      m.im[f] = im / (double)cfg->n_offsets;
-    }
-  }
-  return m;
-}
 
 // Parameters of the fused prune kernel.
 cudaError_t fill_prune(PruneParams &pp, const tria_config *cfg, const tria_stats *st,

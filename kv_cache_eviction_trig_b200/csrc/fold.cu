@@ -10,9 +10,9 @@
 // so the per-key work needs no position and no trigonometry.  The norm term's
 // weight is Nw_f = (1 - R_f) E|q_f| (section 3-2 (3)-(4)).
 //
-// Block (fp, y) handles the RoPE pairs f = 2fp, 2fp+1 (w_f comes from the host,
-// in double precision): it forms EA in float64 (angles reach ~1e5 rad) for every
-// sequence, then writes, for a share y of
+// Block (fp, y) handles the RoPE pairs f = 2fp, 2fp+1 (w_f and the offset average
+// A_f come from the host, in double precision): it forms EA = e^{i w_f cur} A_f in
+// float64 (angles reach ~1e5 rad) for every sequence, then writes, for a share y of
 // the (unit, head) pairs, the float32 weights
 //   w[unit][fp][h] = (Re W_2fp, Re W_2fp+1, Im W_2fp, Im W_2fp+1, Nw_2fp, Nw_2fp+1).
 // Block (0, 0) also snapshots and checks seq_len (blocks (0, y) the per-unit
@@ -28,7 +28,6 @@ __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldP
   dev::pdl_launch_dependents();  // the score kernel may start streaming keys now
   const int fp = blockIdx.x;
   const int F = p.D / 2;
-  __shared__ double red[4][8];
   __shared__ double2 ea[TRIA_MAX_BATCH][2];
   // Loads that do not depend on the trigonometry are issued first.
   const int64_t units = (int64_t)p.L * p.Hkv * p.B;
@@ -54,31 +53,8 @@ __global__ void __launch_bounds__(256) fold_kernel(const __grid_constant__ FoldP
   const int32_t t_in = snap ? p.seq_len[threadIdx.x] : 0;
   // w_f = theta^(-2f/D), evaluated on the host in double precision
   const double w[2] = {p.omega[2 * fp], p.omega[2 * fp + 1]};
-  double a[4] = {0.0, 0.0, 0.0, 0.0};  // (cos, sin) sums for the two pairs
-  for (int j = threadIdx.x; j < p.n_offsets; j += blockDim.x) {
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      double s, c;
-      sincos(w[q] * (double)p.offsets[j], &s, &c);
-      a[2 * q] += c;
-      a[2 * q + 1] += s;
-    }
-  }
-  // fixed-order block reduction (deterministic)
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    for (int o = 16; o > 0; o >>= 1) a[i] += __shfl_xor_sync(0xffffffffu, a[i], o);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0)
-    for (int i = 0; i < 4; ++i) red[i][warp] = a[i];
-  __syncthreads();
-  double A[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    double s = 0.0;
-    for (int k = 0; k < (int)(blockDim.x >> 5); ++k) s += red[i][k];
-    A[i] = (p.flags & TRIA_NO_TRIG) ? 0.0 : s / (double)p.n_offsets;
-  }
+  // the offset average A_f = mean_delta e^{i w_f delta}, from the host (float64)
+  const double A[4] = {p.A[2 * fp].x, p.A[2 * fp].y, p.A[2 * fp + 1].x, p.A[2 * fp + 1].y};
   for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
     const int32_t cb = b == (int)threadIdx.x ? cur : p.cur_pos[b];
 #pragma unroll

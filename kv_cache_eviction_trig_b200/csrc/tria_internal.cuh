@@ -87,11 +87,11 @@ struct FoldParams {
   const float *mrl;         // [L][Hq][F]
   float *w;                 // [L*Hkv*B][F/2][G][6] out
   double theta;
-  int32_t D, B, L, Hkv, Hq, G, n_offsets;
+  int32_t D, B, L, Hkv, Hq, G;
   uint32_t flags;
   int64_t seg_cap[TRIA_MAX_BATCH];
-  int32_t offsets[TRIA_MAX_OFFSETS];
   double omega[128];        // w_f = theta^(-2f/D), f < D/2
+  double2 A[128];           // mean over the offsets of e^{i w_f delta} (0 without the trig term)
 };
 
 struct alignas(64) ScoreParams {

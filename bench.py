@@ -420,6 +420,42 @@ class Bench:
         torch.cuda.empty_cache()
 
 
+def attention_figures(dev, B, T, steps, peak):
+    """tria_decode_attention on one 8B-shaped layer (8 KV heads x 4 query heads, D = 128)
+    with B sequences of T live keys, L2 flushed before every call: mean device time and
+    HBM rate (K and V of the live slots read once)."""
+    H, Hq, D = 8, 32, 128
+    gen = torch.Generator(device=dev).manual_seed(B * 100003 + T)
+    k = torch.randn(1, H, B * T, D, device=dev, generator=gen).to(torch.bfloat16)
+    v = torch.randn(1, H, B * T, D, device=dev, generator=gen).to(torch.bfloat16)
+    pos = torch.zeros(1, H, B * T, dtype=torch.int32, device=dev)
+    sl = torch.full((B,), T, dtype=torch.int32, device=dev)
+    cfg = tria.Config(num_layers=1, batch=B, n_q_heads=Hq, n_kv_heads=H, head_dim=D,
+                      rope_theta=1e6, budget=T, offsets=[1])
+    cache = tria.Cache(k, v, pos, sl, sl.clone(), [b * T for b in range(B + 1)])
+    ws = tria.workspace(cfg, cache)
+    q = torch.randn(B, Hq, D, device=dev, generator=gen).to(torch.bfloat16)
+    out = torch.empty(B, Hq, D, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        tria.tria_decode_attention(cfg, cache, 0, q, out, ws, stream=stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
+        flush.fill_(1)
+        a.record(stream)
+        tria.tria_decode_attention(cfg, cache, 0, q, out, ws, stream=stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    if tria.tria_get_device_error(ws) != 0:
+        raise RuntimeError("device error flag set in decode attention")
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    algo = B * H * T * 4 * D
+    return {"batch": B, "live_keys": T, "us": ms * 1e3, "gbs": algo / (ms / 1e3) / 1e9,
+            "frac": algo / (ms / 1e3) / 1e9 / peak, "algorithmic_bytes": algo, "steps": steps}
+
+
 def run_ours(args):
     rank, world, local = _rank_env()
     torch.cuda.set_device(local)
@@ -560,6 +596,13 @@ def run_ours(args):
                 entry = {"workload": xwl.name, "error": f"{type(e).__name__}: {e}"}
                 torch.cuda.empty_cache()
             extras[key] = entry
+        # decode attention over a pruned (2048) and an unpruned (32768) layer
+        for B, T in ((1, 2048), (1, 32768), (16, 2048), (16, 32768)):
+            try:
+                extras[f"attention_b{B}_t{T}"] = attention_figures(dev, B, T, args.extra_steps, peak)
+            except Exception as e:
+                extras[f"attention_b{B}_t{T}"] = {"error": f"{type(e).__name__}: {e}"}
+            torch.cuda.empty_cache()
         out["extra_workloads"] = extras
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -8,16 +8,21 @@
 // The cache holds post-RoPE keys, so the (non-contiguous) positions of the
 // surviving keys play no part.
 //
-// Design (sm_100a): one 8-CTA cluster per (sequence, KV head); CTA r takes the
-// r-th contiguous slice of the live keys and walks it in tiles of 256 keys with
-// a running maximum (online softmax) for all G query heads of the group, so the
-// group's keys and values are read from HBM once.  In a tile, thread i scores
-// key i against the G queries (16-byte loads of its key row, queries broadcast
-// from shared memory), then threads split the head dimension (and, for D < 256,
-// the tile's keys) to accumulate p * v with coalesced loads of each value row.
-// The eight partial results (running max, sum of exponentials, unnormalised
-// output) are combined by rank 0 through distributed shared memory; no
-// workspace and no second kernel.  Float32 throughout, expf for the weights.
+// Design (sm_100a): one cluster of CL CTAs per (sequence, KV head), one CTA per
+// SM, CL the largest power of two (at most 8) that keeps the launch in one wave.  CTA r takes the r-th contiguous slice of the live keys
+// and walks it in tiles of 16384 / D keys with a running maximum (online
+// softmax) for all G query heads of the group, so the group's keys and values are
+// read from HBM once.  The tiles stream into three shared-memory stages with bulk
+// asynchronous copies (one for the tile's K rows, one for its V rows), the next
+// two tiles' copies in flight while the current one is computed.  In a tile, LPK
+// lanes score a key, each over D / LPK of its dims with those dims of the query
+// heads held in registers, and a butterfly adds their parts; then thread
+// (kg, dg) accumulates p * v over columns [dg * VP, dg * VP + VP) of the tile's
+// rows kg, kg + KG, ....  Every CTA then combines a slice of the output from the
+// CL partial results (running max, sum of exponentials, unnormalised output)
+// through distributed shared memory; no workspace and no second kernel.  Float32
+// throughout, expf for the weights; every sum is taken in a fixed order.  A
+// bounded wait that runs out sets TRIA_DEVERR_TIMEOUT.
 #include <cooperative_groups.h>
 
 #include <math.h>
@@ -30,24 +35,54 @@ namespace tria {
 
 namespace {
 
-constexpr int kAttnCluster = 8;
 constexpr int kAttnThreads = 256;
-constexpr int kAttnTile = 256;  // keys per tile: one per thread when scoring
+constexpr int kAttnNW = kAttnThreads / 32;
 
 __device__ __forceinline__ float bf16_to_f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
 template <int D, int G>
-__global__ void __cluster_dims__(kAttnCluster, 1, 1) __launch_bounds__(kAttnThreads, 1)
+struct AttnShape {
+  static constexpr int TILE = 16384 / D;          // keys per tile (32 KB of K, 32 KB of V)
+  static constexpr int VROW = 2 * D;              // a K or V row in shared memory (bytes)
+  static constexpr int KROW = VROW;
+  static constexpr int KST = TILE * KROW, VST = TILE * VROW;
+  static constexpr int STAGE = KST + VST;
+  static constexpr int VP = G >= 16 ? 4 : 8;      // values of a row per thread in p * v
+  // scoring: HQ query heads per pass, LPK lanes per key, DPL dims per lane, so that a
+  // lane holds at most 64 query values in registers
+  static constexpr int HQ = G * D <= 2048 ? G : 2048 / D;
+  static constexpr int LPK0 = HQ * D / 64 < 1 ? 1 : HQ * D / 64;
+  static constexpr int LPK = LPK0 > 32 ? 32 : LPK0;
+  static constexpr int DPL = D / LPK;
+  static_assert(HQ >= 1 && G % HQ == 0 && (LPK & (LPK - 1)) == 0 && DPL * LPK == D, "scoring");
+  static_assert(DPL % 8 == 0 || DPL == 4, "16-byte (or 8-byte) key loads");
+  static_assert(HQ * DPL <= 64, "query registers");
+  static constexpr int DG = D / VP, KG = kAttnThreads / DG;
+  static constexpr int NST = 3;                             // stages in flight
+  static constexpr int QS = NST * STAGE;                    // float [G][D]
+  static constexpr int SC = QS + G * D * 4;                 // float [G][TILE]
+  static constexpr int BAR = SC + G * TILE * 4;             // NST mbarriers
+  static constexpr int SMEM = BAR + 8 * NST;
+  static_assert(DG * VP == D && KG * DG == kAttnThreads && TILE <= kAttnThreads, "shape");
+  static_assert(KST % 128 == 0 && STAGE % 128 == 0 && QS % 16 == 0, "aligned regions");
+};
+
+template <int D, int G, int CL>
+__global__ void __launch_bounds__(kAttnThreads, 1)
     attention_kernel(const __grid_constant__ AttnParams p) {
-  constexpr int KG = kAttnThreads / D;  // key groups in the p*v pass
-  static_assert(KG >= 1 && KG * D == kAttnThreads, "D divides the block");
-  __shared__ __align__(16) float qo[G][D];          // the queries, later the partial output
-  __shared__ __align__(16) float sc[G][kAttnTile];  // tile scores / weights, later p*v partials
+  using S = AttnShape<D, G>;
+  constexpr int TILE = S::TILE, VP = S::VP, DG = S::DG, KG = S::KG;
+  extern __shared__ __align__(128) uint8_t sm[];
+  float (*qs)[D] = reinterpret_cast<float (*)[D]>(sm + S::QS);  // queries, then partial output
+  float (*sc)[TILE] = reinterpret_cast<float (*)[TILE]>(sm + S::SC);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + S::BAR);
   __shared__ float mrun[G], lrun[G], alpha[G];
+  __shared__ float pm[CL][G], pl[CL][G];
+  __shared__ int all_ok;
 
   cg::cluster_group cl = cg::this_cluster();
   const int r = (int)cl.block_rank();
-  const int unit = blockIdx.x / kAttnCluster;  // b * Hkv + g
+  const int unit = blockIdx.x / CL;  // b * Hkv + g
   const int b = unit / p.Hkv, g = unit - b * p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t cap_b = p.seg_start[b + 1] - p.seg_start[b];
@@ -56,51 +91,119 @@ __global__ void __cluster_dims__(kAttnCluster, 1, 1) __launch_bounds__(kAttnThre
     if (r == 0 && tid == 0 && (g == 0 || p.unit_len)) dev::set_error(p.err, TRIA_DEVERR_SEQ_LEN);
     return;
   }
-  const int t0 = (int)((int64_t)T * r / kAttnCluster), t1 = (int)((int64_t)T * (r + 1) / kAttnCluster);
+  const int t0 = (int)((int64_t)T * r / CL), t1 = (int)((int64_t)T * (r + 1) / CL);
+  const int ntiles = (t1 - t0 + TILE - 1) / TILE;
   const size_t row0 = ((size_t)p.layer * p.Hkv + g) * p.cap + p.seg_start[b];
-  const uint16_t *kb = p.k + row0 * D;
-  const uint16_t *vb = p.v + row0 * D;
+  const uint8_t *kb = reinterpret_cast<const uint8_t *>(p.k + row0 * D);
+  const uint8_t *vb = reinterpret_cast<const uint8_t *>(p.v + row0 * D);
   const uint16_t *qb = p.q + ((size_t)b * p.Hq + (size_t)g * G) * D;
 
-  for (int i = tid; i < G * D; i += kAttnThreads) (&qo[0][0])[i] = bf16_to_f(qb[i]);
+  if (tid == 0) {
+#pragma unroll
+    for (int q = 0; q < S::NST; ++q) dev::mbar_init(&bar[q], 1);
+    dev::fence_mbar_init();
+    all_ok = 1;
+  }
+  for (int i = tid; i < G * D; i += kAttnThreads) (&qs[0][0])[i] = bf16_to_f(qb[i]);
   if (tid < G) {
     mrun[tid] = -INFINITY;
     lrun[tid] = 0.0f;
   }
-  const int d = tid % D, kg = tid / D;
-  float acc[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) acc[h] = 0.0f;
   __syncthreads();
+  // thread 0 streams tile i into stage i % NST: the tile's K rows and its V rows,
+  // one bulk copy each (the rows of a segment are contiguous)
+  auto issue = [&](int i) {
+    const int s = i % S::NST, k0 = t0 + i * TILE, n = min(TILE, t1 - k0);
+    uint8_t *st = sm + s * S::STAGE;
+    dev::mbar_arrive_expect_tx(&bar[s], (uint32_t)(2 * n * S::VROW));
+    dev::bulk_g2s(st, kb + (size_t)k0 * S::VROW, (uint32_t)(n * S::VROW), &bar[s]);
+    dev::bulk_g2s(st + S::KST, vb + (size_t)k0 * S::VROW, (uint32_t)(n * S::VROW), &bar[s]);
+  };
+  if (tid == 0)
+    for (int i = 0; i < S::NST && i < ntiles; ++i) issue(i);
+  const int dg = tid % DG, kg = tid / DG;
+  float acc[G][VP];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < VP; ++e) acc[h][e] = 0.0f;
 
-  for (int tile = t0; tile < t1; tile += kAttnTile) {
-    const int n = min(kAttnTile, t1 - tile);
-    // scores of key tile + tid against the G queries
-    if (tid < n) {
-      const uint4 *kr = reinterpret_cast<const uint4 *>(kb + (size_t)(tile + tid) * D);
-      float s[G];
+  for (int i = 0; i < ntiles; ++i) {
+    const int s = i % S::NST, n = min(TILE, t1 - (t0 + i * TILE));
+    const uint8_t *ks = sm + s * S::STAGE, *vs = ks + S::KST;
+    if (!dev::mbar_wait(&bar[s], (uint32_t)(i / S::NST) & 1u)) all_ok = 0;
+    __syncthreads();
+    if (!all_ok) {  // the copies never arrived: give up on this unit
+      if (tid == 0) {
+        dev::set_error(p.err, TRIA_DEVERR_TIMEOUT);
+        // the other stages' copies (issued for the next tiles) may still land: wait
+        // for them, with a limit, before the shared memory is given up
+        for (int q = i + 1; q < i + S::NST && q < ntiles; ++q)
+          (void)dev::mbar_wait(&bar[q % S::NST], (uint32_t)(q / S::NST) & 1u);
+      }
+      __syncthreads();
+      break;
+    }
+    // scores: LPK lanes per key, each with DPL of the key's dims (16-byte chunks
+    // sub, sub + LPK, ... of the row, so that the lanes of a key read consecutive
+    // chunks) and those dims of HQ query heads in registers; the LPK partial dots
+    // meet in a butterfly
+    {
+      constexpr int HQ = S::HQ, LPK = S::LPK, DPL = S::DPL, KPW = 32 / LPK;
+      const int sub = lane % LPK, kw = lane / LPK;
+#pragma unroll 1
+      for (int h0 = 0; h0 < G; h0 += HQ) {
+        float qr[HQ][DPL];
 #pragma unroll
-      for (int h = 0; h < G; ++h) s[h] = 0.0f;
-#pragma unroll 8
-      for (int i = 0; i < D / 8; ++i) {
-        const uint4 w = __ldg(kr + i);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        for (int h = 0; h < HQ; ++h)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float x0 = bf16_to_f(ws[j] & 0xffffu), x1 = bf16_to_f(ws[j] >> 16);
+          for (int d = 0; d < DPL; ++d)
+            qr[h][d] = DPL % 8 == 0 ? qs[h0 + h][((d >> 3) * LPK + sub) * 8 + (d & 7)]
+                                    : qs[h0 + h][sub * DPL + d];
+        for (int jb = warp * KPW; jb < n; jb += kAttnNW * KPW) {
+          const int j = jb + kw;  // (rows at or past n hold stale data: not written out)
+          const uint8_t *kr = ks + j * S::KROW;
+          float part[HQ];
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            s[h] = fmaf(x0, qo[h][8 * i + 2 * j], s[h]);
-            s[h] = fmaf(x1, qo[h][8 * i + 2 * j + 1], s[h]);
+          for (int h = 0; h < HQ; ++h) part[h] = 0.0f;
+          if constexpr (DPL % 8 == 0) {
+#pragma unroll
+            for (int c = 0; c < DPL / 8; ++c) {
+              const uint4 w = reinterpret_cast<const uint4 *>(kr)[c * LPK + sub];
+              const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float x0 = bf16_to_f(ws[q] & 0xffffu), x1 = bf16_to_f(ws[q] >> 16);
+#pragma unroll
+                for (int h = 0; h < HQ; ++h) {
+                  part[h] = fmaf(x0, qr[h][8 * c + 2 * q], part[h]);
+                  part[h] = fmaf(x1, qr[h][8 * c + 2 * q + 1], part[h]);
+                }
+              }
+            }
+          } else {
+            const uint2 w = reinterpret_cast<const uint2 *>(kr)[sub];
+            const float x[4] = {bf16_to_f(w.x & 0xffffu), bf16_to_f(w.x >> 16),
+                                bf16_to_f(w.y & 0xffffu), bf16_to_f(w.y >> 16)};
+#pragma unroll
+            for (int h = 0; h < HQ; ++h)
+#pragma unroll
+              for (int d = 0; d < 4; ++d) part[h] = fmaf(x[d], qr[h][d], part[h]);
+          }
+#pragma unroll
+          for (int o = LPK / 2; o > 0; o >>= 1)
+#pragma unroll
+            for (int h = 0; h < HQ; ++h) part[h] += __shfl_xor_sync(0xffffffffu, part[h], o);
+          if (sub == 0 && j < n) {
+#pragma unroll
+            for (int h = 0; h < HQ; ++h) sc[h0 + h][j] = part[h] * p.scale;
           }
         }
       }
-#pragma unroll
-      for (int h = 0; h < G; ++h) sc[h][tid] = s[h] * p.scale;
     }
     __syncthreads();
     // running maximum per head (a warp per head)
-    for (int h = warp; h < G; h += kAttnThreads / 32) {
+    for (int h = warp; h < G; h += kAttnNW) {
       float mx = -INFINITY;
       for (int j = lane; j < n; j += 32) mx = fmaxf(mx, sc[h][j]);
 #pragma unroll
@@ -112,13 +215,13 @@ __global__ void __cluster_dims__(kAttnCluster, 1, 1) __launch_bounds__(kAttnThre
       }
     }
     __syncthreads();
-    if (tid < n) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) sc[h][tid] = expf(sc[h][tid] - mrun[h]);
+    for (int idx = tid; idx < G * n; idx += kAttnThreads) {
+      const int h = idx / n, j = idx - h * n;
+      sc[h][j] = expf(sc[h][j] - mrun[h]);
     }
     __syncthreads();
     // sum of the weights (a warp per head) and the weighted values (all threads)
-    for (int h = warp; h < G; h += kAttnThreads / 32) {
+    for (int h = warp; h < G; h += kAttnNW) {
       float sum = 0.0f;
       for (int j = lane; j < n; j += 32) sum += sc[h][j];
 #pragma unroll
@@ -126,70 +229,131 @@ __global__ void __cluster_dims__(kAttnCluster, 1, 1) __launch_bounds__(kAttnThre
       if (lane == 0) lrun[h] = lrun[h] * alpha[h] + sum;
     }
 #pragma unroll
-    for (int h = 0; h < G; ++h) acc[h] *= alpha[h];
-    // eight value loads in flight per thread, then their products in key order
-    int j = kg;
-    for (; j + 7 * KG < n; j += 8 * KG) {
-      float vv[8];
+    for (int h = 0; h < G; ++h) {
+      const float a = alpha[h];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) vv[u] = bf16_to_f(__ldg(vb + (size_t)(tile + j + u * KG) * D + d));
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-#pragma unroll
-        for (int h = 0; h < G; ++h) acc[h] = fmaf(sc[h][j + u * KG], vv[u], acc[h]);
+      for (int e = 0; e < VP; ++e) acc[h][e] *= a;
     }
-    for (; j < n; j += KG) {
-      const float vv = bf16_to_f(__ldg(vb + (size_t)(tile + j) * D + d));
+    for (int j = kg; j < n; j += KG) {
+      const uint8_t *vr = vs + j * S::VROW + dg * VP * 2;
+      float x[VP];
+      if constexpr (VP == 8) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(vr);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] = fmaf(sc[h][j], vv, acc[h]);
+        for (int q = 0; q < 4; ++q) {
+          x[2 * q] = bf16_to_f(ws[q] & 0xffffu);
+          x[2 * q + 1] = bf16_to_f(ws[q] >> 16);
+        }
+      } else {
+        const uint2 w = *reinterpret_cast<const uint2 *>(vr);
+        x[0] = bf16_to_f(w.x & 0xffffu);
+        x[1] = bf16_to_f(w.x >> 16);
+        x[2] = bf16_to_f(w.y & 0xffffu);
+        x[3] = bf16_to_f(w.y >> 16);
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float wt = sc[h][j];
+#pragma unroll
+        for (int e = 0; e < VP; ++e) acc[h][e] = fmaf(wt, x[e], acc[h][e]);
+      }
     }
-    __syncthreads();  // sc, alpha and lrun are rewritten by the next tile
+    __syncthreads();  // stage s, sc, alpha and lrun are free again
+    if (tid == 0 && i + S::NST < ntiles) issue(i + S::NST);
   }
-  // partial output of this CTA: the key groups' sums, into qo (the queries are done)
-  float *part = &sc[0][0];  // [KG][G][D] = kAttnThreads * G floats
-#pragma unroll
-  for (int h = 0; h < G; ++h) part[((size_t)kg * G + h) * D + d] = acc[h];
+  // partial output of this CTA: the key groups' sums, added in key-group order
+  for (int i = tid; i < G * D; i += kAttnThreads) (&qs[0][0])[i] = 0.0f;
   __syncthreads();
-  for (int i = tid; i < G * D; i += kAttnThreads) {
-    float o = 0.0f;
-    for (int k = 0; k < KG; ++k) o += part[(size_t)k * G * D + i];
-    (&qo[0][0])[i] = o;
+  for (int k = 0; k < KG; ++k) {
+    if (kg == k) {
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int e = 0; e < VP; ++e) qs[h][dg * VP + e] += acc[h][e];
+    }
+    __syncthreads();
   }
   cl.sync();  // every CTA's running max, sum and partial output are complete
-  if (r == 0) {
-    float *outb = p.out + ((size_t)b * p.Hq + (size_t)g * G) * D;
-    for (int i = tid; i < G * D; i += kAttnThreads) {
-      const int h = i / D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < kAttnCluster; ++q) M = fmaxf(M, cl.map_shared_rank(&mrun[0], q)[h]);
-      float L = 0.0f, O = 0.0f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int q = 0; q < kAttnCluster; ++q) {
-          const float mq = cl.map_shared_rank(&mrun[0], q)[h];
-          const float e = mq == -INFINITY ? 0.0f : expf(mq - M);
-          L = fmaf(cl.map_shared_rank(&lrun[0], q)[h], e, L);
-          O = fmaf(cl.map_shared_rank(&qo[0][0], q)[i], e, O);
-        }
-      }
-      outb[i] = L > 0.0f ? O / L : 0.0f;
-    }
+  for (int i = tid; i < CL * G; i += kAttnThreads) {
+    const int q = i / G, h = i - q * G;
+    pm[q][h] = cl.map_shared_rank(&mrun[0], q)[h];
+    pl[q][h] = cl.map_shared_rank(&lrun[0], q)[h];
   }
-  cl.sync();  // the peers' shared memory stays valid until rank 0 has read it
+  __syncthreads();
+  // CTA r writes its slice of the G * D outputs
+  float *outb = p.out + ((size_t)b * p.Hq + (size_t)g * G) * D;
+  const int e0 = G * D * r / CL, e1 = G * D * (r + 1) / CL;
+  for (int i = e0 + tid; i < e1; i += kAttnThreads) {
+    const int h = i / D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < CL; ++q) M = fmaxf(M, pm[q][h]);
+    float L = 0.0f, O = 0.0f;
+    if (M != -INFINITY) {
+      float part[CL];
+#pragma unroll
+      for (int q = 0; q < CL; ++q) part[q] = cl.map_shared_rank(&qs[0][0], q)[i];
+#pragma unroll
+      for (int q = 0; q < CL; ++q) {
+        const float e = pm[q][h] == -INFINITY ? 0.0f : expf(pm[q][h] - M);
+        L = fmaf(pl[q][h], e, L);
+        O = fmaf(part[q], e, O);
+      }
+    }
+    outb[i] = L > 0.0f ? O / L : 0.0f;
+  }
+  cl.sync();  // the peers' shared memory stays valid until every CTA has read it
 }
 
-template <int D>
-cudaError_t launch_d(const AttnParams &p, cudaStream_t s, unsigned grid) {
+template <int D, int G, int CL>
+cudaError_t launch_dg(const AttnParams &p, cudaStream_t s, int units) {
+  using S = AttnShape<D, G>;
+  auto kern = attention_kernel<D, G, CL>;
+  static bool set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 64 || !set[dev]) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)units * CL, 1, 1);
+  cfg.blockDim = dim3(kAttnThreads, 1, 1);
+  cfg.dynamicSmemBytes = S::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+template <int D, int CL>
+cudaError_t launch_d(const AttnParams &p, cudaStream_t s, int units) {
   switch (p.G) {
-    case 1: attention_kernel<D, 1><<<grid, kAttnThreads, 0, s>>>(p); break;
-    case 2: attention_kernel<D, 2><<<grid, kAttnThreads, 0, s>>>(p); break;
-    case 4: attention_kernel<D, 4><<<grid, kAttnThreads, 0, s>>>(p); break;
-    case 8: attention_kernel<D, 8><<<grid, kAttnThreads, 0, s>>>(p); break;
-    case 16: attention_kernel<D, 16><<<grid, kAttnThreads, 0, s>>>(p); break;
+    case 1: return launch_dg<D, 1, CL>(p, s, units);
+    case 2: return launch_dg<D, 2, CL>(p, s, units);
+    case 4: return launch_dg<D, 4, CL>(p, s, units);
+    case 8: return launch_dg<D, 8, CL>(p, s, units);
+    case 16: return launch_dg<D, 16, CL>(p, s, units);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+}
+
+template <int CL>
+cudaError_t launch_cl(const AttnParams &p, cudaStream_t s, int units) {
+  switch (p.D) {
+    case 64: return launch_d<64, CL>(p, s, units);
+    case 128: return launch_d<128, CL>(p, s, units);
+    case 256: return launch_d<256, CL>(p, s, units);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
@@ -199,13 +363,25 @@ bool attention_supported(int D, int G) {
 }
 
 cudaError_t launch_attention(const AttnParams &p, cudaStream_t s) {
-  const int64_t grid = (int64_t)p.B * p.Hkv * kAttnCluster;
-  if (grid > INT32_MAX) return cudaErrorInvalidValue;
-  switch (p.D) {
-    case 64: return launch_d<64>(p, s, (unsigned)grid);
-    case 128: return launch_d<128>(p, s, (unsigned)grid);
-    case 256: return launch_d<256>(p, s, (unsigned)grid);
-    default: return cudaErrorInvalidValue;
+  const int64_t units = (int64_t)p.B * p.Hkv;
+  if (units * 16 > INT32_MAX) return cudaErrorInvalidValue;
+  int sms = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms < 1) sms = 148;
+  }
+  // one CTA per SM: the largest cluster (a power of two up to 8) that keeps the
+  // launch in one wave (a B200 holds 15 clusters of 8 such CTAs at once, 33 of 4,
+  // 74 of 2)
+  int cl = 1;
+  while (cl < 8 && units * cl * 2 <= sms) cl *= 2;
+  switch (cl) {
+    case 1: return launch_cl<1>(p, s, (int)units);
+    case 2: return launch_cl<2>(p, s, (int)units);
+    case 4: return launch_cl<4>(p, s, (int)units);
+    default: return launch_cl<8>(p, s, (int)units);
   }
 }
 

@@ -208,7 +208,9 @@ tria_status tria_compact(const tria_config *cfg, const tria_cache *cache, const 
  * seq_len is read once at the start and rewritten at the end.  If sel_out is
  * not NULL it receives the selection as tria_select would write it for the
  * sequences that were pruned and for those with seq_len <= budget; the rows of
- * sequences held back by prune_window are not written. */
+ * sequences held back by prune_window are not written.  By default three
+ * kernels (fold, score, unit) chained by programmatic dependent launch;
+ * cfg->flags TRIA_FUSED_PRUNE selects one persistent cooperative launch. */
 tria_status tria_prune(const tria_config *cfg, const tria_stats *stats, const tria_cache *cache,
                        int32_t *sel_out, void *ws, size_t ws_bytes, void *stream);
 
@@ -252,9 +254,10 @@ tria_status tria_decode_attention(const tria_config *cfg, const tria_cache *cach
  * last: events[0..n_stages].  Returns the number of stages in *n_stages
  * (events must hold TRIA_PRUNE_MAX_STAGES + 1) and, if stage_ids is not NULL
  * (HOST, TRIA_PRUNE_MAX_STAGES entries), the kernel of each stage as an index
- * for tria_prune_stage_name.  tria_prune runs one fused kernel for the shapes
- * it fits (every supported shape except head_dim 256 with G = 16) and three
- * kernels otherwise.  For per-kernel timing only. */
+ * for tria_prune_stage_name.  tria_prune runs three kernels (fold, score,
+ * unit); with TRIA_FUSED_PRUNE it runs one persistent launch for the shapes that
+ * launch takes (every supported shape except head_dim 256 with G >= 8).  For
+ * per-kernel timing only. */
 #define TRIA_PRUNE_MAX_STAGES 8
 tria_status tria_prune_profiled(const tria_config *cfg, const tria_stats *stats,
                                 const tria_cache *cache, int32_t *sel_out, void *ws,

@@ -237,6 +237,15 @@ ATT_CASES = {
     "d128_g16_with_empty": lambda: small("att4", Hq=16, Hkv=1, B=2, seq_lens=[130, 0]),
     "d64_interleaved_g2": lambda: small("att5", D=64, Hq=4, Hkv=2, seq_lens=[700], theta=1e4,
                                         rope_layout=workloads.INTERLEAVED),
+    # long slices: every CTA of an 8-CTA cluster streams more tiles than it has stages
+    # (the stages are reused), with a ragged last tile
+    "d128_g4_long": lambda: small("att6", Hq=8, Hkv=2, seq_lens=[12001]),
+    "d64_g2_long": lambda: small("att7", D=64, Hq=4, Hkv=2, seq_lens=[9000], theta=1e4),
+    # G = 16 at D = 256 scores in two passes of 8 query heads
+    "d256_g16_long": lambda: small("att8", D=256, Hq=16, Hkv=1, seq_lens=[3000]),
+    # more (sequence, KV head) pairs than SMs: one CTA per pair, no cluster
+    "d128_g4_many_sequences": lambda: small("att9", B=80, Hq=8, Hkv=2,
+                                            seq_lens=[700 - (b % 7) * 50 for b in range(80)]),
 }
 
 

@@ -321,6 +321,26 @@ def test_prune_many_units_matches_oracle(fused):
     check_compacted(case, gsel, [3500])
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
+def test_prune_many_groups_matches_oracle(fused):
+    """72 units: the single launch takes them in three groups of at most 32, so its
+    per-group scratch slots are reused; lengths span short, pruned and long units."""
+    case = Case(small("groups", L=3, Hq=16, Hkv=8, B=3, seq_lens=[700, 100, 1500], budget=128,
+                      offsets=range(1, 17), slack=9), fused=fused)
+    wl = case.wl
+    ref = oracle.prune(case.prob, common.bf16_bits(case.host["v"]))
+    sel = torch.full((wl.num_layers, wl.n_kv_heads, wl.batch, wl.budget), -7, dtype=torch.int32,
+                     device="cuda")
+    tria.tria_prune(case.cfg, case.stats, case.cache, case.ws, sel_out=sel)
+    torch.cuda.synchronize()
+    assert tria.tria_get_device_error(case.ws) == 0
+    gsel = sel.cpu().numpy()
+    check_selection(gsel, ref["sel"], ref["raw"], ref["score"], case)
+    kept = [min(T, wl.budget) for T in case.lens]
+    assert case.dev["seq_len"].cpu().tolist() == kept == ref["seq_len"].tolist()
+    check_compacted(case, gsel, kept)
+
+
 def test_compact_rejects_malformed_selection():
     wl = small("badsel", B=2, seq_lens=[300, 300], budget=50)
     case = Case(wl)

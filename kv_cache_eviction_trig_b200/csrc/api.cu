@@ -584,6 +584,13 @@ tria_status tria_decode_attention(const tria_config *cfg, const tria_cache *cach
   ap.D = cfg->head_dim;
   ap.scale = scale > 0.0f ? scale : 1.0f / std::sqrt((float)cfg->head_dim);
   for (int b = 0; b <= cfg->batch; ++b) ap.seg_start[b] = cache->seq_start[b];
+  // the tensor-core path reads K and V through TMA tensor maps (rows addressed as int32)
+  const int64_t rows = (int64_t)cfg->num_layers * cfg->n_kv_heads * cache->cap_total;
+  if (attention_mma_supported(cfg->head_dim, ap.G) && rows <= INT32_MAX && rows > 0 &&
+      aligned(cache->k, 16) && aligned(cache->v, 16) &&
+      make_key_tensor_map(&ap.tk, cache->k, cfg->head_dim, rows, 128) == cudaSuccess &&
+      make_key_tensor_map(&ap.tv, cache->v, cfg->head_dim, rows, 128) == cudaSuccess)
+    ap.mma = 1;
   return cuda_status(launch_attention(ap, static_cast<cudaStream_t>(stream)));
 }
 

@@ -25,6 +25,7 @@
 // bounded wait that runs out sets TRIA_DEVERR_TIMEOUT.
 #include <cooperative_groups.h>
 
+#include <cuda_bf16.h>
 #include <math.h>
 
 #include "attention.cuh"
@@ -306,6 +307,357 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   cl.sync();  // the peers' shared memory stays valid until every CTA has read it
 }
 
+// ------------------------------------------------------------------ tensor-core path
+// For D = 64 or 128 and G <= 8 the two products of a tile run on the tensor cores
+// (mma.sync m16n8k16, bf16 inputs, float32 accumulators):
+//   S^T = K Q^T     warp w scores keys [16w, 16w + 16) of the tile for the G heads
+//                   (padded to 8); K comes straight from the TMA-swizzled stage
+//                   and the queries stay in registers.  bf16 x bf16 products are
+//                   exact, so the scores equal the float32 dot products up to the
+//                   order of the additions.
+//   O^T += V^T P^T  warp w owns 16 of the output dims (D = 64: 16 dims and half of
+//                   the tile's keys); P (the exponentials, in [0, 1]) is written to
+//                   shared memory as a bf16 pair hi + lo (16 significant bits), and
+//                   both parts multiply V, so the weights keep float32-level accuracy.
+// The tiles stream in by 2-D TMA loads with 128-byte swizzle; rows of the last tile
+// past the slice are masked out of the softmax, and their V rows are zeroed.
+template <int D>
+struct MmaShape {
+  static constexpr int TILE = 128;
+  static constexpr int NBOX = D / 64;
+  static constexpr int BOXB = TILE * 128;             // one box: 128 rows x 64 dims
+  static constexpr int TB = NBOX * BOXB;              // a tile's K (or V)
+  static constexpr int STAGE = 2 * TB;
+  static constexpr int NST = D == 64 ? 4 : 3;
+  static constexpr int PROW = TILE * 2 + 16;          // bytes per head row of P^T (padded)
+  static constexpr int OFF_Q = NST * STAGE;           // bf16 [8][D] queries
+  static constexpr int OFF_P = OFF_Q + 8 * D * 2;     // bf16 [2][8][PROW / 2]: hi, lo
+  static constexpr int OFF_O = OFF_P + 2 * 8 * PROW;  // float [8][D] partial output
+  static constexpr int OFF_W = OFF_O + 8 * D * 4;     // float [2][8 warps][8]: max, sum
+  static constexpr int OFF_BAR = OFF_W + 2 * 64 * 4;
+  static constexpr int SMEM = OFF_BAR + 8 * NST + 1024;  // + room to align to 1024
+  static_assert(D == 64 || D == 128, "tensor-core path");
+};
+
+// Address of the 16-byte unit holding dims [dim, dim + 8) of row `row` of a tile
+// stored as 128-byte-swizzled TMA boxes of 64 dims.
+template <int BOXB>
+__device__ __forceinline__ uint32_t swz(uint32_t base, int row, int dim) {
+  return base + (uint32_t)(dim >> 6) * BOXB + (uint32_t)row * 128u +
+         ((uint32_t)(((dim >> 3) & 7) ^ (row & 7)) << 4);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t (&r)[2]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+template <int D, int G, int CL>
+__global__ void __launch_bounds__(256, 1)
+    attention_mma_kernel(const __grid_constant__ AttnParams p) {
+  using M = MmaShape<D>;
+  constexpr int TILE = M::TILE, NBOX = M::NBOX, NST = M::NST, KS = D / 16;
+  static_assert(G <= 8, "heads padded to 8");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = smem_raw + ((1024u - (dev::smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint16_t *qsm = reinterpret_cast<uint16_t *>(sm + M::OFF_Q);
+  uint8_t *pt = sm + M::OFF_P;
+  float *osm = reinterpret_cast<float *>(sm + M::OFF_O);
+  float *wmx = reinterpret_cast<float *>(sm + M::OFF_W);
+  float *wsm = wmx + 64;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + M::OFF_BAR);
+  __shared__ float mrun[8], lrun[8];
+  __shared__ float pm[CL][8], pl[CL][8];
+  __shared__ int all_ok;
+
+  cg::cluster_group cl = cg::this_cluster();
+  const int r = (int)cl.block_rank();
+  const int unit = blockIdx.x / CL;  // b * Hkv + g
+  const int b = unit / p.Hkv, g = unit - b * p.Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t cap_b = p.seg_start[b + 1] - p.seg_start[b];
+  const int32_t T = p.unit_len ? p.unit_len[((int64_t)p.layer * p.Hkv + g) * p.B + b] : p.seq_len[b];
+  if (T < 0 || (int64_t)T > cap_b) {  // the same decision in every CTA of the cluster
+    if (r == 0 && tid == 0 && (g == 0 || p.unit_len)) dev::set_error(p.err, TRIA_DEVERR_SEQ_LEN);
+    return;
+  }
+  const int t0 = (int)((int64_t)T * r / CL), t1 = (int)((int64_t)T * (r + 1) / CL);
+  const int ntiles = (t1 - t0 + TILE - 1) / TILE;
+  // tensor row of the segment's slot 0 (the host checked that every row fits int32)
+  const int32_t y0 = (int32_t)(((int64_t)p.layer * p.Hkv + g) * p.cap + p.seg_start[b]);
+  const uint16_t *qb = p.q + ((size_t)b * p.Hq + (size_t)g * G) * D;
+
+  if (tid == 0) {
+#pragma unroll
+    for (int q = 0; q < NST; ++q) dev::mbar_init(&bar[q], 1);
+    dev::fence_mbar_init();
+    all_ok = 1;
+  }
+  for (int i = tid; i < 8 * D; i += 256) qsm[i] = i < G * D ? qb[i] : (uint16_t)0;
+  if (tid < 8) {
+    mrun[tid] = -INFINITY;
+    lrun[tid] = 0.0f;
+  }
+  __syncthreads();
+  auto issue = [&](int i) {  // thread 0: tile i into stage i % NST
+    const int s = i % NST;
+    uint8_t *st = sm + s * M::STAGE;
+    const int32_t y = y0 + t0 + i * TILE;
+    // the stage's earlier contents were read (and its V tail zeroed) through the
+    // generic proxy: order that before the tensor copies overwrite it
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    dev::mbar_arrive_expect_tx(&bar[s], (uint32_t)M::STAGE);
+#pragma unroll
+    for (int bx = 0; bx < NBOX; ++bx) {
+      dev::tma_load_2d(st + bx * M::BOXB, &p.tk, bx * 64, y, &bar[s]);
+      dev::tma_load_2d(st + M::TB + bx * M::BOXB, &p.tv, bx * 64, y, &bar[s]);
+    }
+  };
+  if (tid == 0)
+    for (int i = 0; i < NST && i < ntiles; ++i) issue(i);
+
+  // queries as the B operand of S^T = K Q^T, one fragment pair per 16 dims
+  uint32_t qf[KS][2];
+  {
+    const uint32_t qa = dev::smem_addr(qsm) + (uint32_t)((lane & 7) * D * 2 + ((lane >> 3) & 1) * 16);
+#pragma unroll
+    for (int t = 0; t < KS; ++t) ldsm_x2(qa + t * 32, qf[t]);
+  }
+  const int hA = 2 * (lane & 3), hB = hA + 1;  // the heads of this lane's accumulators
+  float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};       // O^T: dims dm + lane / 4 (+ 8), heads hA, hB
+  const int dm = D == 128 ? 16 * warp : 16 * (warp & 3);
+  const int j0 = D == 128 ? 0 : 4 * (warp >> 2), j1 = D == 128 ? 8 : j0 + 4;
+  const uint32_t pth = dev::smem_addr(pt), ptl = pth + 8 * M::PROW;
+  uint16_t *pth_g = reinterpret_cast<uint16_t *>(pt), *ptl_g = pth_g + 4 * M::PROW;
+
+  for (int i = 0; i < ntiles; ++i) {
+    const int s = i % NST, n = min(TILE, t1 - (t0 + i * TILE));
+    uint8_t *ks = sm + s * M::STAGE, *vs = ks + M::TB;
+    if (!dev::mbar_wait(&bar[s], (uint32_t)(i / NST) & 1u)) all_ok = 0;
+    // the V rows past the slice are zeroed (they may hold anything)
+    for (int idx = tid; idx < (TILE - n) * NBOX * 8; idx += 256) {
+      const int row = n + idx / (NBOX * 8), rest = idx % (NBOX * 8);
+      *reinterpret_cast<uint4 *>(vs + (rest >> 3) * M::BOXB + row * 128 + (rest & 7) * 16) =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    // S^T for keys [16 warp, 16 warp + 16)
+    float sacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    {
+      const int mat = lane >> 3, key = 16 * warp + (mat & 1) * 8 + (lane & 7);
+      const uint32_t kb = dev::smem_addr(ks);
+#pragma unroll
+      for (int t = 0; t < KS; ++t) {
+        uint32_t a[4];
+        ldsm_x4(swz<M::BOXB>(kb, key, 16 * t + (mat >> 1) * 8), a);
+        mma_bf16(sacc, a, qf[t]);
+      }
+    }
+    const int keyA = 16 * warp + (lane >> 2), keyB = keyA + 8;
+    float sv[4];
+    sv[0] = keyA < n ? sacc[0] * p.scale : -INFINITY;
+    sv[1] = keyA < n ? sacc[1] * p.scale : -INFINITY;
+    sv[2] = keyB < n ? sacc[2] * p.scale : -INFINITY;
+    sv[3] = keyB < n ? sacc[3] * p.scale : -INFINITY;
+    float mA = fmaxf(sv[0], sv[2]), mB = fmaxf(sv[1], sv[3]);
+#pragma unroll
+    for (int o2 = 4; o2 < 32; o2 <<= 1) {
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, o2));
+      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, o2));
+    }
+    if (lane < 4) {
+      wmx[warp * 8 + hA] = mA;
+      wmx[warp * 8 + hB] = mB;
+    }
+    __syncthreads();
+    if (!all_ok) {  // the copies never arrived: give up on this unit
+      if (tid == 0) {
+        dev::set_error(p.err, TRIA_DEVERR_TIMEOUT);
+        for (int q = i + 1; q < i + NST && q < ntiles; ++q)
+          (void)dev::mbar_wait(&bar[q % NST], (uint32_t)(q / NST) & 1u);
+      }
+      __syncthreads();
+      break;
+    }
+    // new running maxima of this lane's heads (the tile has at least one key)
+    float tmA = -INFINITY, tmB = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      tmA = fmaxf(tmA, wmx[w * 8 + hA]);
+      tmB = fmaxf(tmB, wmx[w * 8 + hB]);
+    }
+    const float MA = fmaxf(mrun[hA], tmA), MB = fmaxf(mrun[hB], tmB);
+    const float alA = mrun[hA] == -INFINITY ? 0.0f : expf(mrun[hA] - MA);
+    const float alB = mrun[hB] == -INFINITY ? 0.0f : expf(mrun[hB] - MB);
+    float pv[4];
+    pv[0] = expf(sv[0] - MA);
+    pv[1] = expf(sv[1] - MB);
+    pv[2] = expf(sv[2] - MA);
+    pv[3] = expf(sv[3] - MB);
+    float sA = pv[0] + pv[2], sB = pv[1] + pv[3];
+#pragma unroll
+    for (int o2 = 4; o2 < 32; o2 <<= 1) {
+      sA += __shfl_xor_sync(0xffffffffu, sA, o2);
+      sB += __shfl_xor_sync(0xffffffffu, sB, o2);
+    }
+    if (lane < 4) {
+      wsm[warp * 8 + hA] = sA;
+      wsm[warp * 8 + hB] = sB;
+    }
+    // P^T as bf16 hi + lo: row = head, column = key
+    {
+      const int keys[4] = {keyA, keyA, keyB, keyB}, heads[4] = {hA, hB, hA, hB};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(pv[e]);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(pv[e] - __bfloat162float(hi));
+        const int at = heads[e] * (M::PROW / 2) + keys[e];
+        pth_g[at] = __bfloat16_as_ushort(hi);
+        ptl_g[at] = __bfloat16_as_ushort(lo);
+      }
+    }
+    __syncthreads();
+    // O^T = alpha O^T + V^T P^T over this warp's dims (and, for D = 64, half of the keys)
+    o[0] *= alA;
+    o[1] *= alB;
+    o[2] *= alA;
+    o[3] *= alB;
+    {
+      const int mat = lane >> 3;
+      const uint32_t vb = dev::smem_addr(vs);
+      const uint32_t pa = (uint32_t)((lane & 7) * M::PROW + ((lane >> 3) & 1) * 16);
+#pragma unroll
+      for (int j = j0; j < j1; ++j) {
+        uint32_t a[4], bh[2], bl[2];
+        ldsm_x4_t(swz<M::BOXB>(vb, 16 * j + (mat >> 1) * 8 + (lane & 7), dm + (mat & 1) * 8), a);
+        ldsm_x2(pth + pa + 32 * j, bh);
+        ldsm_x2(ptl + pa + 32 * j, bl);
+        mma_bf16(o, a, bh);
+        mma_bf16(o, a, bl);
+      }
+    }
+    if (tid < 8) {  // running max and sum of head tid (every thread has read them)
+      float tm = -INFINITY, ts = 0.0f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        tm = fmaxf(tm, wmx[w * 8 + tid]);
+        ts += wsm[w * 8 + tid];
+      }
+      const float Mn = fmaxf(mrun[tid], tm);
+      const float al = mrun[tid] == -INFINITY ? 0.0f : expf(mrun[tid] - Mn);
+      lrun[tid] = lrun[tid] * al + ts;
+      mrun[tid] = Mn;
+    }
+    __syncthreads();  // stage s, P^T and the warp arrays are free again
+    if (tid == 0 && i + NST < ntiles) issue(i + NST);
+  }
+  // this CTA's unnormalised output O[h][d] (D = 64: the two key halves added in order)
+  const int dA = dm + (lane >> 2), dB = dA + 8;
+  if (D == 128 || warp < 4) {
+    osm[hA * D + dA] = o[0];
+    osm[hB * D + dA] = o[1];
+    osm[hA * D + dB] = o[2];
+    osm[hB * D + dB] = o[3];
+  }
+  if (D == 64) {
+    __syncthreads();
+    if (warp >= 4) {
+      osm[hA * D + dA] += o[0];
+      osm[hB * D + dA] += o[1];
+      osm[hA * D + dB] += o[2];
+      osm[hB * D + dB] += o[3];
+    }
+  }
+  __syncthreads();
+  cl.sync();  // every CTA's running max, sum and partial output are complete
+  for (int i = tid; i < CL * 8; i += 256) {
+    const int q = i / 8, h = i - q * 8;
+    pm[q][h] = cl.map_shared_rank(&mrun[0], q)[h];
+    pl[q][h] = cl.map_shared_rank(&lrun[0], q)[h];
+  }
+  __syncthreads();
+  float *outb = p.out + ((size_t)b * p.Hq + (size_t)g * G) * D;
+  const int e0 = G * D * r / CL, e1 = G * D * (r + 1) / CL;
+  for (int i = e0 + tid; i < e1; i += 256) {
+    const int h = i / D;
+    float Mx = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < CL; ++q) Mx = fmaxf(Mx, pm[q][h]);
+    float L = 0.0f, O = 0.0f;
+    if (Mx != -INFINITY) {
+      float part[CL];
+#pragma unroll
+      for (int q = 0; q < CL; ++q) part[q] = cl.map_shared_rank(osm, q)[i];
+#pragma unroll
+      for (int q = 0; q < CL; ++q) {
+        const float e = pm[q][h] == -INFINITY ? 0.0f : expf(pm[q][h] - Mx);
+        L = fmaf(pl[q][h], e, L);
+        O = fmaf(part[q], e, O);
+      }
+    }
+    outb[i] = L > 0.0f ? O / L : 0.0f;
+  }
+  cl.sync();  // the peers' shared memory stays valid until every CTA has read it
+}
+
+template <int D, int G, int CL>
+cudaError_t launch_mma_dg(const AttnParams &p, cudaStream_t s, int units) {
+  using M = MmaShape<D>;
+  auto kern = attention_mma_kernel<D, G, CL>;
+  static bool set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 64 || !set[dev]) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, M::SMEM);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)units * CL, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = M::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+template <int D, int CL>
+cudaError_t launch_mma_d(const AttnParams &p, cudaStream_t s, int units) {
+  switch (p.G) {
+    case 1: return launch_mma_dg<D, 1, CL>(p, s, units);
+    case 2: return launch_mma_dg<D, 2, CL>(p, s, units);
+    case 4: return launch_mma_dg<D, 4, CL>(p, s, units);
+    case 8: return launch_mma_dg<D, 8, CL>(p, s, units);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int CL>
+cudaError_t launch_mma_cl(const AttnParams &p, cudaStream_t s, int units) {
+  return p.D == 64 ? launch_mma_d<64, CL>(p, s, units) : launch_mma_d<128, CL>(p, s, units);
+}
+
 template <int D, int G, int CL>
 cudaError_t launch_dg(const AttnParams &p, cudaStream_t s, int units) {
   using S = AttnShape<D, G>;
@@ -362,6 +714,10 @@ bool attention_supported(int D, int G) {
   return (D == 64 || D == 128 || D == 256) && (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
 }
 
+bool attention_mma_supported(int D, int G) {
+  return (D == 64 || D == 128) && (G == 1 || G == 2 || G == 4 || G == 8);
+}
+
 cudaError_t launch_attention(const AttnParams &p, cudaStream_t s) {
   const int64_t units = (int64_t)p.B * p.Hkv;
   if (units * 16 > INT32_MAX) return cudaErrorInvalidValue;
@@ -377,6 +733,14 @@ cudaError_t launch_attention(const AttnParams &p, cudaStream_t s) {
   // 74 of 2)
   int cl = 1;
   while (cl < 8 && units * cl * 2 <= sms) cl *= 2;
+  if (p.mma) {
+    switch (cl) {
+      case 1: return launch_mma_cl<1>(p, s, (int)units);
+      case 2: return launch_mma_cl<2>(p, s, (int)units);
+      case 4: return launch_mma_cl<4>(p, s, (int)units);
+      default: return launch_mma_cl<8>(p, s, (int)units);
+    }
+  }
   switch (cl) {
     case 1: return launch_cl<1>(p, s, (int)units);
     case 2: return launch_cl<2>(p, s, (int)units);

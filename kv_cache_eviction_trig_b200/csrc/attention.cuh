@@ -5,7 +5,10 @@
 
 namespace tria {
 
-struct AttnParams {
+struct alignas(64) AttnParams {
+  CUtensorMap tk, tv;       // K and V as 2-D bf16 tensors [L*Hkv*cap][D], boxes of 64 x 128,
+                            // 128-byte swizzled (tensor-core path only)
+  int32_t mma;              // 1: the tensor-core path (tk and tv are valid)
   const uint16_t *q;        // bf16 [B][Hq][D]
   const uint16_t *k;        // bf16 [L][Hkv][cap][D]
   const uint16_t *v;
@@ -20,6 +23,8 @@ struct AttnParams {
 };
 
 bool attention_supported(int D, int G);
+// Whether the tensor-core path takes this shape (D = 64 or 128, G <= 8).
+bool attention_mma_supported(int D, int G);
 cudaError_t launch_attention(const AttnParams &p, cudaStream_t s);
 
 }  // namespace tria

@@ -589,8 +589,24 @@ tria_status tria_decode_attention(const tria_config *cfg, const tria_cache *cach
   if (attention_mma_supported(cfg->head_dim, ap.G) && rows <= INT32_MAX && rows > 0 &&
       aligned(cache->k, 16) && aligned(cache->v, 16) &&
       make_key_tensor_map(&ap.tk, cache->k, cfg->head_dim, rows, 128) == cudaSuccess &&
-      make_key_tensor_map(&ap.tv, cache->v, cfg->head_dim, rows, 128) == cudaSuccess)
+      make_key_tensor_map(&ap.tv, cache->v, cfg->head_dim, rows, 128) == cudaSuccess) {
     ap.mma = 1;
+    // Few (sequence, KV head) pairs: four clusters per pair when their partial results
+    // fit the raw-score region of the workspace (unused by this call); the arrival
+    // counters live in the workspace's zero-at-rest prefix.
+    const int64_t units = (int64_t)cfg->batch * cfg->n_kv_heads;
+    const size_t need = (size_t)units * 4 * (16 + 8 * (size_t)cfg->head_dim) * 4;
+    const size_t have = 4ull * cfg->num_layers * cfg->n_q_heads * (size_t)cache->cap_total;
+    int64_t most = 0;  // the longest segment: short ones are not worth the extra merge
+    for (int b = 0; b < cfg->batch; ++b)
+      most = std::max<int64_t>(most, cache->seq_start[b + 1] - cache->seq_start[b]);
+    if (units * 16 <= 148 && most >= 8192 && need <= have &&
+        (size_t)units * 4 <= kWsPrefix - kWsHist) {
+      ap.split = 4;
+      ap.scratch = w.raw();
+      ap.counters = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + kWsHist);
+    }
+  }
   return cuda_status(launch_attention(ap, static_cast<cudaStream_t>(stream)));
 }
 

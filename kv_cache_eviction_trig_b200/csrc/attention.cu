@@ -367,7 +367,7 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-template <int D, int G, int CL>
+template <int D, int G, int CL, int SPLIT>
 __global__ void __launch_bounds__(256, 1)
     attention_mma_kernel(const __grid_constant__ AttnParams p) {
   using M = MmaShape<D>;
@@ -387,16 +387,21 @@ __global__ void __launch_bounds__(256, 1)
 
   cg::cluster_group cl = cg::this_cluster();
   const int r = (int)cl.block_rank();
-  const int unit = blockIdx.x / CL;  // b * Hkv + g
+  const int ci = blockIdx.x / CL;                // cluster
+  const int unit = ci / SPLIT, half = ci % SPLIT;  // unit = b * Hkv + g
   const int b = unit / p.Hkv, g = unit - b * p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t cap_b = p.seg_start[b + 1] - p.seg_start[b];
   const int32_t T = p.unit_len ? p.unit_len[((int64_t)p.layer * p.Hkv + g) * p.B + b] : p.seq_len[b];
-  if (T < 0 || (int64_t)T > cap_b) {  // the same decision in every CTA of the cluster
-    if (r == 0 && tid == 0 && (g == 0 || p.unit_len)) dev::set_error(p.err, TRIA_DEVERR_SEQ_LEN);
+  if (T < 0 || (int64_t)T > cap_b) {  // the same decision in every CTA of the unit
+    if (r == 0 && half == 0 && tid == 0 && (g == 0 || p.unit_len))
+      dev::set_error(p.err, TRIA_DEVERR_SEQ_LEN);
     return;
   }
-  const int t0 = (int)((int64_t)T * r / CL), t1 = (int)((int64_t)T * (r + 1) / CL);
+  // the unit's keys are split over SPLIT * CL CTAs
+  const int part = half * CL + r;
+  const int t0 = (int)((int64_t)T * part / (SPLIT * CL));
+  const int t1 = (int)((int64_t)T * (part + 1) / (SPLIT * CL));
   const int ntiles = (t1 - t0 + TILE - 1) / TILE;
   // tensor row of the segment's slot 0 (the host checked that every row fits int32)
   const int32_t y0 = (int32_t)(((int64_t)p.layer * p.Hkv + g) * p.cap + p.seg_start[b]);
@@ -591,6 +596,17 @@ __global__ void __launch_bounds__(256, 1)
   }
   __syncthreads();
   float *outb = p.out + ((size_t)b * p.Hq + (size_t)g * G) * D;
+  // split 2: this cluster's result (its max, sum and unnormalised output per head)
+  float *mine = SPLIT > 1 ? p.scratch + ((size_t)unit * SPLIT + half) * (16 + 8 * D) : nullptr;
+  if (SPLIT > 1 && r == 0 && tid < G) {
+    float Mx = -INFINITY, L = 0.0f;
+    for (int q = 0; q < CL; ++q) Mx = fmaxf(Mx, pm[q][tid]);
+    if (Mx != -INFINITY)
+      for (int q = 0; q < CL; ++q)
+        L = fmaf(pl[q][tid], pm[q][tid] == -INFINITY ? 0.0f : expf(pm[q][tid] - Mx), L);
+    mine[tid] = Mx;
+    mine[8 + tid] = L;
+  }
   const int e0 = G * D * r / CL, e1 = G * D * (r + 1) / CL;
   for (int i = e0 + tid; i < e1; i += 256) {
     const int h = i / D;
@@ -609,15 +625,48 @@ __global__ void __launch_bounds__(256, 1)
         O = fmaf(part[q], e, O);
       }
     }
-    outb[i] = L > 0.0f ? O / L : 0.0f;
+    if (SPLIT > 1) mine[16 + i] = O;
+    else outb[i] = L > 0.0f ? O / L : 0.0f;
   }
   cl.sync();  // the peers' shared memory stays valid until every CTA has read it
+  if constexpr (SPLIT > 1) {
+    // the last of the unit's CTAs to finish merges the two clusters' results
+    __shared__ int last;
+    __threadfence();  // this thread's part of the cluster's result is visible device-wide
+    __syncthreads();
+    if (tid == 0) last = atomicAdd(p.counters + unit, 1) == SPLIT * CL - 1;
+    __syncthreads();
+    if (last) {
+      __threadfence();
+      const float *r0 = p.scratch + (size_t)unit * SPLIT * (16 + 8 * D);
+      for (int i = tid; i < G * D; i += 256) {
+        const int h = i / D;
+        float m[SPLIT], Mx = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < SPLIT; ++q) {
+          m[q] = __ldcg(r0 + q * (16 + 8 * D) + h);
+          Mx = fmaxf(Mx, m[q]);
+        }
+        float O = 0.0f, L = 0.0f;
+        if (Mx != -INFINITY) {
+#pragma unroll
+          for (int q = 0; q < SPLIT; ++q) {
+            const float a = m[q] == -INFINITY ? 0.0f : expf(m[q] - Mx);
+            L = fmaf(__ldcg(r0 + q * (16 + 8 * D) + 8 + h), a, L);
+            O = fmaf(__ldcg(r0 + q * (16 + 8 * D) + 16 + i), a, O);
+          }
+        }
+        outb[i] = L > 0.0f ? O / L : 0.0f;
+      }
+      if (tid == 0) p.counters[unit] = 0;  // zero at rest for the next call
+    }
+  }
 }
 
-template <int D, int G, int CL>
-cudaError_t launch_mma_dg(const AttnParams &p, cudaStream_t s, int units) {
+template <int D, int G, int CL, int SPLIT>
+cudaError_t launch_mma_dgs(const AttnParams &p, cudaStream_t s, int units) {
   using M = MmaShape<D>;
-  auto kern = attention_mma_kernel<D, G, CL>;
+  auto kern = attention_mma_kernel<D, G, CL, SPLIT>;
   static bool set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
@@ -628,7 +677,7 @@ cudaError_t launch_mma_dg(const AttnParams &p, cudaStream_t s, int units) {
     if (dev >= 0 && dev < 64) set[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)units * CL, 1, 1);
+  cfg.gridDim = dim3((unsigned)units * CL * SPLIT, 1, 1);
   cfg.blockDim = dim3(256, 1, 1);
   cfg.dynamicSmemBytes = M::SMEM;
   cfg.stream = s;
@@ -640,6 +689,14 @@ cudaError_t launch_mma_dg(const AttnParams &p, cudaStream_t s, int units) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+template <int D, int G, int CL>
+cudaError_t launch_mma_dg(const AttnParams &p, cudaStream_t s, int units) {
+  if constexpr (CL == 4) {
+    if (p.split == 4) return launch_mma_dgs<D, G, 4, 4>(p, s, units);
+  }
+  return launch_mma_dgs<D, G, CL, 1>(p, s, units);
 }
 
 template <int D, int CL>
@@ -734,11 +791,16 @@ cudaError_t launch_attention(const AttnParams &p, cudaStream_t s) {
   int cl = 1;
   while (cl < 8 && units * cl * 2 <= sms) cl *= 2;
   if (p.mma) {
+    // few (sequence, KV head) pairs: four 4-CTA clusters each (a B200 holds 33 such
+    // clusters at once, but only 15 of 8), merged by the unit's last CTA
+    if (p.split == 4 && units * 16 <= sms) return launch_mma_cl<4>(p, s, (int)units);
+    AttnParams q = p;
+    q.split = 1;
     switch (cl) {
-      case 1: return launch_mma_cl<1>(p, s, (int)units);
-      case 2: return launch_mma_cl<2>(p, s, (int)units);
-      case 4: return launch_mma_cl<4>(p, s, (int)units);
-      default: return launch_mma_cl<8>(p, s, (int)units);
+      case 1: return launch_mma_cl<1>(q, s, (int)units);
+      case 2: return launch_mma_cl<2>(q, s, (int)units);
+      case 4: return launch_mma_cl<4>(q, s, (int)units);
+      default: return launch_mma_cl<8>(q, s, (int)units);
     }
   }
   switch (cl) {

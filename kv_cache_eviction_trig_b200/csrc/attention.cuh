@@ -9,6 +9,9 @@ struct alignas(64) AttnParams {
   CUtensorMap tk, tv;       // K and V as 2-D bf16 tensors [L*Hkv*cap][D], boxes of 64 x 128,
                             // 128-byte swizzled (tensor-core path only)
   int32_t mma;              // 1: the tensor-core path (tk and tv are valid)
+  int32_t split;            // clusters per (sequence, KV head) on the tensor-core path (1 or 4)
+  float *scratch;           // split 4: [units][4][16 + 8 D] per-cluster partial results
+  int32_t *counters;        // split 4: [units] arrivals, zero at rest
   const uint16_t *q;        // bf16 [B][Hq][D]
   const uint16_t *k;        // bf16 [L][Hkv][cap][D]
   const uint16_t *v;

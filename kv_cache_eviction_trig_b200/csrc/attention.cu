@@ -9,7 +9,9 @@
 // surviving keys play no part.
 //
 // Design (sm_100a): one cluster of CL CTAs per (sequence, KV head), one CTA per
-// SM, CL the largest power of two (at most 8) that keeps the launch in one wave.  CTA r takes the r-th contiguous slice of the live keys
+// SM, CL the largest power of two (at most 8) that keeps the launch in one wave.
+// (On the tensor-core path, up to 9 pairs with a segment of 8192 slots or more take
+// four clusters of 4 each, whose results the pair's last CTA merges.)  CTA r takes the r-th contiguous slice of the live keys
 // and walks it in tiles of 16384 / D keys with a running maximum (online
 // softmax) for all G query heads of the group, so the group's keys and values are
 // read from HBM once.  The tiles stream into three shared-memory stages with bulk

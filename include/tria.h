@@ -242,8 +242,11 @@ tria_status tria_append(const tria_config *cfg, const tria_cache *cache, const v
  * aligned; out is DEVICE float32 [B][Hq][D]; a sequence with seq_len 0 gets
  * zeros.  Accumulates in float32 with a running maximum (no overflow for any
  * finite logits).  A seq_len out of range sets TRIA_DEVERR_SEQ_LEN and that
- * sequence's rows are not written.  ws as for the other calls (only its error
- * word is used). */
+ * sequence's rows are not written.  ws as for the other calls, sized for this
+ * cfg and cache: besides its error word, a call over few (sequence, KV head)
+ * pairs with long segments uses the workspace's raw-score region for partial
+ * results and leaves the words it counts with back at zero.  Like every call,
+ * it must not overlap another call on the same workspace. */
 tria_status tria_decode_attention(const tria_config *cfg, const tria_cache *cache, int32_t layer,
                                   const void *q, float scale, float *out, void *ws,
                                   size_t ws_bytes, void *stream);

@@ -3,7 +3,10 @@
 One step = one tria_prune over the whole synthetic workload (score every key,
 z-score + GQA max, select the top budget, compact K/V/pos in place).  Before
 every timed step the pruned rows are restored from a pristine copy and L2 is
-flushed by writing a 512 MiB buffer; neither is inside the timed spans.
+flushed: a 512 MiB buffer is written, then another 512 MiB buffer is read, so the
+cache holds only clean lines of unrelated data (the write-backs of the first
+buffer's dirty lines would otherwise land in the timed span).  Neither is timed;
+the figures with the write alone are reported beside the main ones.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl ours|reference]
 
@@ -319,10 +322,30 @@ def _traffic(kernel, key):
     return None
 
 
+L2_NOTE = ("flushed before every step: 512 MiB written, then another 512 MiB read "
+           "(L2 left holding clean lines of unrelated data)")
+
+
+class L2Flush:
+    """Evicts every line of L2 (126 MB on a B200): a 512 MiB buffer is written, then
+    (unless write_only) a second 512 MiB buffer is read, so that the dirty lines of the
+    first are written back here rather than inside the next timed span."""
+
+    def __init__(self, dev):
+        self.buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        self.other = torch.ones(64 << 20, dtype=torch.int64, device=dev)
+        self.sink = torch.empty(1, dtype=torch.int64, device=dev)
+
+    def __call__(self, write_only=False):
+        self.buf.fill_(1)
+        if not write_only:
+            torch.amax(self.other, dim=0, keepdim=True, out=self.sink)
+
+
 class Bench:
     """One workload resident on the device, ready to be pruned again and again:
     before every step the rows a prune overwrites are restored from a pristine
-    copy and L2 is flushed (512 MiB written); neither is timed."""
+    copy and L2 is flushed (L2Flush); neither is timed."""
 
     def __init__(self, wl, dev, flags=0):
         self.wl, self.dev = wl, dev
@@ -339,15 +362,15 @@ class Bench:
         self.backup = {n: [data[n][:, :, s:s + c].clone() for s, c in self.restore]
                        for n in ("k", "v", "pos")}
         self.seq_len0 = data["seq_len"].clone()
-        self.flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        self.flush = L2Flush(dev)
         self.stream = torch.cuda.current_stream()
 
-    def reset(self):
+    def reset(self, write_only=False):
         for n in ("k", "v", "pos"):
             for (s, c), t in zip(self.restore, self.backup[n]):
                 self.data[n][:, :, s:s + c].copy_(t)
         self.data["seq_len"].copy_(self.seq_len0)
-        self.flush.fill_(1)
+        self.flush(write_only)
 
     def prune(self):
         tria.tria_prune(self.cfg, self.stats, self.cache, self.ws, stream=self.stream)
@@ -363,11 +386,11 @@ class Bench:
         if self.data["seq_len"].tolist() != want:
             raise RuntimeError(f"pruned lengths differ on {self.wl.name}")
 
-    def timed(self, steps):
+    def timed(self, steps, write_only=False):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(steps)]
         for i in range(steps):
-            self.reset()
+            self.reset(write_only)
             ev[i][0].record(self.stream)
             self.prune()
             ev[i][1].record(self.stream)
@@ -423,7 +446,8 @@ class Bench:
 def attention_figures(dev, B, T, steps, peak):
     """tria_decode_attention on one 8B-shaped layer (8 KV heads x 4 query heads, D = 128)
     with B sequences of T live keys, L2 flushed before every call: mean device time and
-    HBM rate (K and V of the live slots read once)."""
+    HBM rate (K and V of the live slots read once); also the time with the flush's write
+    alone."""
     H, Hq, D = 8, 32, 128
     gen = torch.Generator(device=dev).manual_seed(B * 100003 + T)
     k = torch.randn(1, H, B * T, D, device=dev, generator=gen).to(torch.bfloat16)
@@ -436,24 +460,30 @@ def attention_figures(dev, B, T, steps, peak):
     ws = tria.workspace(cfg, cache)
     q = torch.randn(B, Hq, D, device=dev, generator=gen).to(torch.bfloat16)
     out = torch.empty(B, Hq, D, device=dev)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
     for _ in range(3):
         tria.tria_decode_attention(cfg, cache, 0, q, out, ws, stream=stream)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(steps)]
-    for a, b in ev:
-        flush.fill_(1)
-        a.record(stream)
-        tria.tria_decode_attention(cfg, cache, 0, q, out, ws, stream=stream)
-        b.record(stream)
-    torch.cuda.synchronize()
+
+    def run(write_only):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for a, b in ev:
+            flush(write_only)
+            a.record(stream)
+            tria.tria_decode_attention(cfg, cache, 0, q, out, ws, stream=stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    ms, ms_w = run(False), run(True)
     if tria.tria_get_device_error(ws) != 0:
         raise RuntimeError("device error flag set in decode attention")
-    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     algo = B * H * T * 4 * D
     return {"batch": B, "live_keys": T, "us": ms * 1e3, "gbs": algo / (ms / 1e3) / 1e9,
-            "frac": algo / (ms / 1e3) / 1e9 / peak, "algorithmic_bytes": algo, "steps": steps}
+            "frac": algo / (ms / 1e3) / 1e9 / peak, "algorithmic_bytes": algo, "steps": steps,
+            "us_write_only_flush": ms_w * 1e3,
+            "frac_write_only_flush": algo / (ms_w / 1e3) / 1e9 / peak}
 
 
 def run_ours(args):
@@ -479,6 +509,8 @@ def run_ours(args):
     clocks = clk.summary()
     sm_mhz = clocks["sm_mhz"] if clocks else None
     names, kern_ms = bench.kernels(args.steps)
+    # the same steps with the flush's write alone (its dirty lines written back in the span)
+    wo_ms = bench.timed(args.steps, write_only=True)
 
     # ---- end to end through the C ABI with host buffers (pinned), copies timed
     data, restore, backup = bench.data, bench.restore, bench.backup
@@ -501,7 +533,7 @@ def run_ours(args):
            for _ in range(e2e_steps)]
     stream = bench.stream
     for i in range(e2e_steps):
-        bench.flush.fill_(1)
+        bench.flush()
         eev[i][0].record(stream)
         for n in ("k", "v", "pos", "seq_len", "cur_pos"):
             data[n].copy_(host[n], non_blocking=True)
@@ -518,8 +550,8 @@ def run_ours(args):
         raise RuntimeError("device error flag set during the timed runs")
 
     total_ms = sum(step_ms)
-    red = max_over_ranks([total_ms, e2e_ms] + kern_ms, device=dev)
-    total_ms, e2e_ms, kern_ms = red[0], red[1], red[2:]
+    red = max_over_ranks([total_ms, e2e_ms, sum(wo_ms)] + kern_ms, device=dev)
+    total_ms, e2e_ms, wo_total, kern_ms = red[0], red[1], red[2], red[3:]
     step = total_ms / args.steps
     head = bench.summary([step], names, kern_ms, peak, sm_mhz)
     keys = wl.keys_scored
@@ -537,7 +569,7 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded; pages' shapes and value distributions)",
-        "config": dict(wl.describe(), l2="flushed: 512 MiB write before every step",
+        "config": dict(wl.describe(), l2=L2_NOTE,
                        parallelism=f"dp{world} (independent caches per GPU)"),
         "hbm_gbs_path": head["hbm_gbs_path"],
         "frac_path": head["frac_path"],
@@ -553,6 +585,8 @@ def run_ours(args):
         "e2e": {"value": keys * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": len(names) * args.steps,
+        "l2_write_only_flush": {"ms_per_step": wo_total / args.steps,
+                                "value": keys * world / (wo_total / args.steps / 1e3)},
     }
     host_stats = [t.cpu() for t in bench.stats.tensors]
     bench.free()

@@ -394,6 +394,20 @@ __global__ void __launch_bounds__(256, 1)
   const int b = unit / p.Hkv, g = unit - b * p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t cap_b = p.seg_start[b + 1] - p.seg_start[b];
+  // the queries (bf16 [8][D], heads past G zero) load alongside the live length
+  constexpr int QW = 4 * D / 256;  // 32-bit words of the queries per thread
+  const uint16_t *qb = p.q + ((size_t)b * p.Hq + (size_t)g * G) * D;
+  uint32_t qv[QW];
+#pragma unroll
+  for (int k = 0; k < QW; ++k) {
+    const int w = tid + 256 * k;
+    qv[k] = w < G * D / 2 ? reinterpret_cast<const uint32_t *>(qb)[w] : 0u;
+  }
+  if (tid == 0) {
+    // the tensor maps' descriptors travel to the TMA unit meanwhile
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tk)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tv)) : "memory");
+  }
   const int32_t T = p.unit_len ? p.unit_len[((int64_t)p.layer * p.Hkv + g) * p.B + b] : p.seq_len[b];
   if (T < 0 || (int64_t)T > cap_b) {  // the same decision in every CTA of the unit
     if (r == 0 && half == 0 && tid == 0 && (g == 0 || p.unit_len))
@@ -407,20 +421,7 @@ __global__ void __launch_bounds__(256, 1)
   const int ntiles = (t1 - t0 + TILE - 1) / TILE;
   // tensor row of the segment's slot 0 (the host checked that every row fits int32)
   const int32_t y0 = (int32_t)(((int64_t)p.layer * p.Hkv + g) * p.cap + p.seg_start[b]);
-  const uint16_t *qb = p.q + ((size_t)b * p.Hq + (size_t)g * G) * D;
 
-  if (tid == 0) {
-#pragma unroll
-    for (int q = 0; q < NST; ++q) dev::mbar_init(&bar[q], 1);
-    dev::fence_mbar_init();
-    all_ok = 1;
-  }
-  for (int i = tid; i < 8 * D; i += 256) qsm[i] = i < G * D ? qb[i] : (uint16_t)0;
-  if (tid < 8) {
-    mrun[tid] = -INFINITY;
-    lrun[tid] = 0.0f;
-  }
-  __syncthreads();
   auto issue = [&](int i) {  // thread 0: tile i into stage i % NST
     const int s = i % NST;
     uint8_t *st = sm + s * M::STAGE;
@@ -435,8 +436,20 @@ __global__ void __launch_bounds__(256, 1)
       dev::tma_load_2d(st + M::TB + bx * M::BOXB, &p.tv, bx * 64, y, &bar[s]);
     }
   };
-  if (tid == 0)
-    for (int i = 0; i < NST && i < ntiles; ++i) issue(i);
+  if (tid == 0) {
+#pragma unroll
+    for (int q = 0; q < NST; ++q) dev::mbar_init(&bar[q], 1);
+    dev::fence_mbar_init();
+    all_ok = 1;
+    for (int i = 0; i < NST && i < ntiles; ++i) issue(i);  // before the queries are stored
+  }
+#pragma unroll
+  for (int k = 0; k < QW; ++k) reinterpret_cast<uint32_t *>(qsm)[tid + 256 * k] = qv[k];
+  if (tid < 8) {
+    mrun[tid] = -INFINITY;
+    lrun[tid] = 0.0f;
+  }
+  __syncthreads();
 
   // queries as the B operand of S^T = K Q^T, one fragment pair per 16 dims
   uint32_t qf[KS][2];
@@ -446,7 +459,8 @@ __global__ void __launch_bounds__(256, 1)
     for (int t = 0; t < KS; ++t) ldsm_x2(qa + t * 32, qf[t]);
   }
   const int hA = 2 * (lane & 3), hB = hA + 1;  // the heads of this lane's accumulators
-  float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};       // O^T: dims dm + lane / 4 (+ 8), heads hA, hB
+  // O^T: dims dm + lane / 4 (+ 8), heads hA, hB; the P hi and lo products apart
+  float o[4] = {0.0f, 0.0f, 0.0f, 0.0f}, ol[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   const int dm = D == 128 ? 16 * warp : 16 * (warp & 3);
   const int j0 = D == 128 ? 0 : 4 * (warp >> 2), j1 = D == 128 ? 8 : j0 + 4;
   const uint32_t pth = dev::smem_addr(pt), ptl = pth + 8 * M::PROW;
@@ -465,14 +479,20 @@ __global__ void __launch_bounds__(256, 1)
     // S^T for keys [16 warp, 16 warp + 16)
     float sacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     {
+      // even and odd 16-dim steps in two accumulator chains
+      float s2[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       const int mat = lane >> 3, key = 16 * warp + (mat & 1) * 8 + (lane & 7);
       const uint32_t kb = dev::smem_addr(ks);
 #pragma unroll
-      for (int t = 0; t < KS; ++t) {
-        uint32_t a[4];
+      for (int t = 0; t < KS; t += 2) {
+        uint32_t a[4], a2[4];
         ldsm_x4(swz<M::BOXB>(kb, key, 16 * t + (mat >> 1) * 8), a);
+        ldsm_x4(swz<M::BOXB>(kb, key, 16 * (t + 1) + (mat >> 1) * 8), a2);
         mma_bf16(sacc, a, qf[t]);
+        mma_bf16(s2, a2, qf[t + 1]);
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[e] += s2[e];
     }
     const int keyA = 16 * warp + (lane >> 2), keyB = keyA + 8;
     float sv[4];
@@ -543,6 +563,10 @@ __global__ void __launch_bounds__(256, 1)
     o[1] *= alB;
     o[2] *= alA;
     o[3] *= alB;
+    ol[0] *= alA;
+    ol[1] *= alB;
+    ol[2] *= alA;
+    ol[3] *= alB;
     {
       const int mat = lane >> 3;
       const uint32_t vb = dev::smem_addr(vs);
@@ -554,7 +578,7 @@ __global__ void __launch_bounds__(256, 1)
         ldsm_x2(pth + pa + 32 * j, bh);
         ldsm_x2(ptl + pa + 32 * j, bl);
         mma_bf16(o, a, bh);
-        mma_bf16(o, a, bl);
+        mma_bf16(ol, a, bl);
       }
     }
     if (tid < 8) {  // running max and sum of head tid (every thread has read them)
@@ -572,6 +596,8 @@ __global__ void __launch_bounds__(256, 1)
     __syncthreads();  // stage s, P^T and the warp arrays are free again
     if (tid == 0 && i + NST < ntiles) issue(i + NST);
   }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) o[e] += ol[e];
   // this CTA's unnormalised output O[h][d] (D = 64: the two key halves added in order)
   const int dA = dm + (lane >> 2), dB = dA + 8;
   if (D == 128 || warp < 4) {
@@ -598,7 +624,7 @@ __global__ void __launch_bounds__(256, 1)
   }
   __syncthreads();
   float *outb = p.out + ((size_t)b * p.Hq + (size_t)g * G) * D;
-  // split 2: this cluster's result (its max, sum and unnormalised output per head)
+  // SPLIT > 1: this cluster's result (its max, sum and unnormalised output per head)
   float *mine = SPLIT > 1 ? p.scratch + ((size_t)unit * SPLIT + half) * (16 + 8 * D) : nullptr;
   if (SPLIT > 1 && r == 0 && tid < G) {
     float Mx = -INFINITY, L = 0.0f;
@@ -632,7 +658,7 @@ __global__ void __launch_bounds__(256, 1)
   }
   cl.sync();  // the peers' shared memory stays valid until every CTA has read it
   if constexpr (SPLIT > 1) {
-    // the last of the unit's CTAs to finish merges the two clusters' results
+    // the last of the unit's CTAs to finish merges the SPLIT clusters' results
     __shared__ int last;
     __threadfence();  // this thread's part of the cluster's result is visible device-wide
     __syncthreads();
@@ -643,19 +669,22 @@ __global__ void __launch_bounds__(256, 1)
       const float *r0 = p.scratch + (size_t)unit * SPLIT * (16 + 8 * D);
       for (int i = tid; i < G * D; i += 256) {
         const int h = i / D;
-        float m[SPLIT], Mx = -INFINITY;
+        float m[SPLIT], l[SPLIT], oq[SPLIT], Mx = -INFINITY;
 #pragma unroll
-        for (int q = 0; q < SPLIT; ++q) {
+        for (int q = 0; q < SPLIT; ++q) {  // every load issued before any is used
           m[q] = __ldcg(r0 + q * (16 + 8 * D) + h);
-          Mx = fmaxf(Mx, m[q]);
+          l[q] = __ldcg(r0 + q * (16 + 8 * D) + 8 + h);
+          oq[q] = __ldcg(r0 + q * (16 + 8 * D) + 16 + i);
         }
+#pragma unroll
+        for (int q = 0; q < SPLIT; ++q) Mx = fmaxf(Mx, m[q]);
         float O = 0.0f, L = 0.0f;
         if (Mx != -INFINITY) {
 #pragma unroll
           for (int q = 0; q < SPLIT; ++q) {
             const float a = m[q] == -INFINITY ? 0.0f : expf(m[q] - Mx);
-            L = fmaf(__ldcg(r0 + q * (16 + 8 * D) + 8 + h), a, L);
-            O = fmaf(__ldcg(r0 + q * (16 + 8 * D) + 16 + i), a, O);
+            L = fmaf(l[q], a, L);
+            O = fmaf(oq[q], a, O);
           }
         }
         outb[i] = L > 0.0f ? O / L : 0.0f;

@@ -237,15 +237,21 @@ ATT_CASES = {
     "d128_g16_with_empty": lambda: small("att4", Hq=16, Hkv=1, B=2, seq_lens=[130, 0]),
     "d64_interleaved_g2": lambda: small("att5", D=64, Hq=4, Hkv=2, seq_lens=[700], theta=1e4,
                                         rope_layout=workloads.INTERLEAVED),
-    # long slices: every CTA of an 8-CTA cluster streams more tiles than it has stages
-    # (the stages are reused), with a ragged last tile
+    # long segments over few (sequence, KV head) pairs: on the tensor-core path each pair's
+    # keys spread over four 4-CTA clusters (stages reused), merged by the pair's last CTA;
+    # a ragged last tile
     "d128_g4_long": lambda: small("att6", Hq=8, Hkv=2, seq_lens=[12001]),
     "d64_g2_long": lambda: small("att7", D=64, Hq=4, Hkv=2, seq_lens=[9000], theta=1e4),
     # G = 16 at D = 256 scores in two passes of 8 query heads
     "d256_g16_long": lambda: small("att8", D=256, Hq=16, Hkv=1, seq_lens=[3000]),
-    # more (sequence, KV head) pairs than SMs: one CTA per pair, no cluster
+    # more pairs than SMs, ragged: one CTA per pair, no cluster
     "d128_g4_many_sequences": lambda: small("att9", B=80, Hq=8, Hkv=2,
                                             seq_lens=[700 - (b % 7) * 50 for b in range(80)]),
+    # empty sequences around a long one: zero rows from split pairs with nothing to merge
+    "d128_g4_empty_and_long": lambda: small("att10", Hq=8, Hkv=2, B=3, seq_lens=[0, 20000, 0]),
+    # many pairs (1040): one CTA per pair, several waves
+    "d64_g4_over_1024_pairs": lambda: small("att11", D=64, Hq=32, Hkv=8, B=130, theta=1e4,
+                                            seq_lens=[1 + (b * 37) % 300 for b in range(130)]),
 }
 
 

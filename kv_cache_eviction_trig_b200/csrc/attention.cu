@@ -31,6 +31,7 @@
 #include <math.h>
 
 #include "attention.cuh"
+#include "mma_sync.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -340,34 +341,6 @@ struct MmaShape {
   static constexpr int SMEM = OFF_BAR + 8 * NST + 1024;  // + room to align to 1024
   static_assert(D == 64 || D == 128, "tensor-core path");
 };
-
-// Address of the 16-byte unit holding dims [dim, dim + 8) of row `row` of a tile
-// stored as 128-byte-swizzled TMA boxes of 64 dims.
-template <int BOXB>
-__device__ __forceinline__ uint32_t swz(uint32_t base, int row, int dim) {
-  return base + (uint32_t)(dim >> 6) * BOXB + (uint32_t)row * 128u +
-         ((uint32_t)(((dim >> 3) & 7) ^ (row & 7)) << 4);
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t (&r)[2]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
-               : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
-}
-__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
 
 template <int D, int G, int CL, int SPLIT>
 __global__ void __launch_bounds__(256, 1)

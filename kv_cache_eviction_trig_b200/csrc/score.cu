@@ -26,6 +26,7 @@
 
 #include <mutex>
 
+#include "mma_sync.cuh"
 #include "tria_internal.cuh"
 
 namespace tria {
@@ -136,7 +137,142 @@ __device__ __forceinline__ void fma3(float2 &acc, float2 wx, float2 wy, float2 w
   acc = __ffma2_rn(wn, n, acc);
 }
 
+// ---------------------------------------------------------------- tensor-core form
+// For D = 64 or 128 and G <= 8 a warp scores each 16-key block of its chunk with
+// mma.sync m16n8k16 (bf16 operands, float32 accumulators) instead of per-lane FMAs:
+//   s = K Wt + Nrm Wn
+// K the 16 x D block of stored keys straight from the swizzled chunk (exact bf16),
+// Wt (D x 2G) the trigonometric weights on every stored dim (Re W_f on x_f, Im W_f on
+// y_f), Nrm (16 x F) the norms |k_f| and Wn (F x 2G) the norm weights.  Each float32
+// weight enters as a bf16 pair hi + lo in columns h and G + h (so s_h is column h
+// plus column G + h, 16 significant bits of every weight); each norm enters as a
+// bf16 pair too (Nrm_hi and Nrm_lo, two MMAs), so the products keep float32-level
+// accuracy.  The norms are formed from the A fragments of K themselves: with the
+// half-split layout x_f and y_f sit at the same fragment position of the k-steps t
+// and t + D/32; with the interleaved layout one register holds (x_f, y_f), and the
+// norm matrix takes its frequencies in the order the registers hold them
+// (column 2q + e of freq step u is f = 16u + q + 4e, column 2q + 8 + e is
+// f = 16u + 8 + q + 4e), which the norm weights follow.
+template <int D, int G>
+struct TcShape {
+  static constexpr int F = D / 2;
+  static constexpr int KS = D / 16;                // k-steps over the stored dims
+  static constexpr int FS = F / 16;                // k-steps over the frequencies
+  static constexpr int NB = 2 * G > 8 ? 2 * G / 8 : 1;  // n-blocks of 8 columns
+};
+
+// Frequency of column kk (0..15) of frequency step u of the norm matrix.
+template <int LAYOUT>
+__device__ __forceinline__ int norm_freq(int u, int kk) {
+  if constexpr (LAYOUT == TRIA_ROPE_HALF_SPLIT) return 16 * u + kk;
+  else return 16 * u + 8 * (kk >> 3) + ((kk & 7) >> 1) + 4 * (kk & 1);
+}
+
+// This lane's B fragments of Wt and Wn from the unit's float weights in shared
+// memory ([F/2][G][6]: Re W, Re W, Im W, Im W, Nw, Nw for the pairs 2fp, 2fp+1).
 template <int D, int G, int LAYOUT>
+__device__ __forceinline__ void tc_weights(const float *wu, int lane,
+                                           uint32_t (&bt)[TcShape<D, G>::KS][TcShape<D, G>::NB][2],
+                                           uint32_t (&bn)[TcShape<D, G>::FS][TcShape<D, G>::NB][2]) {
+  using T = TcShape<D, G>;
+  constexpr int F = T::F;
+  const int k0 = 2 * (lane & 3);
+  auto col = [&](int nb, float w) -> float {  // hi or lo part of weight w for this lane's column
+    const int c = 8 * nb + (lane >> 2);
+    if (c >= 2 * G) return 0.0f;
+    const float hi = dev::bf16lo(pack_bf16x2(w, 0.0f));  // w rounded to bf16
+    return c < G ? hi : w - hi;
+  };
+  auto head = [&](int nb) { const int c = 8 * nb + (lane >> 2); return c < G ? c : (c < 2 * G ? c - G : 0); };
+  auto wt = [&](int d, int h) -> float {  // weight on stored dim d for head h
+    int f, im;
+    if constexpr (LAYOUT == TRIA_ROPE_HALF_SPLIT) { f = d < F ? d : d - F; im = d >= F; }
+    else { f = d >> 1; im = d & 1; }
+    return wu[(f >> 1) * 6 * G + 6 * h + 2 * im + (f & 1)];
+  };
+  auto wn = [&](int f, int h) -> float { return wu[(f >> 1) * 6 * G + 6 * h + 4 + (f & 1)]; };
+#pragma unroll
+  for (int nb = 0; nb < T::NB; ++nb) {
+    const int h = head(nb);
+#pragma unroll
+    for (int t = 0; t < T::KS; ++t) {
+      const int d = 16 * t + k0;
+      bt[t][nb][0] = pack_bf16x2(col(nb, wt(d, h)), col(nb, wt(d + 1, h)));
+      bt[t][nb][1] = pack_bf16x2(col(nb, wt(d + 8, h)), col(nb, wt(d + 9, h)));
+    }
+#pragma unroll
+    for (int u = 0; u < T::FS; ++u) {
+      bn[u][nb][0] = pack_bf16x2(col(nb, wn(norm_freq<LAYOUT>(u, k0), h)),
+                                 col(nb, wn(norm_freq<LAYOUT>(u, k0 + 1), h)));
+      bn[u][nb][1] = pack_bf16x2(col(nb, wn(norm_freq<LAYOUT>(u, k0 + 8), h)),
+                                 col(nb, wn(norm_freq<LAYOUT>(u, k0 + 9), h)));
+    }
+  }
+}
+
+// Norms of two (x, y) pairs given as bf16 pairs of x and of y, as the bf16 pairs
+// hi and lo of the norm matrix.
+__device__ __forceinline__ void tc_norms(uint32_t xw, uint32_t yw, uint32_t &hi, uint32_t &lo) {
+  const float2 X = bf16x2_to_f2(xw), Y = bf16x2_to_f2(yw);
+  const float2 n2 = __ffma2_rn(Y, Y, __fmul2_rn(X, X));
+  const float na = sqrt_approx(n2.x), nb = sqrt_approx(n2.y);
+  hi = pack_bf16x2(na, nb);
+  const float2 h = bf16x2_to_f2(hi);
+  lo = pack_bf16x2(na - h.x, nb - h.y);
+}
+
+// Accumulators of 16 keys (rows mb*16 ..) of a chunk at shared address cs for all
+// 2G columns: acc[nb] as the C fragment of n-block nb.
+template <int D, int G, int LAYOUT, int BOXB>
+__device__ __forceinline__ void tc_block(uint32_t cs, int mb, int lane,
+                                         const uint32_t (&bt)[TcShape<D, G>::KS][TcShape<D, G>::NB][2],
+                                         const uint32_t (&bn)[TcShape<D, G>::FS][TcShape<D, G>::NB][2],
+                                         float (&acc)[TcShape<D, G>::NB][4]) {
+  using T = TcShape<D, G>;
+  uint32_t a[T::KS][4];
+  {
+    const int mat = lane >> 3, key = 16 * mb + (mat & 1) * 8 + (lane & 7);
+#pragma unroll
+    for (int t = 0; t < T::KS; ++t) ldsm_x4(swz<BOXB>(cs, key, 16 * t + (mat >> 1) * 8), a[t]);
+  }
+  float an[T::NB][4];
+#pragma unroll
+  for (int nb = 0; nb < T::NB; ++nb)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nb][e] = an[nb][e] = 0.0f;
+#pragma unroll
+  for (int t = 0; t < T::KS; ++t)
+#pragma unroll
+    for (int nb = 0; nb < T::NB; ++nb) mma_bf16(acc[nb], a[t], bt[t][nb]);
+#pragma unroll
+  for (int u = 0; u < T::FS; ++u) {
+    uint32_t nh[4], nl[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      if constexpr (LAYOUT == TRIA_ROPE_HALF_SPLIT) {
+        tc_norms(a[u][r], a[u + T::KS / 2][r], nh[r], nl[r]);
+      } else {
+        // registers r (rows r0 or r0 + 8) of k-steps 2u (r < 2) and 2u + 1 (r >= 2): a
+        // register holds (x_f, y_f); two of them give the pair of norms of columns
+        // (2q, 2q + 1) resp. (2q + 8, 2q + 9)
+        const uint32_t *ka = a[2 * u + (r >> 1)];
+        const uint32_t wa = ka[r & 1], wb = ka[(r & 1) + 2];
+        tc_norms(__byte_perm(wa, wb, 0x5410), __byte_perm(wa, wb, 0x7632), nh[r], nl[r]);
+      }
+    }
+#pragma unroll
+    for (int nb = 0; nb < T::NB; ++nb) {
+      mma_bf16(an[nb], nh, bn[u][nb]);
+      mma_bf16(an[nb], nl, bn[u][nb]);
+    }
+  }
+#pragma unroll
+  for (int nb = 0; nb < T::NB; ++nb)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nb][e] += an[nb][e];
+}
+
+template <int D, int G, int LAYOUT, bool TCF>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ ScoreParams p) {
   using S = ScoreShape<D, G>;
@@ -332,6 +468,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
   // ------------------------------------------------------------------ consumers
   int wseen = -1;  // weight slot and fill parity last waited for
+  // the tensor-core form's B fragments of the current weights, and their tag
+  constexpr bool TC = TCF && (D == 64 || D == 128) && G <= 8 && CH % 16 == 0;
+  using TS = TcShape<D, G>;
+  uint32_t bt[TC ? TS::KS : 1][TC ? TS::NB : 1][2], bn[TC ? TS::FS : 1][TC ? TS::NB : 1][2];
+  int ftag = -1;
   // float64 sums of s and s^2 of this lane's keys for the current unit; each warp
   // writes one entry per unit its CTA's chunk run meets (zeros where it had none)
   int u_first = 0, u_last = -1, first_unit = -1;  // set after the warm-up
@@ -409,7 +550,57 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     }
     const float *wu = reinterpret_cast<const float *>(wring + (wtag & 1) * WB);
     const uint8_t *chunk = ring + (size_t)s * CB;
+    const int l = row / p.Hkv, g = row - l * p.Hkv;
+    float *rawp = p.raw + ((size_t)l * p.Hq + (size_t)g * G) * p.cap + p.seg_start[b] + key0;
 
+    if constexpr (TC) {
+      if (wtag != ftag) {  // the unit's weights as this lane's B fragments
+        tc_weights<D, G, LAYOUT>(wu, lane, bt, bn);
+        ftag = wtag;
+      }
+      const uint32_t cs = dev::smem_addr(chunk);
+      const int q4 = lane & 3, r0 = lane >> 2;
+      const int nmb = warm ? 1 : CH / 16;
+#pragma unroll 1
+      for (int mb = 0; mb < nmb; ++mb) {
+        float acc[TcShape<D, G>::NB][4];
+        tc_block<D, G, LAYOUT, S::BOXB>(cs, mb, lane, bt, bn, acc);
+        // s_h = column h + column G + h: this lane ends with heads 2 q4, 2 q4 + 1 of keys
+        // r0 and r0 + 8 (G >= 2), or head 0 (G = 1)
+        float v[4];
+        if constexpr (G == 8) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) v[e] = acc[0][e] + acc[1][e];
+        } else if constexpr (G == 4 || G == 2) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) v[e] = acc[0][e] + __shfl_xor_sync(0xffffffffu, acc[0][e], G / 2);
+        } else {
+          v[0] = acc[0][0] + acc[0][1];
+          v[2] = acc[0][2] + acc[0][3];
+          v[1] = v[3] = 0.0f;
+        }
+        if (G == 1 ? q4 == 0 : 2 * q4 < G) {
+          const int hA = G == 1 ? 0 : 2 * q4;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int r = 16 * mb + r0 + 8 * half;
+            if (r < n) {
+#pragma unroll
+              for (int e = 0; e < (G == 1 ? 1 : 2); ++e) {
+                const float x = v[2 * half + e];
+                rawp[(size_t)(hA + e) * p.cap + r] = x;
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+                  if (h == hA + e) {
+                    s1[h] += (double)x;
+                    s2[h] = fma((double)x, (double)x, s2[h]);
+                  }
+              }
+            }
+          }
+        }
+      }
+    } else {
     float2 acc[KPT][G];
 #pragma unroll
     for (int k = 0; k < KPT; ++k)
@@ -456,8 +647,6 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
       }
     }
-    const int l = row / p.Hkv, g = row - l * p.Hkv;
-    float *rawp = p.raw + ((size_t)l * p.Hq + (size_t)g * G) * p.cap + p.seg_start[b] + key0;
 #pragma unroll
     for (int k = 0; k < KPT; ++k) {
       const int r = lane + 32 * k;
@@ -471,8 +660,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
       }
     }
+    }  // the FMA form
     if (warm) {
       warm = false;
+      ftag = -1;  // the warm-up built fragments from whatever the weight slot held
       dev::named_barrier_arrive(2, (NW + 1) * 32);  // the producer may start the stream
       {
         int row, b, j;
@@ -508,13 +699,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   }
 }
 
-template <int D, int G, int LAYOUT>
+template <int D, int G, int LAYOUT, bool TCF>
 static cudaError_t launch_one(const ScoreParams &p, int grid, cudaStream_t s, bool pdl) {
   using S = ScoreShape<D, G>;
   if constexpr (!S::OK) {
     return cudaErrorInvalidValue;
   } else {
-    auto kern = score_kernel<D, G, LAYOUT>;
+    auto kern = score_kernel<D, G, LAYOUT, TCF>;
     static bool configured[64] = {};  // per device: the attribute is set once per process
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
@@ -538,14 +729,28 @@ static cudaError_t launch_one(const ScoreParams &p, int grid, cudaStream_t s, bo
   }
 }
 
+// The tensor-core form costs more per CTA (a larger warm-up, fragment builds per unit)
+// and less per key: on a B200 it is ahead for G = 8, and for smaller groups once a CTA
+// scores kScoreTcChunks chunks or more (one 8B-shaped layer, 28 chunks per CTA: 27.2
+// against 28.8 us; 36 layers, about 1000 per CTA: 488 against 457 us).
+constexpr int kScoreTcChunks = 64;
+
+template <int D, int G, int LAYOUT>
+static cudaError_t launch_g(const ScoreParams &p, int grid, cudaStream_t s, bool pdl) {
+  if constexpr ((D == 64 || D == 128) && G <= 8) {
+    if (G == 8 || p.chunks_per_cta >= kScoreTcChunks) return launch_one<D, G, LAYOUT, true>(p, grid, s, pdl);
+  }
+  return launch_one<D, G, LAYOUT, false>(p, grid, s, pdl);
+}
+
 template <int D, int LAYOUT>
 static cudaError_t dispatch_g(const ScoreParams &p, int G, int grid, cudaStream_t s, bool pdl) {
   switch (G) {
-    case 1: return launch_one<D, 1, LAYOUT>(p, grid, s, pdl);
-    case 2: return launch_one<D, 2, LAYOUT>(p, grid, s, pdl);
-    case 4: return launch_one<D, 4, LAYOUT>(p, grid, s, pdl);
-    case 8: return launch_one<D, 8, LAYOUT>(p, grid, s, pdl);
-    case 16: return launch_one<D, 16, LAYOUT>(p, grid, s, pdl);
+    case 1: return launch_g<D, 1, LAYOUT>(p, grid, s, pdl);
+    case 2: return launch_g<D, 2, LAYOUT>(p, grid, s, pdl);
+    case 4: return launch_g<D, 4, LAYOUT>(p, grid, s, pdl);
+    case 8: return launch_g<D, 8, LAYOUT>(p, grid, s, pdl);
+    case 16: return launch_g<D, 16, LAYOUT>(p, grid, s, pdl);
     default: return cudaErrorInvalidValue;
   }
 }

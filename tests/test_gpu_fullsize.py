@@ -38,7 +38,31 @@ def _topk_slots(score, budget):
 @pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
 @pytest.mark.parametrize("index,n_units,n_keys", [(1, 8, 48), (4, 4, 12), (2, 6, 24), (3, 6, 16)])
 def test_full_size_workload(index, n_units, n_keys, fused):
-    wl = workloads.workload(index)
+    _check_workload(workloads.workload(index), n_units, n_keys, fused, seed=index)
+
+
+# Caches large enough that every CTA of the score kernel scores 64 chunks or more, so
+# that it takes its tensor-core form, over the head sizes, group sizes and RoPE layouts
+# the 8B-shaped workloads do not cover (those take it at G = 8 and over 36 layers).
+TC_CASES = {
+    "d64_g2_interleaved": dict(L=4, B=1, Hq=16, Hkv=8, D=64, theta=1e4, seq_lens=[40000],
+                               rope_layout=workloads.INTERLEAVED),
+    "d128_g1": dict(L=4, B=1, Hq=8, Hkv=8, D=128, theta=1e6, seq_lens=[20000]),
+    "d64_g4_two_sequences": dict(L=2, B=2, Hq=32, Hkv=8, D=64, theta=1e4,
+                                 seq_lens=[30000, 25000]),
+    "d128_g2_interleaved_ragged": dict(L=2, B=3, Hq=16, Hkv=8, D=128, theta=1e6,
+                                       seq_lens=[20000, 15000, 9001],
+                                       rope_layout=workloads.INTERLEAVED),
+}
+
+
+@pytest.mark.parametrize("name", sorted(TC_CASES))
+def test_tensor_core_score_form(name):
+    wl = workloads.custom(name, budget=1024, offsets=range(1, 129), seed=77, **TC_CASES[name])
+    _check_workload(wl, 4, 12, False, seed=5)
+
+
+def _check_workload(wl, n_units, n_keys, fused, seed):
     data = workloads.generate(wl, device="cuda")
     stats_np = common.stats_fp32(data["q_calib"], wl.rope_layout)
     del data["q_calib"]
@@ -46,7 +70,7 @@ def test_full_size_workload(index, n_units, n_keys, fused):
     cache = tria.Cache.from_data(data)
     stats = tria.Stats(*[torch.from_numpy(s).cuda() for s in stats_np])
     ws = tria.workspace(cfg, cache)
-    units = workloads.sample_units(wl, n_units, seed=index)
+    units = workloads.sample_units(wl, n_units, seed=seed)
     starts = data["seq_start"]
     lens = data["seq_len"].cpu().tolist()
 
@@ -63,7 +87,7 @@ def test_full_size_workload(index, n_units, n_keys, fused):
     for (l, g, b) in units:
         s0, T = starts[b], lens[b]
         pristine[(l, g, b)] = tuple(data[n][l, g, s0:s0 + T].clone() for n in ("k", "v", "pos"))
-    rng = np.random.default_rng(index)
+    rng = np.random.default_rng(seed)
     G = wl.group
     for (l, g, b) in units:
         s0, T = starts[b], lens[b]

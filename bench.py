@@ -304,7 +304,7 @@ def _kernel_hash(names):
 
 
 KERNEL_SOURCES = {"prune_kernel": ("prune.cu", "score_math.cuh", "tria_internal.cuh"),
-                  "score_kernel": ("score.cu", "tria_internal.cuh"),
+                  "score_kernel": ("score.cu", "mma_sync.cuh", "tria_internal.cuh"),
                   "unit_kernel": ("unit.cu", "tria_internal.cuh")}
 
 

@@ -184,6 +184,10 @@ CASES = {
     "d64_interleaved": lambda: small("d64i", D=64, Hq=4, Hkv=2, seq_lens=[700], theta=1e4,
                                      rope_layout=workloads.INTERLEAVED),
     "g8": lambda: small("g8", Hq=8, Hkv=1, seq_lens=[515], budget=77),
+    # G = 8 always takes the score kernel's tensor-core form: D = 64, interleaved RoPE,
+    # two ragged sequences
+    "d64_g8_interleaved": lambda: small("d64g8i", D=64, Hq=16, Hkv=2, B=2, seq_lens=[700, 333],
+                                        theta=1e4, budget=60, rope_layout=workloads.INTERLEAVED),
     "d256": lambda: small("d256", D=256, Hq=4, Hkv=1, seq_lens=[300], budget=50),
     "g1": lambda: small("g1", Hq=4, Hkv=4, seq_lens=[260], budget=33),
     "g16_geometric": lambda: small("g16", D=64, Hq=16, Hkv=1, seq_lens=[200], budget=20,
@@ -356,7 +360,7 @@ def test_compact_rejects_malformed_selection():
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged2seq", "d64_interleaved", "g8", "two_layers",
-                                  "g16_geometric"])
+                                  "g16_geometric", "d64_g8_interleaved"])
 @pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
 def test_prune_matches_oracle(name, fused):
     case = Case(CASES[name](), fused=fused)

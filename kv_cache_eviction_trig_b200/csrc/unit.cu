@@ -257,9 +257,12 @@ __device__ __forceinline__ void stage_rows(const int32_t *src, int m, const uint
 
 }  // namespace
 
-template <int G, int CL>
+// MODE: the mode fixed at compile time (the prune step's own instantiation, so that its
+// code holds no other mode's branches), or -1 to read it from the parameters.
+template <int G, int CL, int MODE>
 __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_constant__ UnitParams p) {
   static_assert(CL == 1 || CL == kUnitCluster, "a unit is one CTA or one full cluster");
+  const int mode = MODE >= 0 ? MODE : p.mode;
   cg::cluster_group cl = cg::this_cluster();
   const int r = (int)cl.block_rank();
   const int64_t unit = blockIdx.x / CL;
@@ -292,12 +295,12 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
   // rounds; the first cluster barrier below makes every peer's clearing visible
   // before anyone counts into them
   for (int i = tid; i < kRounds * kSlice; i += nthr) (&c.slice[0][0])[i] = 0u;
-  const bool zmodes = p.mode == kModeZmax || p.mode == kModePrune;
+  const bool zmodes = mode == kModeZmax || mode == kModePrune;
   if (!zmodes) cl.sync();
   dev::pdl_wait();
 
   int kept = 0;
-  if (p.mode == kModeCompact) {
+  if (mode == kModeCompact) {
     // ------------------------------------------------------------ check the list
     const int64_t j0 = (int64_t)p.budget * r / CL, j1 = (int64_t)p.budget * (r + 1) / CL;
     int first_neg = p.budget, bad = 0;  // index of the first -1 (budget if none)
@@ -355,21 +358,21 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       if (r == 0 && tid == 0) dev::set_error(p.err, TRIA_DEVERR_SEQ_LEN);
       return;  // same decision in every CTA of the cluster
     }
-    const bool selects = (p.mode == kModeSelect || p.mode == kModePrune);
+    const bool selects = (mode == kModeSelect || mode == kModePrune);
     if (selects && !bud_ok) {
       if (r == 0 && tid == 0) dev::set_error(p.err, TRIA_DEVERR_BUDGET);
       return;
     }
     if (selects && T <= bud) {
       // sequence at or under budget: every slot is kept, nothing moves
-      if (p.mode == kModeSelect || p.write_short_sel) {
+      if (mode == kModeSelect || p.write_short_sel) {
         const int64_t j0 = (int64_t)p.budget * r / CL, j1 = (int64_t)p.budget * (r + 1) / CL;
         for (int64_t j = j0 + tid; j < j1; j += nthr) sel[j] = j < T ? (int32_t)j : -1;
       }
       return;
     }
     // held back by the prune window: the unit is left as it is
-    if (p.mode == kModePrune && (int64_t)T < (int64_t)bud + (p.window > 1 ? p.window : 1)) return;
+    if (mode == kModePrune && (int64_t)T < (int64_t)bud + (p.window > 1 ? p.window : 1)) return;
     if (T == 0) return;
     const int64_t lo = (int64_t)T * r / CL, hi = (int64_t)T * (r + 1) / CL;
     const int n = (int)(hi - lo);
@@ -437,7 +440,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
             float zf = -3.0e38f;
 #pragma unroll
             for (int j = 0; j < G; ++j) zf = fmaxf(zf, ((v[u][j] - mh[j]) - ml[j]) * is[j]);
-            if (p.mode == kModeZmax) {
+            if (mode == kModeZmax) {
               score[i] = zf == 0.0f ? 0.0f : zf;
             } else {
               const uint32_t key = dev::order_key(zf);
@@ -455,7 +458,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
           zround(i0);
         }
       }
-      if (p.mode == kModeZmax) return;
+      if (mode == kModeZmax) return;
     } else {
       const float *score = p.score + row * p.cap + seg + lo;
       for (int i = tid; i < n; i += nthr) {
@@ -665,7 +668,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
     // of its keys equal to thr whose cluster-wide rank in slot order is < k_eq.
     // Destination share of each CTA when the unit is compacted in one batch.
     const int per = (bud + CL - 1) / CL;
-    const bool balanced_fit = p.mode == kModePrune &&
+    const bool balanced_fit = mode == kModePrune &&
                               per <= (int)min((size_t)kOwnRows, data_bytes / (2 * (size_t)ROW + 4));
     if (tid < 32) {
       // lane q < CL: peer q's keys equal to thr before it (eqb), the ones it keeps
@@ -748,7 +751,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
          j < bud + (int64_t)(p.budget - bud) * (r + 1) / CL; j += nthr)
       sel[j] = -1;
     cl.sync();  // selection lists complete and visible; peers' keys are no longer read
-    if (p.mode == kModeSelect) return;
+    if (mode == kModeSelect) return;
     if (balanced) {
       // ------------------------------------- one batch: this CTA's share of destinations
       const int j0 = r * per;
@@ -829,7 +832,9 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
 // (portable cluster size; 15 clusters are resident at once on a B200).
 template <int G, int CL>
 static void configure_unit() {
-  cudaFuncSetAttribute(unit_kernel<G, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaFuncSetAttribute(unit_kernel<G, CL, -1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       kUnitSmemLarge);
+  cudaFuncSetAttribute(unit_kernel<G, CL, kModePrune>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        kUnitSmemLarge);
 }
 
@@ -880,12 +885,22 @@ static cudaError_t launch_unit_cl(const UnitParams &p, int units, cudaStream_t s
   cfg.numAttrs = pdl ? 2 : 1;
   // the group size only shapes the z-score stage
   const int G = (p.mode == kModeZmax || p.mode == kModePrune) ? p.G : 1;
+  if (p.mode == kModePrune) {
+    switch (G) {
+      case 1: return cudaLaunchKernelEx(&cfg, unit_kernel<1, CL, kModePrune>, p);
+      case 2: return cudaLaunchKernelEx(&cfg, unit_kernel<2, CL, kModePrune>, p);
+      case 4: return cudaLaunchKernelEx(&cfg, unit_kernel<4, CL, kModePrune>, p);
+      case 8: return cudaLaunchKernelEx(&cfg, unit_kernel<8, CL, kModePrune>, p);
+      case 16: return cudaLaunchKernelEx(&cfg, unit_kernel<16, CL, kModePrune>, p);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (G) {
-    case 1: return cudaLaunchKernelEx(&cfg, unit_kernel<1, CL>, p);
-    case 2: return cudaLaunchKernelEx(&cfg, unit_kernel<2, CL>, p);
-    case 4: return cudaLaunchKernelEx(&cfg, unit_kernel<4, CL>, p);
-    case 8: return cudaLaunchKernelEx(&cfg, unit_kernel<8, CL>, p);
-    case 16: return cudaLaunchKernelEx(&cfg, unit_kernel<16, CL>, p);
+    case 1: return cudaLaunchKernelEx(&cfg, unit_kernel<1, CL, -1>, p);
+    case 2: return cudaLaunchKernelEx(&cfg, unit_kernel<2, CL, -1>, p);
+    case 4: return cudaLaunchKernelEx(&cfg, unit_kernel<4, CL, -1>, p);
+    case 8: return cudaLaunchKernelEx(&cfg, unit_kernel<8, CL, -1>, p);
+    case 16: return cudaLaunchKernelEx(&cfg, unit_kernel<16, CL, -1>, p);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -36,7 +36,10 @@ struct ScoreShape {
   static constexpr int F = D / 2;
   static constexpr int FP = F / 2;                                 // RoPE pair pairs
   static constexpr int KPT_D = 256 / D;                            // 16 KB chunks
-  static constexpr int KPT_G = G <= 2 ? 4 : (G == 4 ? 2 : 1);      // accumulator registers
+  // keys per lane: bounded by the FMA form's accumulator registers, except at G = 8 with
+  // D <= 128, which always takes the tensor-core form (64-key chunks: 276 against 349 us
+  // for 32-key chunks on 4 x 131072 keys)
+  static constexpr int KPT_G = G <= 2 ? 4 : (G == 4 ? 2 : (G == 8 && D <= 128 ? 2 : 1));
   static constexpr int KPT0 = KPT_D < KPT_G ? KPT_D : KPT_G;
   static constexpr int KPT = KPT0 < kScoreKptCap ? KPT0 : kScoreKptCap;  // keys per lane
   static constexpr int CH = 32 * KPT;                              // keys per chunk

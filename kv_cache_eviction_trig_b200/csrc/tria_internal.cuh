@@ -72,7 +72,8 @@ constexpr int kScoreRingBytes = 220 * 1024;  // shared memory for key chunks and
 #endif
 constexpr int kUnitThreads = TRIA_UNIT_THREADS;  // build-time tunable: 256, 512 or 1024
 constexpr int kUnitCluster = 8;
-constexpr int kUnitClustersAtOnce = 15;  // 8-CTA clusters of 200 KB resident at once on a B200
+constexpr int kUnitClustersAtOnce = 15;   // 8-CTA clusters of 200 KB resident at once on a B200
+constexpr int kUnit4ClustersAtOnce = 33;  // 4-CTA clusters of 200 KB resident at once on a B200
 constexpr int kUnitSmemLarge = 200 * 1024;  // one CTA per SM
 
 struct FoldParams {
@@ -140,7 +141,7 @@ struct UnitParams {
   int32_t mode;
   int32_t write_short_sel;  // prune: also write identity lists for seq_len <= budget
   int32_t smem_bytes;       // dynamic shared memory of the launch
-  int32_t cluster;          // CTAs per unit (1 or kUnitCluster)
+  int32_t cluster;          // CTAs per unit (1, 4 or kUnitCluster)
   int64_t seg_start[TRIA_MAX_BATCH + 1];
 };
 

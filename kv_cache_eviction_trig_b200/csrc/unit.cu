@@ -55,7 +55,9 @@ constexpr int kMaxCluster = 16;
 constexpr int kWarps = kUnitThreads / 32;
 static_assert(kWarps >= 1 && kWarps <= 32, "one lane per warp in the emit prefix");
 constexpr int kBins = 4096;                   // cluster-wide histogram bins
-constexpr int kSlice = kBins / kUnitCluster;  // bins each CTA of the cluster owns
+// A CTA's slices of the cluster histograms of the refinement rounds (12, 12 and 8 key bits),
+// stored back to back: kBins / CL, kBins / CL and 256 / CL bins; 2112 words at CL = 4.
+constexpr int kSliceWords = 2 * (kBins / 4) + 256 / 4;
 constexpr int kRounds = 3;                    // refinement rounds (12, 12, 8 key bits)
 constexpr int kCoarse = 64;                   // coarse bins of the first round (64 bins each)
 constexpr int kCandMax = 4096;                // bucket keys a CTA may gather
@@ -82,7 +84,7 @@ struct Ctl {
   uint32_t coarse[kCoarse];         // this CTA's first-round counts per coarse bin
   uint32_t gc[kUnitCluster][kCoarse];  // the cluster's coarse counts, then fine counts
   uint32_t lh[kLocalBins];          // histogram of the rounds inside a gathered bucket
-  uint32_t slice[kRounds][kSlice];  // this CTA's slice of the cluster histogram, per round
+  uint32_t slice[kSliceWords];      // this CTA's slices of the cluster histograms, per round
 };
 static_assert(sizeof(Ctl) <= kCtl, "control region too small");
 
@@ -261,7 +263,7 @@ __device__ __forceinline__ void stage_rows(const int32_t *src, int m, const uint
 // code holds no other mode's branches), or -1 to read it from the parameters.
 template <int G, int CL, int MODE>
 __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_constant__ UnitParams p) {
-  static_assert(CL == 1 || CL == kUnitCluster, "a unit is one CTA or one full cluster");
+  static_assert(CL == 1 || CL == 4 || CL == kUnitCluster, "a unit is one CTA or a cluster of 4 or 8");
   const int mode = MODE >= 0 ? MODE : p.mode;
   cg::cluster_group cl = cg::this_cluster();
   const int r = (int)cl.block_rank();
@@ -294,7 +296,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
   // prologue (overlaps the score kernel's tail): clear the histogram slices of all
   // rounds; the first cluster barrier below makes every peer's clearing visible
   // before anyone counts into them
-  for (int i = tid; i < kRounds * kSlice; i += nthr) (&c.slice[0][0])[i] = 0u;
+  for (int i = tid; i < kSliceWords; i += nthr) c.slice[i] = 0u;
   const bool zmodes = mode == kModeZmax || mode == kModePrune;
   if (!zmodes) cl.sync();
   dev::pdl_wait();
@@ -542,15 +544,15 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
         }
         __syncthreads();
       } else {
-        const int per_log2 = dbits - 3;  // bins per owner: nb / 8
+        const int per_log2 = dbits - (CL == 8 ? 3 : 2);  // bins per owner: nb / CL
         for (int i = tid; i < n; i += nthr) {
           const uint32_t key = zkey[i];
           if (in_bucket(key))
-            cluster_hist_add(cl, &c.slice[round][0], (key >> dshift) & (nb - 1), per_log2);
+            cluster_hist_add(cl, &c.slice[round * (kBins / CL)], (key >> dshift) & (nb - 1), per_log2);
         }
         cl.sync();  // every count of this round has landed
         for (int i = tid; i < nb; i += nthr)
-          tot[i] = cl.map_shared_rank(&c.slice[round][0], i >> per_log2)[i & ((1 << per_log2) - 1)];
+          tot[i] = cl.map_shared_rank(&c.slice[round * (kBins / CL)], i >> per_log2)[i & ((1 << per_log2) - 1)];
         __syncthreads();
       }
       int bin, above;
@@ -848,6 +850,11 @@ int unit_smem_bytes() {
     configure_unit<4, 1>();
     configure_unit<8, 1>();
     configure_unit<16, 1>();
+    configure_unit<1, 4>();
+    configure_unit<2, 4>();
+    configure_unit<4, 4>();
+    configure_unit<8, 4>();
+    configure_unit<16, 4>();
     configure_unit<1, kUnitCluster>();
     configure_unit<2, kUnitCluster>();
     configure_unit<4, kUnitCluster>();
@@ -861,10 +868,17 @@ int unit_smem_bytes() {
 int unit_cluster_size(int64_t units, int64_t max_segment) {
   // Few units: a cluster of CTAs per unit (latency).  Many units: one CTA per unit
   // (more units at once), when a CTA's shared memory holds a whole segment's keys:
-  // zkey + first-round histogram + gathered slots + a minimal bucket list.
+  // zkey + first-round histogram + gathered slots + a minimal bucket list.  Between
+  // the two (up to 33 units whose segments need more than one CTA): clusters of 4,
+  // which a B200 holds all at once where clusters of 8 would take several waves.
   const int64_t data = kUnitSmemLarge - kCtl;
-  const bool fits = 4 * ((max_segment + 3) & ~3ll) + 4ll * kBins + 4ll * kCandMax + 8ll * 256 <= data;
-  return (units > kUnitClustersAtOnce && fits) ? 1 : kUnitCluster;
+  auto fits = [&](int64_t keys) {
+    return 4 * ((keys + 3) & ~3ll) + 4ll * kBins + 4ll * kCandMax + 8ll * 256 <= data;
+  };
+  if (units <= kUnitClustersAtOnce) return kUnitCluster;
+  if (fits(max_segment)) return 1;
+  if (units <= kUnit4ClustersAtOnce && fits((max_segment + 3) / 4)) return 4;
+  return kUnitCluster;
 }
 
 template <int CL>
@@ -906,8 +920,9 @@ static cudaError_t launch_unit_cl(const UnitParams &p, int units, cudaStream_t s
 }
 
 cudaError_t launch_unit(const UnitParams &p, int units, cudaStream_t s, bool pdl) {
-  return p.cluster == 1 ? launch_unit_cl<1>(p, units, s, pdl)
-                        : launch_unit_cl<kUnitCluster>(p, units, s, pdl);
+  if (p.cluster == 1) return launch_unit_cl<1>(p, units, s, pdl);
+  if (p.cluster == 4) return launch_unit_cl<4>(p, units, s, pdl);
+  return launch_unit_cl<kUnitCluster>(p, units, s, pdl);
 }
 
 }  // namespace tria

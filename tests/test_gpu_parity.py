@@ -309,6 +309,32 @@ def test_compact_many_units_multi_batch(kind, L, D, budget, T):
     check_compacted(case, sel, [budget])
 
 
+def test_four_cta_clusters_select_and_compact_exactly():
+    """16 units whose segments (40000 and 36001 slots) do not fit one CTA: the unit kernel
+    takes clusters of 4 CTAs (all resident at once). Selection on given scores with exact
+    ties, then in-place compaction of a random selection, both against the oracle."""
+    wl = small("cl4", Hq=16, Hkv=8, B=2, seq_lens=[40000, 36001], budget=3000,
+               offsets=range(1, 5), n_calib=32)
+    case = Case(wl)
+    rng = np.random.default_rng(13)
+    score = rng.normal(size=(wl.num_layers, wl.n_kv_heads, wl.cap_total)).astype(np.float32)
+    score[..., ::7] = score[..., 3:4]          # many exact ties
+    score[..., 1::11] = 0.0
+    sel = torch.empty((wl.num_layers, wl.n_kv_heads, wl.batch, wl.budget), dtype=torch.int32,
+                      device="cuda")
+    tria.tria_select(case.cfg, case.cache, torch.from_numpy(score).cuda(), sel, case.ws)
+    ref = oracle.select(case.prob, score.astype(np.float64))
+    np.testing.assert_array_equal(sel.cpu().numpy(), ref)
+    csel = np.stack([np.stack([np.stack([_adversarial_sel("random", T, wl.budget, rng)
+                                         for T in case.lens]) for _ in range(wl.n_kv_heads)])
+                     for _ in range(wl.num_layers)])
+    tria.tria_compact(case.cfg, case.cache, torch.from_numpy(csel).cuda(), case.ws)
+    torch.cuda.synchronize()
+    assert tria.tria_get_device_error(case.ws) == 0
+    assert case.dev["seq_len"].cpu().tolist() == [wl.budget] * wl.batch
+    check_compacted(case, csel, [wl.budget] * wl.batch)
+
+
 @pytest.mark.parametrize("fused", [False, True], ids=["kernels3", "fused"])
 def test_prune_many_units_matches_oracle(fused):
     case = Case(small("prune-multi", L=2, Hq=32, Hkv=8, B=1, seq_lens=[4000], budget=3500,

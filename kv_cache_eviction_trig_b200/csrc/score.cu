@@ -21,7 +21,10 @@
 // time).  The folded weights of a unit (3 KB at D = 128, G = 4) are brought
 // into one of two shared-memory weight slots by a bulk copy when the producer
 // reaches the unit, and read as broadcasts.  No cross-lane reduction and no
-// synchronisation between consumer warps are needed.
+// synchronisation between consumer warps are needed.  For D <= 128 and G <= 8 a
+// second consumer form scores each 16-key block on the tensor cores instead (see
+// "tensor-core form" below); the launch takes it at G = 8, or when a CTA scores many
+// chunks.
 #include <cudaTypedefs.h>
 
 #include <mutex>

@@ -50,7 +50,7 @@ WsLayout ws_layout(const tria_config &cfg, const int64_t *seq_start, int64_t cap
   w.raw = o;      o = align_up(o + 4ull * cfg.num_layers * cfg.n_q_heads * (size_t)cap, 256);
   w.sel = o;      o = align_up(o + 4ull * units * cfg.budget, 256);
   w.partials = o;
-  o = align_up(o + 16ull * units * (size_t)w.max_slots * kScoreConsumerWarps * G, 256);
+  o = align_up(o + 16ull * units * (size_t)w.max_slots * kScoreMaxWarps * G, 256);
   size_t end = o;
   const PrunePlan pl = (cfg.flags & TRIA_FUSED_PRUNE) ? prune_plan(cfg, seq_start) : PrunePlan{};
   w.fused = pl.ok;
@@ -282,6 +282,7 @@ cudaError_t fill_score(ScoreParams &sp, const tria_config *cfg, const tria_cache
   if (sg.total > INT32_MAX - 64) return cudaErrorInvalidValue;  // excluded by check_key_rows
   sp.total_chunks = (int32_t)sg.total;
   sp.chunks_per_cta = sg.chunks_per_cta;
+  sp.tc = score_uses_tc(cfg->head_dim, cfg->n_q_heads / cfg->n_kv_heads, sg.chunks_per_cta) ? 1 : 0;
   if (sg.total == 0) return cudaSuccess;
   const int64_t rows = (int64_t)cfg->num_layers * cfg->n_kv_heads * c->cap_total;
   cudaError_t e = make_key_tensor_map(&sp.tmap, c->k, cfg->head_dim, rows, ch);
@@ -296,6 +297,7 @@ void link_unit_to_score(UnitParams &up, const ScoreParams &sp) {
   up.max_slots = sp.max_slots;
   up.chunks_per_cta = sp.chunks_per_cta > 0 ? sp.chunks_per_cta : 1;
   up.chunks_per_row = sp.chunks_per_row;
+  up.score_warps = sp.tc ? kScoreTcWarps : kScoreConsumerWarps;
   for (int b = 0; b <= TRIA_MAX_BATCH; ++b) up.chunk_prefix[b] = sp.chunk_prefix[b];
 }
 

@@ -49,12 +49,12 @@ struct ScoreShape {
   static constexpr int NBOX = D / 64;                              // 128-byte boxes per row
   static constexpr int BOXB = CH * 128;                            // bytes per box region
   static constexpr int CB = CH * 2 * D;                            // bytes per chunk
-  static constexpr int NW = kScoreConsumerWarps;
   static constexpr int WB = FP * G * 24;                           // weight bytes per unit
   static constexpr int NSLOT0 = (kScoreRingBytes - 2 * WB) / CB;
   static constexpr int NSLOT = NSLOT0 < 24 ? NSLOT0 : 24;
   static constexpr bool OK = (D == 64 || D == 128 || D == 256) &&
-                             (G == 1 || G == 2 || G == 4 || G == 8 || G == 16) && NSLOT > NW;
+                             (G == 1 || G == 2 || G == 4 || G == 8 || G == 16) && NSLOT > kScoreConsumerWarps;
+  static constexpr bool TC_OK = OK && NSLOT > kScoreTcWarps;  // the tensor-core form's consumers
   static constexpr size_t SMEM = 1024 + (size_t)NSLOT * CB + 2ull * WB + (size_t)NSLOT * 16 +
                                  2ull * NSLOT * 8 + 2ull * 8 + 4ull * TRIA_MAX_BATCH + 32 * 20;
 };
@@ -279,10 +279,11 @@ __device__ __forceinline__ void tc_block(uint32_t cs, int mb, int lane,
 }
 
 template <int D, int G, int LAYOUT, bool TCF>
-__global__ void __launch_bounds__(kScoreThreads, 1)
+__global__ void __launch_bounds__(((TCF ? kScoreTcWarps : kScoreConsumerWarps) + 1) * 32, 1)
     score_kernel(const __grid_constant__ ScoreParams p) {
   using S = ScoreShape<D, G>;
-  constexpr int F = S::F, FP = S::FP, KPT = S::KPT, CH = S::CH, CB = S::CB, NW = S::NW;
+  constexpr int F = S::F, FP = S::FP, KPT = S::KPT, CH = S::CH, CB = S::CB;
+  constexpr int NW = TCF ? kScoreTcWarps : kScoreConsumerWarps;  // consumer warps
   constexpr int NSLOT = S::NSLOT;
 
   constexpr int WB = S::WB;
@@ -708,7 +709,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 template <int D, int G, int LAYOUT, bool TCF>
 static cudaError_t launch_one(const ScoreParams &p, int grid, cudaStream_t s, bool pdl) {
   using S = ScoreShape<D, G>;
-  if constexpr (!S::OK) {
+  if constexpr (!S::OK || (TCF && !S::TC_OK)) {
     return cudaErrorInvalidValue;
   } else {
     auto kern = score_kernel<D, G, LAYOUT, TCF>;
@@ -723,7 +724,7 @@ static cudaError_t launch_one(const ScoreParams &p, int grid, cudaStream_t s, bo
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
-    cfg.blockDim = dim3(kScoreThreads, 1, 1);
+    cfg.blockDim = dim3(((TCF ? kScoreTcWarps : kScoreConsumerWarps) + 1) * 32, 1, 1);
     cfg.dynamicSmemBytes = S::SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr;
@@ -741,11 +742,17 @@ static cudaError_t launch_one(const ScoreParams &p, int grid, cudaStream_t s, bo
 // against 28.8 us; 36 layers, about 1000 per CTA: 488 against 457 us).
 constexpr int kScoreTcChunks = 64;
 
+bool score_uses_tc(int D, int G, int chunks_per_cta) {
+  return (D == 64 || D == 128) && (G == 1 || G == 2 || G == 4 || G == 8) &&
+         (G == 8 || chunks_per_cta >= kScoreTcChunks);
+}
+
 template <int D, int G, int LAYOUT>
 static cudaError_t launch_g(const ScoreParams &p, int grid, cudaStream_t s, bool pdl) {
   if constexpr ((D == 64 || D == 128) && G <= 8) {
-    if (G == 8 || p.chunks_per_cta >= kScoreTcChunks) return launch_one<D, G, LAYOUT, true>(p, grid, s, pdl);
+    if (p.tc) return launch_one<D, G, LAYOUT, true>(p, grid, s, pdl);
   }
+  if (p.tc) return cudaErrorInvalidValue;  // the tensor-core form does not take this shape
   return launch_one<D, G, LAYOUT, false>(p, grid, s, pdl);
 }
 

@@ -58,13 +58,19 @@ ScoreGrid score_grid(const tria_config &cfg, const int64_t *seq_start);
 #ifndef TRIA_SCORE_KPT_CAP
 #define TRIA_SCORE_KPT_CAP 4
 #endif
-constexpr int kScoreConsumerWarps = TRIA_SCORE_WARPS;  // build-time tunables
+#ifndef TRIA_SCORE_TC_WARPS
+#define TRIA_SCORE_TC_WARPS 10
+#endif
+constexpr int kScoreConsumerWarps = TRIA_SCORE_WARPS;  // build-time tunables: consumer warps of
+constexpr int kScoreTcWarps = TRIA_SCORE_TC_WARPS;     // the FMA form and of the tensor-core form
+// the larger of the two: sizes the workspace for the score kernel's partial sums, which
+// hold one entry per (unit, CTA slot, consumer warp) of the form that ran
+constexpr int kScoreMaxWarps = kScoreConsumerWarps > kScoreTcWarps ? kScoreConsumerWarps : kScoreTcWarps;
 constexpr int kScoreKptCap = TRIA_SCORE_KPT_CAP;
 #ifndef TRIA_SCORE_JU
 #define TRIA_SCORE_JU 4
 #endif
 constexpr int kScoreJu = TRIA_SCORE_JU;  // pairs of RoPE pairs per inner iteration: 1, 2 or 4
-constexpr int kScoreThreads = (kScoreConsumerWarps + 1) * 32;
 constexpr int kScoreRingBytes = 220 * 1024;  // shared memory for key chunks and weights
 
 #ifndef TRIA_UNIT_THREADS
@@ -101,6 +107,7 @@ struct alignas(64) ScoreParams {
   const int32_t *seq_len;   // [B] caller's live lengths (not modified during the call)
   const int32_t *unit_len;  // [U] per-unit live lengths instead, or null
   const int32_t *head_budget;  // [L*Hkv] per-head budgets (with skip_short), or null
+  int32_t tc;               // 1: the tensor-core form (kScoreTcWarps consumer warps)
   int32_t budget, window;   // with skip_short: units shorter than budget + max(window, 1) are skipped
   float *raw;               // [L][Hq][cap]
   double *partials;         // per (unit, slot, warp): float64 sums of s and s^2 per head
@@ -126,6 +133,7 @@ struct UnitParams {
   const float *raw;         // [L][Hq][cap]      (zmax, prune)
   const double *partials;   // the score kernel's per-(unit, slot, warp) sums (zmax, prune)
   int32_t max_slots, chunks_per_cta, chunks_per_row;
+  int32_t score_warps;      // consumer warps the score kernel ran with (entries per slot)
   int32_t chunk_prefix[TRIA_MAX_BATCH + 1];
   float *score;             // [L][Hkv][cap]     (zmax writes, select reads)
   int32_t *sel;             // [L][Hkv][B][budget]
@@ -219,6 +227,8 @@ cudaError_t launch_fold(const FoldParams &p, cudaStream_t s);
 cudaError_t launch_score(const ScoreParams &p, int D, int G, int layout, int grid,
                          cudaStream_t s, bool pdl);
 bool score_supported(int D, int G, int layout);
+// Whether the score kernel takes its tensor-core form for this shape and chunk run.
+bool score_uses_tc(int D, int G, int chunks_per_cta);
 int score_chunk_keys(int D, int G);
 // Encodes the tensor map of the key cache viewed as [rows][D] bf16.
 cudaError_t make_key_tensor_map(CUtensorMap *map, const void *k, int D, int64_t rows,

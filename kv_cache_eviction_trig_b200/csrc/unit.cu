@@ -345,8 +345,8 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_kernel(const __grid_cons
       const int64_t first = (int64_t)row * p.chunks_per_row + p.chunk_prefix[b];
       const int nch = p.chunk_prefix[b + 1] - p.chunk_prefix[b];
       const int slots = nch > 0 ? (int)((first + nch - 1) / p.chunks_per_cta - first / p.chunks_per_cta) + 1 : 0;
-      const int entries = slots * kScoreConsumerWarps;
-      const double *pu = p.partials + unit * (int64_t)p.max_slots * kScoreConsumerWarps * (2 * G);
+      const int entries = slots * p.score_warps;
+      const double *pu = p.partials + unit * (int64_t)p.max_slots * p.score_warps * (2 * G);
       const int warp = tid >> 5, lane = tid & 31;
       for (int col = warp; col < 2 * G; col += kWarps) {
         double a = 0.0;

@@ -59,7 +59,7 @@ ScoreGrid score_grid(const tria_config &cfg, const int64_t *seq_start);
 #define TRIA_SCORE_KPT_CAP 4
 #endif
 #ifndef TRIA_SCORE_TC_WARPS
-#define TRIA_SCORE_TC_WARPS 10
+#define TRIA_SCORE_TC_WARPS 11
 #endif
 constexpr int kScoreConsumerWarps = TRIA_SCORE_WARPS;  // build-time tunables: consumer warps of
 constexpr int kScoreTcWarps = TRIA_SCORE_TC_WARPS;     // the FMA form and of the tensor-core form

@@ -128,7 +128,19 @@ def _check_workload(wl, n_units, n_keys, fused, seed):
     for (l, g, b), gs in host_k.items():
         s0, T = starts[b], lens[b]
         got = sel[l, g, b].cpu().numpy()
-        assert np.array_equal(got, _topk_slots(gs, wl.budget))
+        want = _topk_slots(gs, wl.budget)
+        if fused:
+            # the single launch scores with its own float32 arithmetic: keys within the
+            # parity tolerance of the threshold may order differently (never others)
+            diff = set(got.tolist()) ^ set(want.tolist())
+            if diff:
+                thr = np.sort(gs)[::-1][wl.budget - 1]
+                gr = raw[l, g * G:(g + 1) * G, s0:s0 + T].double().cpu().numpy()
+                f = max(1.0, max(np.sqrt(np.mean(r ** 2)) / r.std() for r in gr if r.std() > 0))
+                tol = 1e-4 * (2.0 + abs(thr)) * f
+                assert all(abs(gs[t] - thr) <= tol for t in diff), (l, g, b, len(diff))
+        else:
+            assert np.array_equal(got, want)
         idx = torch.from_numpy(got.astype(np.int64)).cuda()
         pk, pv, pp = pristine[(l, g, b)]
         n = wl.budget

@@ -7,8 +7,10 @@ properties that hold at any size:
   * the group score equals max_h (s_h - mean) / std computed in float64 on
     the host from the GPU's raw scores of the whole unit;
   * the prune keeps exactly the top-`budget` of those scores (ties to the
-    lower slot), in ascending order, and the compacted K/V/pos rows are
-    bit-identical to the pristine rows at the kept slots.
+    lower slot), in ascending order (the single launch, which scores with its
+    own float32 arithmetic, up to keys within the parity tolerance of the
+    threshold), and the compacted K/V/pos rows are bit-identical to the
+    pristine rows at the kept slots.
 """
 import numpy as np
 import pytest
